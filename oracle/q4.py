@@ -1,0 +1,224 @@
+"""fp64 definitions: unpack, dequantize, contract, bound.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  Sources, by page:
+
+* onnx-genai PR #1000 (cp.async re-test of the int4 MatMulNBits M=1 decode
+  GEMV), section "What it does": the int4 blockwise format with fp16 scales
+  and per-column fp32 accumulation.  The byte layout is not printed there; the
+  reading taken is the plain row-major MatMulNBits one (codes [N][K/2], two
+  per byte, low nibble = even k; scales [N][K/bs] fp16; zero-points packed
+  two per byte, low nibble = even block; no zero-point array means z = 8) and
+  w = (q - z)·s.
+* minfer doc 62 "r59 — q4_K W_dsc plane", §2.1 (the per-chunk coefficients
+  d·sc and -dmin·m), §2.2 (the chunk-major float2 plane and its size), §2.3
+  (bit-identity rules), §3.2 (super-block byte offsets and the 6-bit
+  scale/min unpacking rule).
+* AstrAI commit log (astrai/extension/backend), the uint4-anchoring bullet:
+  the bf16 GEMV is defined for any K >= 1 and any 2-byte storage offset.
+
+Readings where the pages are silent are listed in the design notes; the one
+that matters for values is the order of the 128 q4_K code bytes (``q4k_codes``).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+QK_K = 256            # weights per q4_K super-block
+Q4K_BLOCK_BYTES = 144  # 2 (d) + 2 (dmin) + 12 (scales/mins) + 128 (codes)
+Q4K_CHUNK = 32        # weights sharing one (scale, min) pair
+
+
+# --------------------------------------------------------------------------
+# shared little helpers (value conversions only)
+# --------------------------------------------------------------------------
+
+def f16_bits_to_f64(bits) -> np.ndarray:
+    """IEEE binary16 bit patterns -> float64 (exact widening)."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact: bf16 is the top half of a binary32)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def exact_in_f32(w: np.ndarray) -> bool:
+    """True when every float64 value survives a round trip through float32."""
+    w = np.asarray(w, dtype=np.float64)
+    return bool(np.all(w.astype(np.float32).astype(np.float64) == w))
+
+
+# --------------------------------------------------------------------------
+# int4 MatMulNBits-style blockwise (onnx-genai PR #1000, "What it does")
+# --------------------------------------------------------------------------
+
+def int4_codes(w_packed, N: int, K: int) -> np.ndarray:
+    """Unpack the 4-bit codes q[n, k] in 0..15 from [N][K/2] bytes, low nibble first."""
+    if K % 2:
+        raise ValueError("int4 K must be even")
+    b = np.asarray(w_packed, dtype=np.uint8).reshape(N, K // 2)
+    q = np.empty((N, K), dtype=np.int64)
+    q[:, 0::2] = b & 0x0F
+    q[:, 1::2] = b >> 4
+    return q
+
+
+def int4_zero_points(zeros, N: int, n_blocks: int) -> np.ndarray:
+    """Zero-points z[n, b]: uint4 packed two per byte (low nibble = even block); None means 8."""
+    if zeros is None:
+        return np.full((N, n_blocks), 8, dtype=np.int64)
+    per_row = (n_blocks + 1) // 2
+    b = np.asarray(zeros, dtype=np.uint8).reshape(N, per_row)
+    z = np.empty((N, 2 * per_row), dtype=np.int64)
+    z[:, 0::2] = b & 0x0F
+    z[:, 1::2] = b >> 4
+    return z[:, :n_blocks]
+
+
+def dequant_int4(w_packed, scales, zeros, N: int, K: int, block_size: int) -> np.ndarray:
+    """W[n, k] = (q[n,k] - z[n, k//bs]) · s[n, k//bs] in float64 (exact)."""
+    if block_size <= 0 or K % block_size:
+        raise ValueError("K must be a positive multiple of block_size")
+    nb = K // block_size
+    q = int4_codes(w_packed, N, K)
+    s = f16_bits_to_f64(np.asarray(scales).view(np.uint16).reshape(N, nb))
+    z = int4_zero_points(zeros, N, nb)
+    blk = np.arange(K) // block_size
+    return (q - z[:, blk]).astype(np.float64) * s[:, blk]
+
+
+# --------------------------------------------------------------------------
+# q4_K super-blocks (minfer doc 62, §2.1, §2.2, §3.2)
+# --------------------------------------------------------------------------
+
+def q4k_fields(raw, N: int, K: int):
+    """Split [N][K/256][144] bytes into (d, dmin, sc12, qs) with d, dmin as float64.
+
+    Byte offsets per super-block (§3.2): fp16 d at 0..1, fp16 dmin at 2..3
+    (little-endian), 12 packed scale/min bytes at 4..15, 128 code bytes at 16..143.
+    """
+    if K % QK_K:
+        raise ValueError("q4_K needs K % 256 == 0")
+    blk = np.asarray(raw, dtype=np.uint8).reshape(N, K // QK_K, Q4K_BLOCK_BYTES)
+    d_bits = blk[..., 0].astype(np.uint16) | (blk[..., 1].astype(np.uint16) << 8)
+    m_bits = blk[..., 2].astype(np.uint16) | (blk[..., 3].astype(np.uint16) << 8)
+    return f16_bits_to_f64(d_bits), f16_bits_to_f64(m_bits), blk[..., 4:16], blk[..., 16:144]
+
+
+def get_scale_min_k4(j: int, sc12) -> tuple:
+    """6-bit (scale, min) of chunk j (0..7) from the 12 packed bytes (§2.1, §3.2).
+
+    Chunks 0..3 keep their scale in the low 6 bits of byte j and their min in
+    the low 6 bits of byte j+4.  Chunks 4..7 combine a low nibble of byte j+4
+    (scale) or its high nibble (min) with the two top bits of byte j-4
+    (scale) or byte j (min) as bits 4..5.  Works elementwise on arrays whose
+    last axis holds the 12 bytes.
+    """
+    b = np.asarray(sc12).astype(np.int64)
+    if j < 4:
+        return b[..., j] & 63, b[..., j + 4] & 63
+    scale = (b[..., j + 4] & 0x0F) | ((b[..., j - 4] >> 6) << 4)
+    mn = (b[..., j + 4] >> 4) | ((b[..., j] >> 6) << 4)
+    return scale, mn
+
+
+def q4k_scales_mins(sc12):
+    """All eight (scale, min) pairs: two int arrays with a trailing axis of 8."""
+    pairs = [get_scale_min_k4(j, sc12) for j in range(8)]
+    return (np.stack([p[0] for p in pairs], axis=-1), np.stack([p[1] for p in pairs], axis=-1))
+
+
+def q4k_codes(qs) -> np.ndarray:
+    """Codes q[..., e] for the 256 elements of a super-block from its 128 code bytes.
+
+    Reading (the pages only say "128 B of 4-bit q" in 32-element chunks): the
+    llama.cpp grouping.  Code bytes come in four runs of 32; run p holds chunk
+    2p in its low nibbles and chunk 2p+1 in its high nibbles, element i of
+    each chunk in byte i of the run.
+    """
+    b = np.asarray(qs, dtype=np.uint8).astype(np.int64)
+    out = np.empty(b.shape[:-1] + (QK_K,), dtype=np.int64)
+    for p in range(4):
+        run = b[..., 32 * p:32 * p + 32]
+        out[..., 64 * p:64 * p + 32] = run & 0x0F
+        out[..., 64 * p + 32:64 * p + 64] = run >> 4
+    return out
+
+
+def dequant_q4k(raw, N: int, K: int) -> np.ndarray:
+    """W[n, k] = d·sc_c·q − dmin·m_c in float64, c = the 32-element chunk of k (§2.1)."""
+    d, dmin, sc12, qs = q4k_fields(raw, N, K)
+    sc, mn = q4k_scales_mins(sc12)                     # [N, nsb, 8]
+    q = q4k_codes(qs)                                  # [N, nsb, 256]
+    chunk = np.arange(QK_K) // Q4K_CHUNK               # chunk of each element
+    scale = d[..., None] * sc[..., chunk]              # d·sc   (exact in fp64)
+    offset = dmin[..., None] * mn[..., chunk]          # dmin·m (exact in fp64)
+    w = scale * q - offset
+    return w.reshape(N, K)
+
+
+def q4k_plane(raw, N: int, K: int) -> np.ndarray:
+    """The chunk-major W_dsc plane as float32 [K/32, N, 2] (§2.2, §2.3).
+
+    Entry (c, n) = (fp32(d)·fp32(sc), −(fp32(dmin)·fp32(m))) for global chunk
+    c = 8·superblock + j of row n: one IEEE binary32 multiply each (numpy
+    float32 multiply, no contraction) and an exact negation.  Flattened, entry
+    (c, n) sits at byte offset (c·N + n)·8, so the plane is N·K/4 bytes.
+    """
+    d, dmin, sc12, _ = q4k_fields(raw, N, K)
+    sc, mn = q4k_scales_mins(sc12)                     # [N, nsb, 8]
+    d32 = d.astype(np.float32)
+    m32 = dmin.astype(np.float32)
+    px = d32[..., None] * sc.astype(np.float32)        # [N, nsb, 8]
+    py = -(m32[..., None] * mn.astype(np.float32))
+    plane = np.empty((K // Q4K_CHUNK, N, 2), dtype=np.float32)
+    plane[:, :, 0] = px.reshape(N, K // Q4K_CHUNK).T
+    plane[:, :, 1] = py.reshape(N, K // Q4K_CHUNK).T
+    return plane
+
+
+def dequant_q4k_from_plane(raw, plane, N: int, K: int) -> np.ndarray:
+    """W[n, k] = P.x·q + P.y with P the plane entry of k's chunk, in float64."""
+    _, _, _, qs = q4k_fields(raw, N, K)
+    q = q4k_codes(qs).reshape(N, K).astype(np.float64)
+    P = np.asarray(plane, dtype=np.float32).reshape(K // Q4K_CHUNK, N, 2).astype(np.float64)
+    chunk = np.arange(K) // Q4K_CHUNK
+    return P[chunk, :, 0].T * q + P[chunk, :, 1].T
+
+
+# --------------------------------------------------------------------------
+# bf16 (AstrAI commit log, uint4-anchoring bullet: any K, any 2-byte offset)
+# --------------------------------------------------------------------------
+
+def dequant_bf16(w_bits, N: int, K: int, offset: int = 0) -> np.ndarray:
+    """W[n, k] from bf16 bits stored row-major with row stride K, `offset` elements in."""
+    flat = np.asarray(w_bits, dtype=np.uint16).reshape(-1)
+    return bf16_bits_to_f64(flat[offset:offset + N * K]).reshape(N, K)
+
+
+# --------------------------------------------------------------------------
+# contraction, bound and acceptance
+# --------------------------------------------------------------------------
+
+def gemv(W, x) -> np.ndarray:
+    """y[m, n] = Σ_k W[n, k]·x[m, k] in float64 (x given as its stored values)."""
+    W = np.asarray(W, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    return x @ W.T
+
+
+def bound(W, x) -> np.ndarray:
+    """B[m, n] = Σ_k |W[n, k]·x[m, k]|, the scale of the acceptance test."""
+    return np.abs(np.asarray(x, dtype=np.float64)) @ np.abs(np.asarray(W, dtype=np.float64)).T
+
+
+def violations(y, y_ref, B, rel: float = 2e-3, abs_: float = 1e-3) -> np.ndarray:
+    """Boolean mask of elements with |y − y_ref| > rel·B + abs_."""
+    y = np.asarray(y, dtype=np.float64)
+    return ~(np.abs(y - y_ref) <= rel * B + abs_)
+
+
+def accept(y, y_ref, B, rel: float = 2e-3, abs_: float = 1e-3) -> bool:
+    """True iff every element satisfies |y − y_ref| ≤ rel·B + abs_ (NaN fails)."""
+    return not bool(np.any(violations(y, y_ref, B, rel, abs_)))

@@ -1,0 +1,359 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each pin takes a namespace ``o`` holding the oracle's functions, so the same
+pins run against the real oracle (tests/test_oracle_pins.py) and against
+deliberately broken copies of it (tests/test_oracle_mutants.py), which shows
+that a plausible mistake in the oracle fails at least one pin.
+
+Sources of truth used here: hand-worked golden fixtures under tests/golden/
+(each citing the page passage it follows), closed forms, the bijection of
+the 12-byte 6-bit packing, brute-force pure-Python loops on tiny inputs, and
+math.fsum for exact sums.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+from weight_only_quantized_q4_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _f16_bytes(v):
+    return list(np.array([v], dtype=np.float16).view(np.uint8))
+
+
+# ---------------------------------------------------------------- q4_K pins
+
+def pin_scale_min_golden(o):
+    """Hand-worked examples of the two-case 6-bit unpacking rule."""
+    for case in _golden("q4k_scale_min_k4.json")["cases"]:
+        sc12 = np.array(case["sc12"], dtype=np.uint8)
+        for j in range(8):
+            s, m = o.get_scale_min_k4(j, sc12)
+            assert int(s) == case["scales"][j], (j, int(s), case["scales"][j])
+            assert int(m) == case["mins"][j], (j, int(m), case["mins"][j])
+
+
+def _pack_scale_min(s, m):
+    """Inverse of the 6-bit rule, written from the bit positions it names.
+
+    scales 0..3 -> low 6 bits of bytes 0..3, their top 2 bits unused by them;
+    mins 0..3 -> low 6 bits of bytes 4..7;
+    scales 4..7 -> low nibble of bytes 8..11 and the top 2 bits of bytes 0..3;
+    mins 4..7 -> high nibble of bytes 8..11 and the top 2 bits of bytes 4..7.
+    """
+    b = [0] * 12
+    for j in range(4):
+        b[j] = (s[j] & 63) | ((s[j + 4] >> 4) << 6)
+        b[j + 4] = (m[j] & 63) | ((m[j + 4] >> 4) << 6)
+        b[j + 8] = (s[j + 4] & 15) | ((m[j + 4] & 15) << 4)
+    return b
+
+
+def pin_scale_min_bijection(o):
+    """The 12 bytes carry exactly 8 six-bit scales + 8 six-bit mins (96 bits, each once)."""
+    rng = np.random.default_rng(7)
+    for _ in range(300):
+        s = [int(v) for v in rng.integers(0, 64, 8)]
+        m = [int(v) for v in rng.integers(0, 64, 8)]
+        b = np.array(_pack_scale_min(s, m), dtype=np.uint8)
+        got = [o.get_scale_min_k4(j, b) for j in range(8)]
+        assert [int(g[0]) for g in got] == s
+        assert [int(g[1]) for g in got] == m
+    for _ in range(300):
+        b = [int(v) for v in rng.integers(0, 256, 12)]
+        got = [o.get_scale_min_k4(j, np.array(b, dtype=np.uint8)) for j in range(8)]
+        assert _pack_scale_min([int(g[0]) for g in got], [int(g[1]) for g in got]) == b
+
+
+def _hand_superblock():
+    g = _golden("q4k_superblock_hand.json")
+    blk = np.zeros(144, dtype=np.uint8)
+    blk[0:2] = np.array([g["d_f16_bits"]], dtype=np.uint16).view(np.uint8)
+    blk[2:4] = np.array([g["dmin_f16_bits"]], dtype=np.uint16).view(np.uint8)
+    blk[4:16] = g["sc12"]
+    for k, v in g["qs_nonzero"].items():
+        blk[16 + int(k)] = v
+    return g, blk
+
+
+def pin_q4k_hand_superblock(o):
+    """A hand-built super-block with hand-worked dequantized values."""
+    g, blk = _hand_superblock()
+    W = o.dequant_q4k(blk.reshape(1, 1, 144), 1, 256)
+    for e, v in g["expect"].items():
+        assert W[0, int(e)] == v, (e, W[0, int(e)], v)
+
+
+def _brute_q4k(raw, N, K):
+    """Element-by-element q4_K dequantization in pure Python (tiny inputs only)."""
+    raw = np.asarray(raw, dtype=np.uint8).reshape(N, K // 256, 144)
+    out = np.zeros((N, K))
+    for n in range(N):
+        for sb in range(K // 256):
+            blk = [int(v) for v in raw[n, sb]]
+            d = float(np.array([blk[0] | (blk[1] << 8)], dtype=np.uint16).view(np.float16)[0])
+            dmin = float(np.array([blk[2] | (blk[3] << 8)], dtype=np.uint16).view(np.float16)[0])
+            sc = blk[4:16]
+            for e in range(256):
+                c = e // 32
+                if c < 4:
+                    s, m = sc[c] & 63, sc[c + 4] & 63
+                else:
+                    s = (sc[c + 4] & 15) | ((sc[c - 4] >> 6) << 4)
+                    m = (sc[c + 4] >> 4) | ((sc[c] >> 6) << 4)
+                run, i = divmod(e, 64)
+                byte = blk[16 + 32 * run + (i % 32)]
+                q = (byte & 15) if i < 32 else (byte >> 4)
+                out[n, 256 * sb + e] = d * s * q - dmin * m
+    return out
+
+
+def pin_q4k_brute(o):
+    """q4_K value = d·sc·q − dmin·m, element by element, on a 3×512 tensor."""
+    raw = synth.q4k_weights(3, 512, workload=901)
+    W = o.dequant_q4k(raw, 3, 512)
+    assert np.array_equal(W, _brute_q4k(raw, 3, 512))
+
+
+def pin_q4k_sc_zero(o):
+    """With all scales 0 every weight of a chunk is the constant −dmin·m."""
+    raw = synth.q4k_weights(2, 256, workload=902).copy()
+    s = [0] * 8
+    m = [1, 7, 13, 63, 2, 40, 5, 33]
+    raw[:, :, 4:16] = np.array(_pack_scale_min(s, m), dtype=np.uint8)
+    W = o.dequant_q4k(raw, 2, 256)
+    for n in range(2):
+        dmin = float(raw[n, 0, 2:4].view(np.float16)[0])
+        for c in range(8):
+            assert np.all(W[n, 32 * c:32 * c + 32] == -dmin * m[c])
+
+
+def pin_q4k_plane(o):
+    """Plane entries reproduce the products: P.x == d·sc, P.y == −dmin·m (exact),
+    P.x·q + P.y == W bitwise in fp32 and exactly in fp64, the plane is
+    chunk-major (entry (c, n) at flat index c·N + n) and N·K/4 bytes."""
+    N, K = 5, 768
+    raw = synth.q4k_weights(N, K, workload=903)
+    P = np.asarray(o.q4k_plane(raw, N, K))
+    assert P.dtype == np.float32 and P.nbytes == N * K // 4
+    flat = P.reshape(-1, 2)
+    for n in range(N):
+        for sb in range(K // 256):
+            blk = raw.reshape(N, K // 256, 144)[n, sb]
+            d = float(blk[0:2].view(np.float16)[0])
+            dmin = float(blk[2:4].view(np.float16)[0])
+            sc = [int(v) for v in blk[4:16]]
+            for j in range(8):
+                if j < 4:
+                    s, m = sc[j] & 63, sc[j + 4] & 63
+                else:
+                    s = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4)
+                    m = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4)
+                c = 8 * sb + j
+                assert float(flat[c * N + n, 0]) == d * s
+                assert float(flat[c * N + n, 1]) == -(dmin * m)
+    W = o.dequant_q4k(raw, N, K)
+    Wp = o.dequant_q4k_from_plane(raw, P, N, K)
+    assert np.array_equal(W, Wp)
+    assert np.array_equal(W.astype(np.float32), Wp.astype(np.float32))
+
+
+def pin_q4k_codes_layout(o):
+    """Code-byte order: a byte whose low nibble is l and high nibble h in run p
+    at position i gives element 64p+i = l and element 64p+32+i = h."""
+    qs = np.zeros(128, dtype=np.uint8)
+    rng = np.random.default_rng(11)
+    qs[:] = rng.integers(0, 256, 128)
+    q = o.q4k_codes(qs)
+    for p in range(4):
+        for i in range(32):
+            b = int(qs[32 * p + i])
+            assert q[64 * p + i] == (b & 15)
+            assert q[64 * p + 32 + i] == (b >> 4)
+
+
+# ---------------------------------------------------------------- int4 pins
+
+def _hand_int4(with_zeros):
+    g = _golden("int4_hand.json")
+    w = np.zeros((1, 16), dtype=np.uint8)
+    for k, v in g["w_bytes_nonzero"].items():
+        w[0, int(k)] = v
+    s = np.array([g["scales_f16"]], dtype=np.float16)
+    z = np.array([[g["zeros_byte"]]], dtype=np.uint8) if with_zeros else None
+    return g, w, s, z
+
+
+def pin_int4_hand(o):
+    """Hand-worked (q − z)·s values, with and without a zero-point array."""
+    for with_zeros, key in ((True, "expect_with_zeros"), (False, "expect_without_zeros")):
+        g, w, s, z = _hand_int4(with_zeros)
+        W = o.dequant_int4(w, s, z, 1, 32, 16)
+        for k, v in g[key].items():
+            assert W[0, int(k)] == v, (key, k, W[0, int(k)], v)
+
+
+def _brute_int4(w, s, z, N, K, bs):
+    out = np.zeros((N, K))
+    nb = K // bs
+    for n in range(N):
+        for k in range(K):
+            byte = int(w[n, k // 2])
+            q = (byte & 15) if k % 2 == 0 else (byte >> 4)
+            b = k // bs
+            if z is None:
+                zz = 8
+            else:
+                zb = int(z[n, b // 2])
+                zz = (zb & 15) if b % 2 == 0 else (zb >> 4)
+            out[n, k] = (q - zz) * float(s[n, b])
+    assert nb == s.shape[1]
+    return out
+
+
+def pin_int4_brute(o):
+    """(q − z)·s element by element, odd block count included (3 blocks of 32)."""
+    for with_zeros in (True, False):
+        t = synth.int4_weights(3, 96, 32, scale_lo=0.005, scale_hi=0.02,
+                               with_zeros=with_zeros, workload=904)
+        W = o.dequant_int4(t["w_packed"], t["scales"], t["zeros"], 3, 96, 32)
+        assert np.array_equal(W, _brute_int4(t["w_packed"], t["scales"], t["zeros"], 3, 96, 32))
+
+
+def pin_int4_zero_equals_code(o):
+    """z = q everywhere (every code equal to its block's zero-point) gives W ≡ 0, y ≡ 0."""
+    N, K, bs = 4, 64, 16
+    codes = np.random.default_rng(3).integers(0, 16, (N, K // bs))
+    w = np.zeros((N, K // 2), dtype=np.uint8)
+    z = np.zeros((N, K // bs // 2), dtype=np.uint8)
+    for n in range(N):
+        for b in range(K // bs):
+            c = int(codes[n, b])
+            for k in range(b * bs, (b + 1) * bs, 2):
+                w[n, k // 2] = c | (c << 4)
+            z[n, b // 2] |= c << (4 * (b % 2))
+    s = np.random.default_rng(4).uniform(0.01, 1.0, (N, K // bs)).astype(np.float16)
+    W = o.dequant_int4(w, s, z, N, K, bs)
+    assert np.all(W == 0)
+    x = synth.activations_f16(3, K, workload=905)
+    assert np.all(o.gemv(W, x) == 0)
+
+
+# ---------------------------------------------------------------- bf16 pins
+
+def pin_bf16_offsets_and_odd_k(o):
+    """bf16 for K ∈ {7, 12, 100, 1534} at offsets 0 and +1 element (2 bytes):
+    identical values, and y equal to a brute-force fsum loop."""
+    for K in (7, 12, 100, 1534):
+        N, M = 3, 2
+        wb = synth.bf16_weights_bits(N, K, workload=906)
+        xb = synth.activations_bf16_bits(M, K, workload=906)
+        ref = None
+        for off in (0, 1):
+            buf, _ = synth.with_element_offset(wb, off)
+            W = o.dequant_bf16(buf, N, K, offset=off)
+            if ref is None:
+                ref = W
+            assert np.array_equal(W, ref)
+        x = o.dequant_bf16(xb, M, K)
+        y = o.gemv(ref, x)
+        for m in range(M):
+            for n in range(N):
+                w_row = [float(np.array([int(wb[n, k]) << 16], dtype=np.uint32).view(np.float32)[0])
+                         for k in range(K)]
+                x_row = [float(np.array([int(xb[m, k]) << 16], dtype=np.uint32).view(np.float32)[0])
+                         for k in range(K)]
+                exact = math.fsum(a * b for a, b in zip(w_row, x_row))
+                assert abs(y[m, n] - exact) <= 1e-12 * math.fsum(abs(a * b) for a, b in zip(w_row, x_row)) + 1e-300
+
+
+# ------------------------------------------------------- contraction pins
+
+def pin_gemv_one_hot(o):
+    """x = e_k picks column k of W exactly."""
+    t = synth.int4_weights(6, 64, 32, scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=907)
+    W = o.dequant_int4(t["w_packed"], t["scales"], t["zeros"], 6, 64, 32)
+    for k in (0, 1, 31, 63):
+        x = np.zeros((1, 64))
+        x[0, k] = 1.0
+        assert np.array_equal(o.gemv(W, x)[0], W[:, k])
+
+
+def pin_gemv_constant(o):
+    """x ≡ 1 with a constant W gives y = K·w."""
+    K = 40
+    W = np.full((3, K), -1.375)
+    x = np.ones((2, K))
+    assert np.all(o.gemv(W, x) == K * -1.375)
+
+
+def pin_gemv_fsum(o):
+    """y equals a brute-force fsum of the products (to fp64 rounding) and the
+    bound equals the fsum of absolute products; x and W not transposed."""
+    rng = np.random.default_rng(12)
+    W = rng.standard_normal((4, 9))
+    x = rng.standard_normal((3, 9))
+    y = o.gemv(W, x)
+    B = o.bound(W, x)
+    assert y.shape == (3, 4) and B.shape == (3, 4)
+    for m in range(3):
+        for n in range(4):
+            exact = math.fsum(W[n, k] * x[m, k] for k in range(9))
+            absum = math.fsum(abs(W[n, k] * x[m, k]) for k in range(9))
+            assert abs(y[m, n] - exact) <= 1e-13 * absum
+            assert abs(B[m, n] - absum) <= 1e-13 * absum
+
+
+def pin_accept_threshold(o):
+    """The acceptance test passes at 0.99× the tolerance and fails at 1.01× and on NaN."""
+    for y0, b in ((1.0, 10.0), (-2.0, 3.0), (0.0, 0.0), (5.0, 1000.0)):
+        y_ref = np.array([[y0]])
+        B = np.array([[b]])
+        tol = 2e-3 * b + 1e-3
+        assert o.accept(y_ref + 0.99 * tol, y_ref, B)
+        assert o.accept(y_ref - 0.99 * tol, y_ref, B)
+        assert not o.accept(y_ref + 1.01 * tol, y_ref, B)
+        assert not o.accept(y_ref - 1.01 * tol, y_ref, B)
+    assert not o.accept(np.array([[np.nan]]), np.array([[0.0]]), np.array([[1.0]]))
+
+
+def pin_exact_in_f32(o):
+    """Dequantized weights of every workload distribution are exact fp32 values."""
+    t = synth.int4_weights(64, 1024, 32, scale_lo=0.005, scale_hi=0.02, with_zeros=False, workload=1)
+    assert o.exact_in_f32(o.dequant_int4(t["w_packed"], t["scales"], None, 64, 1024, 32))
+    t = synth.int4_weights(64, 1024, 128, scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=3)
+    assert o.exact_in_f32(o.dequant_int4(t["w_packed"], t["scales"], t["zeros"], 64, 1024, 128))
+    raw = synth.q4k_weights(64, 1024, workload=4)
+    assert o.exact_in_f32(o.dequant_q4k(raw, 64, 1024))
+    assert not o.exact_in_f32(np.array([1.0 + 2.0 ** -30]))
+
+
+ALL_PINS = [
+    pin_scale_min_golden,
+    pin_scale_min_bijection,
+    pin_q4k_hand_superblock,
+    pin_q4k_brute,
+    pin_q4k_sc_zero,
+    pin_q4k_plane,
+    pin_q4k_codes_layout,
+    pin_int4_hand,
+    pin_int4_brute,
+    pin_int4_zero_equals_code,
+    pin_bf16_offsets_and_odd_k,
+    pin_gemv_one_hot,
+    pin_gemv_constant,
+    pin_gemv_fsum,
+    pin_accept_threshold,
+    pin_exact_in_f32,
+]

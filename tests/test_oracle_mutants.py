@@ -1,0 +1,133 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+Every mutant is a small, realistic slip: a swapped nibble order, a wrong
+byte index in the 6-bit unpacking, a dropped or sign-flipped min term, a
+row-major plane, an operand read backwards, a missing absolute value.
+"""
+import numpy as np
+import pytest
+
+import oracle.q4 as oq
+from _pins import ALL_PINS
+
+_orig = {name: getattr(oq, name) for name in dir(oq) if not name.startswith("__")}
+
+
+def _int4_codes_high_first(w_packed, N, K):
+    b = np.asarray(w_packed, dtype=np.uint8).reshape(N, K // 2)
+    q = np.empty((N, K), dtype=np.int64)
+    q[:, 0::2] = b >> 4
+    q[:, 1::2] = b & 0x0F
+    return q
+
+
+def _zero_points_default_zero(zeros, N, n_blocks):
+    if zeros is None:
+        return np.zeros((N, n_blocks), dtype=np.int64)
+    return _orig["int4_zero_points"](zeros, N, n_blocks)
+
+
+def _scale_min_wrong_byte(j, sc12):
+    b = np.asarray(sc12).astype(np.int64)
+    if j < 4:
+        return b[..., j] & 63, b[..., j + 4] & 63
+    return ((b[..., j + 4] & 0x0F) | ((b[..., j - 4] >> 6) << 4),
+            (b[..., j + 4] >> 4) | ((b[..., j - 4] >> 6) << 4))  # min takes byte j-4
+
+
+def _scale_min_nibbles_swapped(j, sc12):
+    b = np.asarray(sc12).astype(np.int64)
+    if j < 4:
+        return b[..., j] & 63, b[..., j + 4] & 63
+    return ((b[..., j + 4] >> 4) | ((b[..., j - 4] >> 6) << 4),
+            (b[..., j + 4] & 0x0F) | ((b[..., j] >> 6) << 4))
+
+
+def _codes_sequential(qs):
+    b = np.asarray(qs, dtype=np.uint8).astype(np.int64)
+    out = np.empty(b.shape[:-1] + (256,), dtype=np.int64)
+    out[..., 0::2] = b & 15
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def _dequant_q4k_no_min(raw, N, K):
+    d, dmin, sc12, qs = oq.q4k_fields(raw, N, K)
+    sc, mn = oq.q4k_scales_mins(sc12)
+    q = oq.q4k_codes(qs)
+    chunk = np.arange(256) // 32
+    return (d[..., None] * sc[..., chunk] * q).reshape(N, K)
+
+
+def _dequant_q4k_plus_min(raw, N, K):
+    d, dmin, sc12, qs = oq.q4k_fields(raw, N, K)
+    sc, mn = oq.q4k_scales_mins(sc12)
+    q = oq.q4k_codes(qs)
+    chunk = np.arange(256) // 32
+    return (d[..., None] * sc[..., chunk] * q + dmin[..., None] * mn[..., chunk]).reshape(N, K)
+
+
+def _fields_d_dmin_swapped(raw, N, K):
+    d, dmin, sc12, qs = _orig["q4k_fields"](raw, N, K)
+    return dmin, d, sc12, qs
+
+
+def _plane_row_major(raw, N, K):
+    P = _orig["q4k_plane"](raw, N, K)                 # [K/32, N, 2]
+    return np.ascontiguousarray(P.transpose(1, 0, 2)).reshape(K // 32, N, 2)
+
+
+def _gemv_k_reversed(W, x):
+    return np.asarray(x, dtype=np.float64) @ np.asarray(W, dtype=np.float64)[:, ::-1].T
+
+
+def _bound_no_abs(W, x):
+    return np.asarray(x, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T
+
+
+def _accept_loose(y, y_ref, B, rel=2e-3, abs_=1e-3):
+    return _orig["accept"](y, y_ref, B, rel * 2, abs_)
+
+
+def _dequant_bf16_ignores_offset(w_bits, N, K, offset=0):
+    return _orig["dequant_bf16"](w_bits, N, K, 0)
+
+
+def _dequant_int4_block_off_by_one(w_packed, scales, zeros, N, K, block_size):
+    nb = K // block_size
+    q = oq.int4_codes(w_packed, N, K)
+    s = oq.f16_bits_to_f64(np.asarray(scales).view(np.uint16).reshape(N, nb))
+    z = oq.int4_zero_points(zeros, N, nb)
+    blk = np.minimum((np.arange(K) + 1) // block_size, nb - 1)
+    return (q - z[:, blk]).astype(np.float64) * s[:, blk]
+
+
+MUTANTS = {
+    "int4 nibbles high-first": ("int4_codes", _int4_codes_high_first),
+    "int4 default zero-point 0": ("int4_zero_points", _zero_points_default_zero),
+    "int4 block index off by one": ("dequant_int4", _dequant_int4_block_off_by_one),
+    "6-bit min from byte j-4": ("get_scale_min_k4", _scale_min_wrong_byte),
+    "6-bit nibbles swapped": ("get_scale_min_k4", _scale_min_nibbles_swapped),
+    "q4_K codes sequential": ("q4k_codes", _codes_sequential),
+    "q4_K min term dropped": ("dequant_q4k", _dequant_q4k_no_min),
+    "q4_K min term sign": ("dequant_q4k", _dequant_q4k_plus_min),
+    "q4_K d/dmin swapped": ("q4k_fields", _fields_d_dmin_swapped),
+    "plane row-major": ("q4k_plane", _plane_row_major),
+    "gemv k reversed": ("gemv", _gemv_k_reversed),
+    "bound without abs": ("bound", _bound_no_abs),
+    "acceptance twice as loose": ("accept", _accept_loose),
+    "bf16 offset ignored": ("dequant_bf16", _dequant_bf16_ignores_offset),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(oq, attr, fn)
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(oq)
+        except Exception:  # noqa: BLE001 - any failure of a pin counts as caught
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name!r} passed every pin"
