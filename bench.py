@@ -1,0 +1,491 @@
+#!/usr/bin/env python3
+"""Benchmark of the weight-only quantized decode GEMV on B200.
+
+One step = one call of the decode linear layer y = x·Wᵀ (the whole hot path:
+weight stream, unpack, dequantize, multiply-accumulate, reduce, epilogue)
+over one batch of synthetic activations.  The default workload is the int4
+MatMulNBits-style GEMV with block 128, uint4 zero-points, M = 1 and
+N×K = 4096×14336 (the 4096×14336-class shape); ``--workload`` picks another.
+
+Metric: achieved HBM GB/s (weight + scale + zero-point bytes ÷ device time)
+and µs per call.  Timing: CUDA graphs of back-to-back calls, each call on the
+next of R weight copies whose total exceeds 3× the L2, CUDA events on the
+launching stream, barrier + synchronize on both sides, max over ranks.
+
+``--impl reference`` times the CPU oracle (test infrastructure) on the host
+cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_only_quantized_q4_b200 import synth  # noqa: E402
+
+# ---------------------------------------------------------------- workloads
+
+
+def _int4(M, N, K, bs, zeros, workload, s_lo, s_hi):
+    return dict(fmt="int4", M=M, N=N, K=K, bs=bs, zeros=zeros, workload=workload, s_lo=s_lo, s_hi=s_hi)
+
+
+WORKLOADS = {
+    "int4_b128_zp_m1_4096x14336": _int4(1, 4096, 14336, 128, True, 3, 0.002, 0.01),
+    "int4_b128_zp_m4_4096x14336": _int4(4, 4096, 14336, 128, True, 3, 0.002, 0.01),
+    "int4_b128_zp_m1_14336x4096": _int4(1, 14336, 4096, 128, True, 3, 0.002, 0.01),
+    "int4_b128_zp_m4_14336x4096": _int4(4, 14336, 4096, 128, True, 3, 0.002, 0.01),
+    "int4_b128_zp_m1_4096x4096": _int4(1, 4096, 4096, 128, True, 3, 0.002, 0.01),
+    "int4_b32_m1_256x1024": _int4(1, 256, 1024, 32, False, 1, 0.005, 0.02),
+}
+for _M in (1, 2, 4, 8):
+    for _N, _K in ((4096, 4096), (11008, 4096), (4096, 11008)):
+        WORKLOADS[f"q4k_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=False, workload=4)
+        WORKLOADS[f"q4k_dsc_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=True, workload=4)
+for _M in (1, 3, 8):
+    for _N, _K in ((1536, 1536), (256, 1536), (1536, 6912), (151936, 1536)):
+        WORKLOADS[f"bf16_m{_M}_{_N}x{_K}"] = dict(fmt="bf16", M=_M, N=_N, K=_K, workload=2)
+for _M in (2, 4, 8):
+    WORKLOADS[f"int4_b128_zp_m{_M}_4096x14336"] = _int4(_M, 4096, 14336, 128, True, 3, 0.002, 0.01)
+
+DEFAULT_WORKLOAD = "int4_b128_zp_m1_4096x14336"
+SWEEP = ["int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
+         "int4_b32_m1_256x1024", "q4k_m1_4096x11008", "q4k_dsc_m1_4096x11008", "q4k_m4_11008x4096",
+         "q4k_m8_4096x4096", "bf16_m1_1536x6912", "bf16_m3_1536x6912", "bf16_m8_1536x6912", "bf16_m1_151936x1536"]
+
+
+def weight_bytes(w) -> int:
+    """Algorithmic bytes one call must read for the weights (x and y excluded)."""
+    N, K = w["N"], w["K"]
+    if w["fmt"] == "int4":
+        nb = K // w["bs"]
+        return N * K // 2 + 2 * N * nb + (N * ((nb + 1) // 2) if w["zeros"] else 0)
+    if w["fmt"] == "q4k":
+        return N * K // 2 + N * K // 4 if w["dsc"] else N * (K // 256) * 144
+    return 2 * N * K
+
+
+def dtype_of(w) -> str:
+    return {"int4": "int4xf16->f32", "q4k": "q4kxf16->f32", "bf16": "bf16xbf16->f32"}[w["fmt"]]
+
+
+def host_inputs(w):
+    """Seeded canonical arrays for one workload (numpy)."""
+    M, N, K = w["M"], w["N"], w["K"]
+    if w["fmt"] == "int4":
+        t = synth.int4_weights(N, K, w["bs"], scale_lo=w["s_lo"], scale_hi=w["s_hi"], with_zeros=w["zeros"],
+                               workload=w["workload"])
+        return dict(x=synth.activations_f16(M, K, workload=w["workload"]), **t)
+    if w["fmt"] == "q4k":
+        return dict(x=synth.activations_f16(M, K, workload=w["workload"]),
+                    raw=synth.q4k_weights(N, K, workload=w["workload"]))
+    return dict(x=synth.activations_bf16_bits(M, K, workload=w["workload"]),
+                w=synth.bf16_weights_bits(N, K, workload=w["workload"]))
+
+
+# ---------------------------------------------------------------- clocks (NVML, read-only)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- our arm
+
+
+class DeviceWorkload:
+    """Device buffers for one workload plus a callable that issues one call on copy i."""
+
+    def __init__(self, w, host, torch, wq, l2_bytes):
+        self.w, self.torch, self.wq = w, torch, wq
+        dev = torch.device("cuda", torch.cuda.current_device())
+        M, N, K = w["M"], w["N"], w["K"]
+        self.M, self.N, self.K = M, N, K
+        self.bytes = weight_bytes(w)
+        # enough weight copies that a round trip exceeds 3x L2
+        self.R = max(1, -(-3 * l2_bytes // max(self.bytes, 1)))
+        self.R = min(self.R, max(1, int(8e9 // max(self.bytes, 1))))
+        self.copies = []
+        if w["fmt"] == "int4":
+            base = [torch.from_numpy(host["w_packed"]).to(dev), torch.from_numpy(host["scales"]).to(dev),
+                    torch.from_numpy(host["zeros"]).to(dev) if host["zeros"] is not None else None]
+            for _ in range(self.R):
+                self.copies.append([t.clone() if t is not None else None for t in base])
+            self.x = torch.from_numpy(host["x"]).to(dev)
+            self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        elif w["fmt"] == "q4k":
+            raw = torch.from_numpy(host["raw"]).to(dev)
+            for _ in range(self.R):
+                c = [raw.clone()]
+                if w["dsc"]:
+                    P = torch.empty((K // 32, N, 2), dtype=torch.float32, device=dev)
+                    wq.wq_build_q4k_dsc_device(c[0], P, N, K)
+                    c.append(P)
+                self.copies.append(c)
+            self.x = torch.from_numpy(host["x"]).to(dev)
+            self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        else:
+            wt = torch.from_numpy(host["w"].view(np.int16)).to(dev).view(torch.bfloat16)
+            for _ in range(self.R):
+                self.copies.append([wt.clone()])
+            self.x = torch.from_numpy(host["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+            self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+
+    def call(self, i, x=None, y=None, stream=None):
+        c = self.copies[i % self.R]
+        x = self.x if x is None else x
+        y = self.y if y is None else y
+        w, wq = self.w, self.wq
+        if w["fmt"] == "int4":
+            wq.gemv_int4_blockwise(x, c[0], c[1], c[2], y, self.M, self.N, self.K, w["bs"], stream=stream)
+        elif w["fmt"] == "q4k":
+            if w["dsc"]:
+                wq.gemv_q4k_dsc(x, c[0], c[1], y, self.M, self.N, self.K, stream=stream)
+            else:
+                wq.gemv_q4k(x, c[0], y, self.M, self.N, self.K, stream=stream)
+        else:
+            wq.gemv_bf16(x, c[0], y, self.M, self.N, self.K, stream=stream)
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return 6650.0, "fallback"
+
+
+def _kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantized_q4_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t.get(workload)
+        if e and e.get("kernel_src_sha") == _kernel_src_hash():
+            return e.get("dram_bytes_per_launch")
+    except Exception:  # noqa: BLE001
+        pass
+    return None
+
+
+def run_ours(args, w, wname, rank, world, dist):
+    import torch
+
+    import weight_only_quantized_q4_b200 as wq
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    host = host_inputs(w)
+    d = DeviceWorkload(w, host, torch, wq, l2)
+    stream = torch.cuda.Stream()
+
+    # configure every kernel once outside capture, then capture a graph of G calls
+    with torch.cuda.stream(stream):
+        d.call(0, stream=stream)
+    torch.cuda.synchronize()
+    label = wq.last_kernel()
+    G = max(d.R, min(args.graph_calls, args.steps))
+    G = -(-G // d.R) * d.R
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(G):
+            d.call(i, stream=torch.cuda.current_stream())
+    # per-launch durations: events between consecutive calls in a second graph
+    n_ev = min(G, 256)
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev + 1)]
+    g_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ev, stream=stream):
+        cs = torch.cuda.current_stream()
+        for i in range(n_ev):
+            evs[i].record(cs)
+            d.call(i, stream=cs)
+        evs[n_ev].record(cs)
+
+    reps = max(1, -(-args.steps // G))
+    steps = reps * G
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        # per-launch timing pass (same clocks window)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g_ev.replay()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(n_ev)]
+    avg_launch_ms = float(np.mean(per_launch))
+
+    # e2e: pinned host x in, device GEMV, pinned host y out, every step, through the API
+    xh = torch.empty_like(d.x, device="cpu").pin_memory()
+    xh.copy_(d.x.cpu())
+    yh = torch.empty_like(d.y, device="cpu").pin_memory()
+    xd, yd = torch.empty_like(d.x), torch.empty_like(d.y)
+    Ge = min(G, 256)
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=stream):
+        cs = torch.cuda.current_stream()
+        for i in range(Ge):
+            xd.copy_(xh, non_blocking=True)
+            d.call(i, x=xd, y=yd, stream=cs)
+            yh.copy_(yd, non_blocking=True)
+    for _ in range(2):
+        ge.replay()
+    torch.cuda.synchronize()
+    reps_e = max(1, -(-min(args.steps, 20000) // Ge))
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps_e):
+            ge.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = t0.elapsed_time(t1)
+    steps_e2e = reps_e * Ge
+
+    if dist is not None:
+        t = torch.tensor([ms, ms_e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+
+    bytes_call = d.bytes
+    ms_step = ms / steps
+    value = world * bytes_call * steps / (ms * 1e-3) / 1e9
+    e2e_value = world * bytes_call * steps_e2e / (ms_e2e * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    achieved = bytes_call / (avg_launch_ms * 1e-3) / 1e9
+    out = {
+        "metric": "achieved HBM GB/s per quantized GEMV call (weight+scale bytes / device time)",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_step,
+        "us_per_call": round(ms_step * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": dtype_of(w),
+        "data": "synthetic (seeded; value distributions of the workload definition)",
+        "config": {"workload": wname, "fmt": w["fmt"], "M": w["M"], "N": w["N"], "K": w["K"],
+                   "weight_bytes_per_call": bytes_call, "weight_copies_rotated": d.R,
+                   "l2": f"inputs larger than L2: {d.R} rotating weight copies, {d.R * bytes_call / 1e6:.0f} MB "
+                         f">= 3x L2 ({l2 / 1e6:.0f} MB)",
+                   "timing": f"CUDA graph of {G} back-to-back calls replayed {reps}x, CUDA events on the stream",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "kernel": label},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(d.x.numel() * d.x.element_size()),
+                "d2h_bytes_per_step": int(d.y.numel() * d.y.element_size()),
+                "us_per_call": round(ms_e2e / steps_e2e * 1e3, 3),
+                "how": "per step: pinned x -> device, GEMV through the C ABI, y -> pinned host; graph-captured"},
+        "gpu_launches": steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": _traffic(wname),
+                     "peak_kind": f"{peak_kind} copy bandwidth", "avg_launch_us": round(avg_launch_ms * 1e3, 3)},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, host, budget_s=args.cpu_budget)
+    return out
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+
+
+def cpu_baseline(w, host, budget_s=15.0):
+    """Time the CPU oracle as it stands on a bounded row sample; scale to GB/s of weights."""
+    import oracle
+
+    N, K, M = w["N"], w["K"], w["M"]
+    rows = 8
+    done_rows, t_total = 0, 0.0
+    x = host["x"]
+    while t_total < budget_s and done_rows < N:
+        r = np.arange(done_rows, min(done_rows + rows, N))
+        t0 = time.perf_counter()
+        if w["fmt"] == "int4":
+            z = host["zeros"][r] if host["zeros"] is not None else None
+            W = oracle.dequant_int4(host["w_packed"][r], host["scales"][r], z, len(r), K, w["bs"])
+            xv = x.astype(np.float64)
+        elif w["fmt"] == "q4k":
+            if w["dsc"]:
+                P = oracle.q4k_plane(host["raw"][r], len(r), K)
+                W = oracle.dequant_q4k_from_plane(host["raw"][r], P, len(r), K)
+            else:
+                W = oracle.dequant_q4k(host["raw"][r], len(r), K)
+            xv = x.astype(np.float64)
+        else:
+            W = oracle.dequant_bf16(host["w"][r], len(r), K)
+            xv = oracle.dequant_bf16(x, M, K)
+        oracle.gemv(W, xv)
+        oracle.bound(W, xv)
+        t_total += time.perf_counter() - t0
+        done_rows += len(r)
+        rows = min(rows * 2, 4096)
+    frac = done_rows / N
+    bytes_done = weight_bytes(w) * frac
+    gbs = bytes_done / t_total / 1e9
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "us_per_call_equiv": round(t_total / frac * 1e6, 1),
+            "sample": f"{done_rows} of {N} rows ({100 * frac:.1f}%) of the workload, numpy fp64 dequant + GEMV + bound, "
+                      f"{t_total:.1f} s; threads as numpy/BLAS uses them"}
+
+
+def run_reference(args, w, wname):
+    host = host_inputs(w)
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_baseline(w, host, budget_s=0.5)
+    budget = max(1.0, min(args.cpu_budget, 120.0 / max(1, args.steps)))
+    vals = [cpu_baseline(w, host, budget_s=budget) for _ in range(max(1, min(args.steps, 8)))]
+    v = float(np.median([c["value"] for c in vals]))
+    cb = dict(vals[0])
+    cb["value"] = round(v, 4)
+    return {
+        "metric": "achieved HBM GB/s per quantized GEMV call (weight+scale bytes / device time)",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": 1, "steps": len(vals), "warmup": args.warmup,
+        "ms_per_step": float(np.median([c["us_per_call_equiv"] for c in vals])) / 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "impl": "reference",
+        "config": {"workload": wname, "fmt": w["fmt"], "M": w["M"], "N": w["N"], "K": w["K"]},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--sweep", action="store_true", help="one JSON line per workload of the sweep list")
+    ap.add_argument("--graph-calls", type=int, default=1000)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, WORKLOADS[args.workload], args.workload)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    names = SWEEP if args.sweep else [args.workload]
+    for name in names:
+        out = run_ours(args, WORKLOADS[name], name, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+/*
+ * wq.h — C ABI of libwq.so: weight-only quantized decode linear layer
+ * y = x·Wᵀ for B200 (sm_100a), with W dequantized on the fly.
+ *
+ * Shapes: x is [M, K] row-major, W is logically [N, K], y is [M, N] row-major.
+ * M is the decode batch (the GEMV family serves M = 1..8; M >= 9 runs the
+ * tensor-core dequant-then-MMA family), N the output features, K the input
+ * features.  Every floating-point result is accumulated in fp32.
+ *
+ * Conventions for every entry point below:
+ *  - Pointers named *_host are host pointers; every other pointer is a CUDA
+ *    device pointer owned by the caller.  The library never frees, keeps or
+ *    allocates memory on these paths, and it has no CPU fallback.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Launch entry points are asynchronous on that stream; they return after
+ *    enqueueing.  Argument errors are reported before anything is enqueued.
+ *  - Return value: WQ_OK (0) or a negative WQ_ERR_* code.  wq_last_error()
+ *    then holds a one-line message (per calling thread).
+ *  - wq_last_kernel() names the kernel variant the last successful launch on
+ *    the calling thread used (a liveness label such as
+ *    "int4.gemv.cc.m1.b128"), so a test can assert which path ran.
+ *
+ * Weight formats (canonical byte layouts, layout version WQ_LAYOUT_CANONICAL):
+ *  - int4 MatMulNBits-style blocks (onnx-genai PR #1000, "What it does": int4
+ *    blockwise weights with fp16 scales and zero-points).  w_packed is
+ *    [N][K/2] bytes, two 4-bit codes per byte, low nibble = even k.  scales
+ *    is [N][K/block_size] fp16.  zeros is [N][ceil((K/block_size)/2)] bytes,
+ *    two uint4 zero-points per byte, low nibble = even block; NULL means
+ *    z = 8 for every block.  w = (q - z)·s.
+ *  - q4_K super-blocks (minfer doc 62 "r59 — q4_K W_dsc plane", §3.2): row n
+ *    holds K/256 blocks of 144 bytes: fp16 d (bytes 0-1), fp16 dmin (2-3),
+ *    12 bytes of packed 6-bit scales and mins (4-15), 128 bytes of 4-bit
+ *    codes (16-143) in four runs of 32 bytes, run p holding chunk 2p in its
+ *    low nibbles and chunk 2p+1 in its high nibbles.  For the 32-element
+ *    chunk c of a block, w = d·sc_c·q - dmin·m_c (§2.1).
+ *  - W_dsc plane (same page, §2.2): for global chunk c = 8·block + j and row
+ *    n, the float2 (d·sc_j, -(dmin·m_j)), each one fp32 multiply, stored
+ *    chunk-major at byte offset (c·N + n)·8: (K/32)·N float2 = N·K/4 bytes.
+ *  - bf16: W [N][K] row-major, x [M][K] row-major, any K >= 1 and any 2-byte
+ *    aligned base (AstrAI commit log, astrai/extension/backend: the bf16 GEMV
+ *    accepts any K and any storage offset).
+ *
+ * Alignment: the int4 and q4_K entry points need 16-byte aligned device
+ * pointers (cudaMalloc and PyTorch allocations are); otherwise they return
+ * WQ_ERR_ALIGN.  The bf16 entry points accept any 2-byte aligned pointers.
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define WQ_OK 0
+#define WQ_ERR_ARG (-1)         /* bad pointer, dimension, block size or layout value */
+#define WQ_ERR_ALIGN (-2)       /* a device pointer is not 16-byte aligned (int4, q4_K) */
+#define WQ_ERR_LAYOUT (-3)      /* weights were packed for another layout version */
+#define WQ_ERR_CUDA (-4)        /* a CUDA runtime call or launch failed; see wq_last_error() */
+#define WQ_ERR_DEVICE (-5)      /* the current device is not sm_100 */
+#define WQ_ERR_TIMEOUT (-6)     /* a bounded device-side wait expired (see wq_device_status) */
+#define WQ_ERR_UNSUPPORTED (-7) /* valid arguments this build has no kernel for */
+
+/* Weight layout versions. */
+#define WQ_LAYOUT_CANONICAL 0
+
+/* ---------------------------------------------------------------------------
+ * GEMV / GEMM entry points.  All device pointers; y is written, never read.
+ * ------------------------------------------------------------------------- */
+
+/* y[M,N] fp16 = x[M,K] fp16 · dequant(int4)ᵀ.
+ * block_size: a power of two in [16, 256] with K % block_size == 0.
+ * zeros_u4 may be NULL (z = 8).  layout must be WQ_LAYOUT_CANONICAL.
+ * M >= 1, N >= 1, K >= 1.  Errors: WQ_ERR_ARG, WQ_ERR_ALIGN, WQ_ERR_LAYOUT,
+ * WQ_ERR_DEVICE, WQ_ERR_CUDA. */
+int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* scales_f16,
+                        const void* zeros_u4, void* y_f16, int M, int N, int K,
+                        int block_size, int layout, void* stream);
+
+/* y[M,N] fp16 = x[M,K] fp16 · dequant(q4_K)ᵀ, scales decoded in-kernel from
+ * the packed 6-bit fields.  K % 256 == 0.  w_q4k is N·(K/256)·144 bytes. */
+int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K,
+             int layout, void* stream);
+
+/* As gemv_q4k, but the per-chunk coefficients come from the W_dsc plane w_dsc
+ * ((K/32)·N float2, chunk-major, N·K/4 bytes; build it with wq_build_q4k_dsc or
+ * wq_build_q4k_dsc_device).  Only the code bytes of w_q4k are read. */
+int gemv_q4k_dsc(const void* x_f16, const void* w_q4k, const void* w_dsc, void* y_f16,
+                 int M, int N, int K, int layout, void* stream);
+
+/* y[M,N] bf16 = x[M,K] bf16 · W[N,K]ᵀ bf16.  Any K >= 1; x, w, y only need
+ * 2-byte alignment (rows of W and x are contiguous with stride K). */
+int gemv_bf16(const void* x_bf16, const void* w_bf16, void* y_bf16, int M, int N, int K,
+              void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Device dequantization exports: w_out [N,K] fp32 row-major, through the same
+ * device unpacking code the GEMV kernels use.  Every value is exact (the
+ * dequantized weights of these formats are exactly representable in fp32).
+ * ------------------------------------------------------------------------- */
+int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const void* zeros_u4,
+                           float* w_out, int N, int K, int block_size, int layout, void* stream);
+
+/* w_dsc NULL: coefficients decoded from the packed fields; else taken from the plane. */
+int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K, int layout,
+                void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Weight packing (load time).
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of each canonical int4 array (codes + scales + zero-points) for a
+ * layout; 0 for invalid arguments. */
+size_t wq_int4_bytes(int N, int K, int block_size, int layout);
+
+/* Bytes of a q4_K tensor and of its W_dsc plane; 0 for invalid arguments. */
+size_t wq_q4k_bytes(int N, int K);
+size_t wq_q4k_dsc_bytes(int N, int K);
+
+/* Build the W_dsc plane on the host (minfer doc 62, §2.2-§2.3): one IEEE fp32
+ * multiply per coefficient and an exact negation, no contraction.
+ * w_q4k_host: N·(K/256)·144 bytes; out_host: wq_q4k_dsc_bytes(N, K) bytes. */
+int wq_build_q4k_dsc(const void* w_q4k_host, int N, int K, void* out_host);
+
+/* The same plane built on the device (bit-identical to the host builder). */
+int wq_build_q4k_dsc_device(const void* w_q4k, void* out, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics.
+ * ------------------------------------------------------------------------- */
+const char* wq_last_error(void);   /* message of the last failure on this thread */
+const char* wq_last_kernel(void);  /* liveness label of the last launch on this thread */
+int wq_layout_version(void);       /* newest layout version this build reads */
+const char* wq_build_info(void);   /* "sm_100a ..." build description */
+
+/* Synchronizes the current device, then reads and clears the device-side
+ * error word that bounded waits set when they give up.  Returns WQ_OK or
+ * WQ_ERR_TIMEOUT (or WQ_ERR_CUDA if the synchronization itself fails). */
+int wq_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */

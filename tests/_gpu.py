@@ -1,0 +1,129 @@
+"""Helpers for the GPU parity tests: seeded inputs on the device, calls through
+the C ABI binding, and oracle comparisons (whole outputs or sampled rows)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import weight_only_quantized_q4_b200 as wq
+from weight_only_quantized_q4_b200 import synth
+
+DEV = "cuda:0"
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def f16_of(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy()
+
+
+def bf16_bits_of(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def check(y_dev: np.ndarray, W: np.ndarray, x: np.ndarray, what: str) -> None:
+    """Accept iff |y − y_ref| ≤ 2e-3·Σ|w·x| + 1e-3 for every element."""
+    y_ref = oracle.gemv(W, x)
+    B = oracle.bound(W, x)
+    bad = oracle.violations(y_dev, y_ref, B)
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        detail = [(tuple(i), float(y_dev[tuple(i)]), float(y_ref[tuple(i)]), float(B[tuple(i)])) for i in idx]
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; first: {detail}")
+
+
+# ----------------------------------------------------------------- int4
+
+class Int4Case:
+    def __init__(self, M, N, K, bs, zeros, workload=3, s_lo=0.002, s_hi=0.01):
+        self.M, self.N, self.K, self.bs = M, N, K, bs
+        t = synth.int4_weights(N, K, bs, scale_lo=s_lo, scale_hi=s_hi, with_zeros=zeros, workload=workload)
+        self.w, self.s, self.z = t["w_packed"], t["scales"], t["zeros"]
+        self.x = synth.activations_f16(M, K, workload=workload)
+        self.dw, self.ds = dev(self.w), dev(self.s)
+        self.dz = dev(self.z) if self.z is not None else None
+        self.dx = dev(self.x)
+
+    def run(self, stream=None) -> np.ndarray:
+        y = torch.empty((self.M, self.N), dtype=torch.float16, device=DEV)
+        wq.gemv_int4_blockwise(self.dx, self.dw, self.ds, self.dz, y, self.M, self.N, self.K, self.bs, stream=stream)
+        torch.cuda.synchronize()
+        return f16_of(y).astype(np.float64)
+
+    def W(self, rows=None):
+        r = slice(None) if rows is None else rows
+        z = None if self.z is None else self.z[r]
+        n = self.N if rows is None else len(rows)
+        return oracle.dequant_int4(self.w[r], self.s[r], z, n, self.K, self.bs)
+
+
+# ----------------------------------------------------------------- q4_K
+
+class Q4KCase:
+    def __init__(self, M, N, K, workload=4):
+        self.M, self.N, self.K = M, N, K
+        self.raw = synth.q4k_weights(N, K, workload=workload)
+        self.x = synth.activations_f16(M, K, workload=workload)
+        self.draw, self.dx = dev(self.raw), dev(self.x)
+        self._plane = None
+
+    def plane_dev(self):
+        if self._plane is None:
+            P = torch.empty((self.K // 32, self.N, 2), dtype=torch.float32, device=DEV)
+            wq.wq_build_q4k_dsc_device(self.draw, P, self.N, self.K)
+            torch.cuda.synchronize()
+            self._plane = P
+        return self._plane
+
+    def run(self, dsc: bool, stream=None) -> np.ndarray:
+        y = torch.empty((self.M, self.N), dtype=torch.float16, device=DEV)
+        if dsc:
+            wq.gemv_q4k_dsc(self.dx, self.draw, self.plane_dev(), y, self.M, self.N, self.K, stream=stream)
+        else:
+            wq.gemv_q4k(self.dx, self.draw, y, self.M, self.N, self.K, stream=stream)
+        torch.cuda.synchronize()
+        return f16_of(y).astype(np.float64)
+
+    def W(self, rows=None):
+        if rows is None:
+            return oracle.dequant_q4k(self.raw, self.N, self.K)
+        return oracle.dequant_q4k(self.raw[rows], len(rows), self.K)
+
+
+# ----------------------------------------------------------------- bf16
+
+class BF16Case:
+    def __init__(self, M, N, K, offset=0, workload=2):
+        self.M, self.N, self.K, self.offset = M, N, K, offset
+        self.wb = synth.bf16_weights_bits(N, K, workload=workload)
+        self.xb = synth.activations_bf16_bits(M, K, workload=workload)
+        wbuf, _ = synth.with_element_offset(self.wb, offset)
+        xbuf, _ = synth.with_element_offset(self.xb, offset)
+        self.dwbuf = dev(wbuf.view(np.int16)).view(torch.bfloat16)
+        self.dxbuf = dev(xbuf.view(np.int16)).view(torch.bfloat16)
+
+    def run(self, stream=None) -> np.ndarray:
+        ybuf = torch.zeros(self.M * self.N + 8, dtype=torch.bfloat16, device=DEV)
+        yp = ybuf.data_ptr() + 2 * self.offset
+        wq.gemv_bf16(self.dxbuf.data_ptr() + 2 * self.offset, self.dwbuf.data_ptr() + 2 * self.offset, yp,
+                     self.M, self.N, self.K, stream=stream)
+        torch.cuda.synchronize()
+        bits = bf16_bits_of(ybuf)[self.offset:self.offset + self.M * self.N].reshape(self.M, self.N)
+        return oracle.q4.bf16_bits_to_f64(bits)
+
+    def W(self, rows=None):
+        wb = self.wb if rows is None else self.wb[rows]
+        return oracle.dequant_bf16(wb, wb.shape[0], self.K)
+
+    def X(self):
+        return oracle.dequant_bf16(self.xb, self.M, self.K)
+
+
+def sample_rows(N: int, count: int = 48, seed: int = 0) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(0, N, count).tolist())
+    rows.update({0, 1, N - 1, N - 2, N // 2})
+    return np.array(sorted(r for r in rows if 0 <= r < N))

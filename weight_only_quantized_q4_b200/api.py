@@ -1,0 +1,94 @@
+"""Python face of the C ABI: the same names, tensors in, status checked.
+
+Each function takes torch CUDA tensors (or raw integer device pointers),
+passes their addresses and sizes to libwq.so on the current torch stream (or
+an explicit ``stream``), and raises WQError on a negative status.  Nothing
+here touches the data.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from ._lib import WQ_LAYOUT_CANONICAL, WQError, _check, last_error, last_kernel, lib  # noqa: F401
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def gemv_int4_blockwise(x, w_packed, scales, zeros, y, M, N, K, block_size, layout=WQ_LAYOUT_CANONICAL,
+                        stream=None):
+    _check(lib().gemv_int4_blockwise(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(zeros), _ptr(y), M, N, K,
+                                     block_size, layout, _stream(stream)), "gemv_int4_blockwise")
+
+
+def gemv_q4k(x, w_q4k, y, M, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
+    _check(lib().gemv_q4k(_ptr(x), _ptr(w_q4k), _ptr(y), M, N, K, layout, _stream(stream)), "gemv_q4k")
+
+
+def gemv_q4k_dsc(x, w_q4k, w_dsc, y, M, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
+    _check(lib().gemv_q4k_dsc(_ptr(x), _ptr(w_q4k), _ptr(w_dsc), _ptr(y), M, N, K, layout, _stream(stream)),
+           "gemv_q4k_dsc")
+
+
+def gemv_bf16(x, w, y, M, N, K, stream=None):
+    _check(lib().gemv_bf16(_ptr(x), _ptr(w), _ptr(y), M, N, K, _stream(stream)), "gemv_bf16")
+
+
+def dequant_int4_blockwise(w_packed, scales, zeros, w_out, N, K, block_size, layout=WQ_LAYOUT_CANONICAL,
+                           stream=None):
+    _check(lib().dequant_int4_blockwise(_ptr(w_packed), _ptr(scales), _ptr(zeros), _ptr(w_out), N, K, block_size,
+                                        layout, _stream(stream)), "dequant_int4_blockwise")
+
+
+def dequant_q4k(w_q4k, w_dsc, w_out, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
+    _check(lib().dequant_q4k(_ptr(w_q4k), _ptr(w_dsc), _ptr(w_out), N, K, layout, _stream(stream)), "dequant_q4k")
+
+
+def wq_int4_bytes(N, K, block_size, layout=WQ_LAYOUT_CANONICAL) -> int:
+    return int(lib().wq_int4_bytes(N, K, block_size, layout))
+
+
+def wq_q4k_bytes(N, K) -> int:
+    return int(lib().wq_q4k_bytes(N, K))
+
+
+def wq_q4k_dsc_bytes(N, K) -> int:
+    return int(lib().wq_q4k_dsc_bytes(N, K))
+
+
+def wq_build_q4k_dsc(w_q4k_host: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Host plane builder: returns float32 [K/32, N, 2] built by libwq's C++ packer."""
+    src = np.ascontiguousarray(w_q4k_host, dtype=np.uint8)
+    out = np.empty((K // 32, N, 2), dtype=np.float32)
+    _check(lib().wq_build_q4k_dsc(src.ctypes.data_as(ctypes.c_void_p), N, K, out.ctypes.data_as(ctypes.c_void_p)),
+           "wq_build_q4k_dsc")
+    return out
+
+
+def wq_build_q4k_dsc_device(w_q4k, out, N, K, stream=None):
+    _check(lib().wq_build_q4k_dsc_device(_ptr(w_q4k), _ptr(out), N, K, _stream(stream)), "wq_build_q4k_dsc_device")
+
+
+def wq_layout_version() -> int:
+    return int(lib().wq_layout_version())
+
+
+def wq_device_status() -> None:
+    _check(lib().wq_device_status(), "wq_device_status")

@@ -1,0 +1,532 @@
+// api.cu — the extern "C" entry points of libwq.so (declared in include/wq.h):
+// argument validation, kernel choice, launch, status and liveness labels.
+//
+// Nothing here computes on the host: every entry point either rejects its
+// arguments or enqueues kernels on the caller's stream.  There is no CPU
+// fallback and no silent kernel fallback: wq_last_kernel() names the kernel
+// each call launched.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/wq.h"
+#include "gemv_cc.cuh"
+#include "gemv_simple.cuh"
+#include "wq_host.h"
+
+namespace wq {
+
+namespace {
+thread_local std::string t_last_error;
+thread_local std::string t_last_kernel = "none";
+
+struct DeviceInfo {
+  int sms = 0;
+  bool is_sm100 = false;
+  bool valid = false;
+};
+DeviceInfo g_dev[64];
+std::mutex g_dev_mu;
+
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(WQ_ERR_DEVICE, "device ordinal out of range");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.valid) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return fail(WQ_ERR_CUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
+    d.sms = sms;
+    d.is_sm100 = (major == 10 && minor == 0);
+    d.valid = true;
+  }
+  *out = d;
+  if (!d.is_sm100) return fail(WQ_ERR_DEVICE, "libwq is built for sm_100a (B200); the current device is not sm_100");
+  return WQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0; }
+int ilog2_int(int v) {
+  int r = 0;
+  while ((1 << r) < v) ++r;
+  return r;
+}
+
+int launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return WQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// streaming CUDA-core GEMV: kernel table and planner
+// ---------------------------------------------------------------------------
+using CCKernel = void (*)(const CCParams);
+
+template <Fmt F, int M, int KS>
+CCKernel cc_ptr() {
+  return &gemv_cc_kernel<F, M, KS>;
+}
+
+// Instantiated segment sizes per format and batch (activation registers stay
+// at or below 32 per thread for the preferred choice, 64 for the fallback).
+template <Fmt F, int M>
+CCKernel cc_lookup(int KS) {
+  constexpr bool four = F != Fmt::BF16;
+  if constexpr (four) {
+    switch (KS) {
+      case 64:
+        if constexpr (M <= 1) return cc_ptr<F, M, 64>();
+        break;
+      case 32:
+        if constexpr (M <= 4) return cc_ptr<F, M, 32>();
+        break;
+      case 16:
+        if constexpr (M <= 8) return cc_ptr<F, M, 16>();
+        break;
+      case 8:
+        if constexpr (M >= 5) return cc_ptr<F, M, 8>();
+        break;
+      default:
+        break;
+    }
+  } else {
+    switch (KS) {
+      case 32:
+        if constexpr (M <= 2) return cc_ptr<F, M, 32>();
+        break;
+      case 16:
+        if constexpr (M <= 8) return cc_ptr<F, M, 16>();
+        break;
+      case 8:
+        if constexpr (M >= 2) return cc_ptr<F, M, 8>();
+        break;
+      default:
+        break;
+    }
+  }
+  return nullptr;
+}
+
+template <Fmt F>
+CCKernel cc_kernel_for(int M, int KS) {
+  switch (M) {
+    case 1: return cc_lookup<F, 1>(KS);
+    case 2: return cc_lookup<F, 2>(KS);
+    case 3: return cc_lookup<F, 3>(KS);
+    case 4: return cc_lookup<F, 4>(KS);
+    case 5: return cc_lookup<F, 5>(KS);
+    case 6: return cc_lookup<F, 6>(KS);
+    case 7: return cc_lookup<F, 7>(KS);
+    case 8: return cc_lookup<F, 8>(KS);
+    default: return nullptr;
+  }
+}
+
+CCKernel cc_kernel(Fmt f, int M, int KS) {
+  switch (f) {
+    case Fmt::Int4: return cc_kernel_for<Fmt::Int4>(M, KS);
+    case Fmt::Q4K: return cc_kernel_for<Fmt::Q4K>(M, KS);
+    case Fmt::Q4KDsc: return cc_kernel_for<Fmt::Q4KDsc>(M, KS);
+    case Fmt::BF16: return cc_kernel_for<Fmt::BF16>(M, KS);
+  }
+  return nullptr;
+}
+
+// Segment-size preference per format and batch.
+int ks_candidates(Fmt f, int M, int* out) {
+  if (f != Fmt::BF16) {
+    if (M == 1) { out[0] = 64; out[1] = 32; out[2] = 16; return 3; }
+    if (M == 2) { out[0] = 32; out[1] = 16; return 2; }
+    if (M <= 4) { out[0] = 16; out[1] = 32; return 2; }
+    out[0] = 8; out[1] = 16; return 2;
+  }
+  if (M == 1) { out[0] = 32; out[1] = 16; return 2; }
+  if (M == 2) { out[0] = 32; out[1] = 16; out[2] = 8; return 3; }
+  if (M <= 4) { out[0] = 16; out[1] = 8; return 2; }
+  out[0] = 8; out[1] = 16; return 2;
+}
+
+constexpr int kStageCap = 32 * 1024;
+constexpr int kSmemPerSm = 220 * 1024;
+
+struct CCPlan {
+  CCKernel fn = nullptr;
+  CCParams p{};
+  int threads = 0, grid = 0, smem = 0, KS = 0;
+};
+
+int round16(long long v) { return static_cast<int>((v + 15) & ~15ll); }
+
+bool plan_cc(Fmt f, int M, int N, int K, long long row_bytes, int nb, int zb, int block_size, bool has_zeros,
+             int sms, CCPlan* plan) {
+  int cands[4];
+  const int nc = ks_candidates(f, M, cands);
+  // Prefer a candidate without idle lanes in the last warp of a row group.
+  int best = -1;
+  double best_idle = 2.0;
+  for (int i = 0; i < nc; ++i) {
+    const int KS = cands[i];
+    if (K % KS) continue;
+    if (f == Fmt::Int4 && KS > block_size) continue;
+    const int S = K / KS;
+    const int WK = (S + 31) / 32;
+    if (WK * 32 > 512) continue;
+    if (!cc_kernel(f, M, KS)) continue;
+    const double idle = double(WK * 32 - S) / double(WK * 32);
+    if (idle < best_idle - 0.05) {  // earlier candidates win unless clearly less idle
+      best_idle = idle;
+      best = KS;
+    }
+  }
+  if (best < 0) return false;
+  const int KS = best;
+  const int S = K / KS;
+  const int WK = (S + 31) / 32;
+  const int RGMAX = rg_max(M);
+
+  auto stage_bytes_for = [&](int RS, int* o_sc, int* o_z, int* o_pl, int* pstride) {
+    long long off = round16(RS * row_bytes);
+    *o_sc = *o_z = *o_pl = 0;
+    *pstride = 0;
+    if (f == Fmt::Int4) {
+      *o_sc = static_cast<int>(off);
+      off += round16(2ll * RS * nb + 32);
+      if (has_zeros) {
+        *o_z = static_cast<int>(off);
+        off += round16(1ll * RS * zb + 32);
+      }
+    }
+    if (f == Fmt::Q4KDsc) {
+      *o_pl = static_cast<int>(off);
+      *pstride = round16(8ll * RS + 16);
+      off += static_cast<long long>(*pstride) * (K / 32);
+    }
+    return off;
+  };
+
+  const int Gmax = std::max(1, 512 / (WK * 32));
+  int G = std::min(Gmax, std::max(1, (256 + WK * 32 - 1) / (WK * 32)));
+  int RG = RGMAX;
+  int o_sc, o_z, o_pl, pstride;
+  long long sb = 0;
+  while (true) {
+    sb = stage_bytes_for(G * RG, &o_sc, &o_z, &o_pl, &pstride);
+    if (sb <= kStageCap) break;
+    if (RG > 1) {
+      --RG;
+    } else if (G > 1) {
+      --G;
+    } else {
+      break;  // one row per stage is over the cap: accept a bigger stage
+    }
+  }
+  const int RS = G * RG;
+  const long long red = 2ll * RS * WK * M * 4;
+  const long long tail = red + 8ll * 8 + 16;
+  int NS = 4, ctas_per_sm = 2;
+  if (NS * sb + tail > kSmemPerSm / 2) {
+    ctas_per_sm = 1;
+    NS = static_cast<int>(std::min<long long>(6, (kSmemPerSm - tail) / sb));
+  }
+  if (NS < 2) return false;
+  const int n_granules = (N + 1) / 2;
+  const int grid = std::max(1, std::min(ctas_per_sm * sms, n_granules));
+
+  CCParams& p = plan->p;
+  p.N = N;
+  p.K = K;
+  p.nb = nb;
+  p.zb = zb;
+  p.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
+  p.row_bytes = row_bytes;
+  p.S = S;
+  p.WK = WK;
+  p.G = G;
+  p.RG = RG;
+  p.RS = RS;
+  p.NS = NS;
+  p.n_granules = n_granules;
+  p.stage_bytes = static_cast<int>(sb);
+  p.off_scales = o_sc;
+  p.off_zeros = o_z;
+  p.off_plane = o_pl;
+  p.plane_stride = pstride;
+  p.red_offset = static_cast<int>(NS * sb);
+  plan->fn = cc_kernel(f, M, KS);
+  plan->threads = G * WK * 32;
+  plan->grid = grid;
+  plan->smem = static_cast<int>(NS * sb + tail);
+  plan->KS = KS;
+  return plan->fn != nullptr;
+}
+
+int launch_cc(const CCPlan& plan, cudaStream_t st) {
+  static std::mutex mu;
+  static std::pair<CCKernel, int> configured[512];
+  static int n_configured = 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    bool found = false;
+    for (int i = 0; i < n_configured; ++i)
+      if (configured[i].first == plan.fn && configured[i].second == dev) found = true;
+    if (!found) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(plan.fn),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      if (n_configured < 512) configured[n_configured++] = {plan.fn, dev};
+    }
+  }
+  plan.fn<<<plan.grid, plan.threads, plan.smem, st>>>(plan.p);
+  return launch_check("gemv_cc launch");
+}
+
+std::string cc_label(const char* fmt, int M, int KS, const char* extra) {
+  char buf[96];
+  std::snprintf(buf, sizeof(buf), "%s.gemv.cc.m%d.ks%d%s", fmt, M, KS, extra);
+  return buf;
+}
+
+template <Fmt F>
+int launch_simple(const SimpleParams& sp, int M, int sms, cudaStream_t st) {
+  const int threads = 256;
+  const int rows_per_block = threads / 32;
+  const int grid = std::max(1, std::min((sp.N + rows_per_block - 1) / rows_per_block, sms * 16));
+  switch (M) {
+    case 1: gemv_simple_kernel<F, 1><<<grid, threads, 0, st>>>(sp); break;
+    case 2: gemv_simple_kernel<F, 2><<<grid, threads, 0, st>>>(sp); break;
+    case 3: gemv_simple_kernel<F, 3><<<grid, threads, 0, st>>>(sp); break;
+    case 4: gemv_simple_kernel<F, 4><<<grid, threads, 0, st>>>(sp); break;
+    case 5: gemv_simple_kernel<F, 5><<<grid, threads, 0, st>>>(sp); break;
+    case 6: gemv_simple_kernel<F, 6><<<grid, threads, 0, st>>>(sp); break;
+    case 7: gemv_simple_kernel<F, 7><<<grid, threads, 0, st>>>(sp); break;
+    case 8: gemv_simple_kernel<F, 8><<<grid, threads, 0, st>>>(sp); break;
+    default: return fail(WQ_ERR_ARG, "simple kernel: M chunk out of range");
+  }
+  return launch_check("gemv_simple launch");
+}
+
+// Run one format over all M in chunks of at most 8 rows of x.
+template <Fmt F>
+int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros,
+             const uint8_t* plane, void* y, int M, int N, int K, long long row_bytes, int nb, int zb,
+             int block_size, bool fast_ok, cudaStream_t st) {
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  std::string label;
+  const int x_elt = 2;
+  for (int m0 = 0; m0 < M; m0 += 8) {
+    const int mc = std::min(8, M - m0);
+    const void* xc = static_cast<const uint8_t*>(x) + static_cast<long long>(m0) * K * x_elt;
+    void* yc = static_cast<uint8_t*>(y) + static_cast<long long>(m0) * N * 2;
+    CCPlan plan;
+    const bool use_cc = fast_ok && aligned16(xc) &&
+                        plan_cc(F, mc, N, K, row_bytes, nb, zb, block_size, zeros != nullptr, di.sms, &plan);
+    if (use_cc) {
+      plan.p.x = xc;
+      plan.p.w = w;
+      plan.p.scales = scales;
+      plan.p.zeros = zeros;
+      plan.p.plane = plane;
+      plan.p.y = yc;
+      rc = launch_cc(plan, st);
+      if (rc) return rc;
+      label = cc_label(fmt_name, mc, plan.KS, M > 8 ? ".chunked" : "");
+    } else {
+      SimpleParams sp{};
+      sp.x = xc;
+      sp.w = w;
+      sp.scales = scales;
+      sp.zeros = zeros;
+      sp.plane = plane;
+      sp.y = yc;
+      sp.M = mc;
+      sp.N = N;
+      sp.K = K;
+      sp.nb = nb;
+      sp.zb = zb;
+      sp.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
+      rc = launch_simple<F>(sp, mc, di.sms, st);
+      if (rc) return rc;
+      char buf[64];
+      std::snprintf(buf, sizeof(buf), "%s.gemv.simple.m%d%s", fmt_name, mc, M > 8 ? ".chunked" : "");
+      label = buf;
+    }
+  }
+  set_last_kernel(label);
+  return WQ_OK;
+}
+
+int check_dims(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "M, N and K must be >= 1");
+  return WQ_OK;
+}
+
+int check_int4(int K, int block_size, int layout) {
+  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown int4 layout version");
+  if (block_size < 16 || block_size > 256 || (block_size & (block_size - 1)))
+    return fail(WQ_ERR_ARG, "block_size must be a power of two in [16, 256]");
+  if (K % block_size) return fail(WQ_ERR_ARG, "K must be a multiple of block_size");
+  return WQ_OK;
+}
+
+}  // namespace
+
+int fail(int code, const std::string& msg) {
+  t_last_error = msg;
+  return code;
+}
+int ok() { return WQ_OK; }
+void set_last_kernel(const std::string& label) { t_last_kernel = label; }
+
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" {
+
+int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* scales_f16, const void* zeros_u4,
+                        void* y_f16, int M, int N, int K, int block_size, int layout, void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if ((rc = check_int4(K, block_size, layout))) return rc;
+  if (!x_f16 || !w_packed || !scales_f16 || !y_f16) return fail(WQ_ERR_ARG, "gemv_int4_blockwise: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_packed) || !aligned16(scales_f16) || !aligned16(y_f16) ||
+      (zeros_u4 && !aligned16(zeros_u4)))
+    return fail(WQ_ERR_ALIGN, "gemv_int4_blockwise: device pointers must be 16-byte aligned");
+  const int nb = K / block_size;
+  const int zb = (nb + 1) / 2;
+  const long long row_bytes = K / 2;
+  const bool fast = (row_bytes % 16) == 0;
+  return run_gemv<Fmt::Int4>("int4", x_f16, static_cast<const uint8_t*>(w_packed),
+                             static_cast<const uint8_t*>(scales_f16), static_cast<const uint8_t*>(zeros_u4), nullptr,
+                             y_f16, M, N, K, row_bytes, nb, zb, block_size, fast, static_cast<cudaStream_t>(stream));
+}
+
+int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K, int layout, void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
+  if (K % 256) return fail(WQ_ERR_ARG, "gemv_q4k: K must be a multiple of 256");
+  if (!x_f16 || !w_q4k || !y_f16) return fail(WQ_ERR_ARG, "gemv_q4k: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_q4k) || !aligned16(y_f16))
+    return fail(WQ_ERR_ALIGN, "gemv_q4k: device pointers must be 16-byte aligned");
+  return run_gemv<Fmt::Q4K>("q4k", x_f16, static_cast<const uint8_t*>(w_q4k), nullptr, nullptr, nullptr, y_f16, M,
+                            N, K, static_cast<long long>(K / 256) * 144, 0, 0, 0, true,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int gemv_q4k_dsc(const void* x_f16, const void* w_q4k, const void* w_dsc, void* y_f16, int M, int N, int K,
+                 int layout, void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
+  if (K % 256) return fail(WQ_ERR_ARG, "gemv_q4k_dsc: K must be a multiple of 256");
+  if (!x_f16 || !w_q4k || !w_dsc || !y_f16) return fail(WQ_ERR_ARG, "gemv_q4k_dsc: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_q4k) || !aligned16(w_dsc) || !aligned16(y_f16))
+    return fail(WQ_ERR_ALIGN, "gemv_q4k_dsc: device pointers must be 16-byte aligned");
+  return run_gemv<Fmt::Q4KDsc>("q4k_dsc", x_f16, static_cast<const uint8_t*>(w_q4k), nullptr, nullptr,
+                               static_cast<const uint8_t*>(w_dsc), y_f16, M, N, K,
+                               static_cast<long long>(K / 256) * 144, 0, 0, 0, true,
+                               static_cast<cudaStream_t>(stream));
+}
+
+int gemv_bf16(const void* x_bf16, const void* w_bf16, void* y_bf16, int M, int N, int K, void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (!x_bf16 || !w_bf16 || !y_bf16) return fail(WQ_ERR_ARG, "gemv_bf16: null pointer");
+  if (!aligned2(x_bf16) || !aligned2(w_bf16) || !aligned2(y_bf16))
+    return fail(WQ_ERR_ARG, "gemv_bf16: pointers must be 2-byte aligned");
+  const bool fast = aligned16(x_bf16) && aligned16(w_bf16) && (K % 8) == 0;
+  return run_gemv<Fmt::BF16>("bf16", x_bf16, static_cast<const uint8_t*>(w_bf16), nullptr, nullptr, nullptr, y_bf16,
+                             M, N, K, 2ll * K, 0, 0, 0, fast, static_cast<cudaStream_t>(stream));
+}
+
+int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const void* zeros_u4, float* w_out, int N,
+                           int K, int block_size, int layout, void* stream) {
+  int rc = check_dims(1, N, K);
+  if (rc) return rc;
+  if ((rc = check_int4(K, block_size, layout))) return rc;
+  if (!w_packed || !scales_f16 || !w_out) return fail(WQ_ERR_ARG, "dequant_int4_blockwise: null pointer");
+  if (!aligned16(w_packed) || !aligned16(scales_f16) || (zeros_u4 && !aligned16(zeros_u4)) || !aligned16(w_out))
+    return fail(WQ_ERR_ALIGN, "dequant_int4_blockwise: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  const int nb = K / block_size;
+  const long long words = static_cast<long long>(N) * (K / 8);
+  const int grid = static_cast<int>(std::min<long long>((words + 255) / 256, di.sms * 32ll));
+  dequant_int4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_packed), static_cast<const uint8_t*>(scales_f16),
+      static_cast<const uint8_t*>(zeros_u4), w_out, N, K, nb, (nb + 1) / 2, ilog2_int(block_size));
+  if ((rc = launch_check("dequant_int4 launch"))) return rc;
+  set_last_kernel("int4.dequant");
+  return WQ_OK;
+}
+
+int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K, int layout, void* stream) {
+  int rc = check_dims(1, N, K);
+  if (rc) return rc;
+  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
+  if (K % 256) return fail(WQ_ERR_ARG, "dequant_q4k: K must be a multiple of 256");
+  if (!w_q4k || !w_out) return fail(WQ_ERR_ARG, "dequant_q4k: null pointer");
+  if (!aligned16(w_q4k) || (w_dsc && !aligned16(w_dsc)) || !aligned16(w_out))
+    return fail(WQ_ERR_ALIGN, "dequant_q4k: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  const long long words = static_cast<long long>(N) * (K / 256) * 32;
+  const int grid = static_cast<int>(std::min<long long>((words + 255) / 256, di.sms * 32ll));
+  dequant_q4k_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_q4k), static_cast<const uint8_t*>(w_dsc), w_out, N, K);
+  if ((rc = launch_check("dequant_q4k launch"))) return rc;
+  set_last_kernel(w_dsc ? "q4k_dsc.dequant" : "q4k.dequant");
+  return WQ_OK;
+}
+
+int wq_build_q4k_dsc_device(const void* w_q4k, void* out, int N, int K, void* stream) {
+  if (N <= 0 || K <= 0 || K % 256) return fail(WQ_ERR_ARG, "wq_build_q4k_dsc_device: need N > 0, K % 256 == 0");
+  if (!w_q4k || !out) return fail(WQ_ERR_ARG, "wq_build_q4k_dsc_device: null pointer");
+  if (!aligned16(w_q4k) || !aligned16(out))
+    return fail(WQ_ERR_ALIGN, "wq_build_q4k_dsc_device: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const long long total = static_cast<long long>(K / 32) * N;
+  const int grid = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 32ll));
+  build_q4k_dsc_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<const uint8_t*>(w_q4k),
+                                                                            static_cast<float2*>(out), N, K);
+  if ((rc = launch_check("build_q4k_dsc launch"))) return rc;
+  set_last_kernel("q4k.build_dsc");
+  return WQ_OK;
+}
+
+const char* wq_last_error(void) { return t_last_error.c_str(); }
+const char* wq_last_kernel(void) { return t_last_kernel.c_str(); }
+int wq_layout_version(void) { return WQ_LAYOUT_CANONICAL; }
+const char* wq_build_info(void) { return "libwq sm_100a; CUDA-core streaming GEMV (M<=8), fallback GEMV, exports"; }
+
+int wq_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaDeviceSynchronize: ") + cudaGetErrorString(e));
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("read device error word: ") + cudaGetErrorString(e));
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("clear device error word: ") + cudaGetErrorString(e));
+  if (v & kDevErrTimeout) return fail(WQ_ERR_TIMEOUT, "a bounded device-side wait expired");
+  return WQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+// gemv_simple.cuh — general-shape kernels: the fallback GEMV (any alignment,
+// any K, any M in chunks of 8), the dequantization exports and the device
+// W_dsc plane builder.
+//
+// The exports walk the codes exactly the way the streaming GEMV does (one
+// 32-bit word -> four fp16x2 subnormal code pairs via lo4/hi4, q4_K chunk
+// pairs via q4k_scale_min_pair), then widen each code exactly to fp32, so a
+// bit-exact comparison of the export against the oracle checks the unpacking
+// and coefficient decoding the fast kernels rely on.
+#pragma once
+
+#include "wq_device.cuh"
+#include "gemv_cc.cuh"
+
+namespace wq {
+
+struct SimpleParams {
+  const void* x;
+  const uint8_t* w;
+  const uint8_t* scales;
+  const uint8_t* zeros;
+  const uint8_t* plane;
+  void* y;
+  int M, N, K;
+  int nb, zb, block_shift;
+};
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float((b16 & 0xFFFFu) << 16); }
+
+// Exact fp32 weight W[row, k] for the scalar fallback (plain byte reads).
+template <Fmt F>
+__device__ __forceinline__ float weight_scalar(const SimpleParams& p, int row, int k) {
+  if constexpr (F == Fmt::Int4) {
+    const uint32_t byte = p.w[static_cast<long long>(row) * (p.K / 2) + (k >> 1)];
+    const uint32_t q = (k & 1) ? (byte >> 4) : (byte & 15u);
+    const int b = k >> p.block_shift;
+    const uint32_t sb = reinterpret_cast<const uint16_t*>(p.scales)[static_cast<long long>(row) * p.nb + b];
+    uint32_t z = 8u;
+    if (p.zeros) {
+      const uint32_t zb = p.zeros[static_cast<long long>(row) * p.zb + (b >> 1)];
+      z = (b & 1) ? (zb >> 4) : (zb & 15u);
+    }
+    return static_cast<float>(static_cast<int>(q) - static_cast<int>(z)) * h16_to_f32(sb);
+  } else if constexpr (F == Fmt::Q4K || F == Fmt::Q4KDsc) {
+    const uint8_t* blk = p.w + (static_cast<long long>(row) * (p.K / 256) + (k >> 8)) * 144;
+    const int e = k & 255;
+    const int c = e >> 5;
+    const uint32_t byte = blk[16 + 32 * (e >> 6) + (e & 31)];
+    const uint32_t q = (e & 32) ? (byte >> 4) : (byte & 15u);
+    float A, B;
+    if constexpr (F == Fmt::Q4K) {
+      const uint32_t* hw = reinterpret_cast<const uint32_t*>(blk);
+      uint32_t sc, mn;
+      q4k_scale_min(hw[1], hw[2], hw[3], c, sc, mn);
+      A = __fmul_rn(h16_to_f32(hw[0]), static_cast<float>(sc));
+      B = -__fmul_rn(h16_to_f32(hw[0] >> 16), static_cast<float>(mn));
+    } else {
+      const float2 P = reinterpret_cast<const float2*>(p.plane)[static_cast<long long>((k >> 5)) * p.N + row];
+      A = P.x;
+      B = P.y;
+    }
+    return fmaf(A, static_cast<float>(q), B);
+  } else {
+    return bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(p.w)[static_cast<long long>(row) * p.K + k]);
+  }
+}
+
+template <Fmt F>
+__device__ __forceinline__ float act_scalar(const SimpleParams& p, int m, int k) {
+  const uint16_t b = reinterpret_cast<const uint16_t*>(p.x)[static_cast<long long>(m) * p.K + k];
+  if constexpr (F == Fmt::BF16)
+    return bf16_bits_to_f32(b);
+  else
+    return h16_to_f32(b);
+}
+
+// One warp per row (grid-stride), lanes stride over K, fp32 products and sums.
+template <Fmt F, int M>
+__global__ void __launch_bounds__(256) gemv_simple_kernel(const SimpleParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long row = warp; row < p.N; row += n_warps) {
+    float acc[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) acc[m] = 0.f;
+    for (int k = lane; k < p.K; k += 32) {
+      const float wv = weight_scalar<F>(p, static_cast<int>(row), k);
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[m] = fmaf(wv, act_scalar<F>(p, m, k), acc[m]);
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const long long o = static_cast<long long>(m) * p.N + row;
+        if constexpr (F == Fmt::BF16)
+          reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(acc[m]);
+        else
+          reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(acc[m]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dequantization exports (fp32 [N, K]); one thread per 32-bit word of codes
+// ---------------------------------------------------------------------------
+
+// Exact value of a code held as a subnormal in half `h` of a pair produced by
+// lo4 (scale 2^-24) or hi4 (scale 2^-20).
+__device__ __forceinline__ float code_of(uint32_t pair, int h, bool high_class) {
+  const float v = h16_to_f32(pair >> (16 * h));
+  return high_class ? v * 1048576.0f : v * 16777216.0f;
+}
+
+__global__ void dequant_int4_kernel(const uint8_t* w, const uint8_t* scales, const uint8_t* zeros, float* out,
+                                    int N, int K, int nb, int zb, int block_shift) {
+  const long long words_per_row = K / 8;
+  const long long total = static_cast<long long>(N) * words_per_row;
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = t / words_per_row;
+    const int wd = static_cast<int>(t - row * words_per_row);
+    const uint32_t v = reinterpret_cast<const uint32_t*>(w + row * (K / 2))[wd];
+    const uint32_t pr[4] = {lo4(v), hi4(v), lo4(v >> 8), hi4(v >> 8)};  // (n0,n4) (n1,n5) (n2,n6) (n3,n7)
+    const int k0 = 8 * wd;
+    const int b = k0 >> block_shift;  // a word never straddles a block (block >= 16)
+    const float s = h16_to_f32(reinterpret_cast<const uint16_t*>(scales)[row * nb + b]);
+    float z = 8.f;
+    if (zeros) {
+      const uint32_t zbyte = zeros[row * zb + (b >> 1)];
+      z = static_cast<float>((b & 1) ? (zbyte >> 4) : (zbyte & 15u));
+    }
+    float* o = out + row * K + k0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool high = (i & 1) != 0;
+      const int e0 = (i >> 1) * 2 + (high ? 1 : 0);  // nibble index of the pair's low half
+      o[e0] = (code_of(pr[i], 0, high) - z) * s;
+      o[e0 + 4] = (code_of(pr[i], 1, high) - z) * s;
+    }
+  }
+}
+
+// q4_K: thread per 32-bit word of codes; word t of block covers code bytes
+// 4t'..4t'+3 of run p, i.e. elements i..i+3 of chunks 2p and 2p+1.
+__global__ void dequant_q4k_kernel(const uint8_t* w, const uint8_t* plane, float* out, int N, int K) {
+  const long long words_per_row = (K / 256) * 32;
+  const long long total = static_cast<long long>(N) * words_per_row;
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = t / words_per_row;
+    const int wr = static_cast<int>(t - row * words_per_row);
+    const int sb = wr >> 5;
+    const int wq = wr & 31;            // word inside the 128 code bytes
+    const int pp = wq >> 3;            // run
+    const int i = (wq & 7) * 4;        // first element inside the chunk
+    const uint8_t* blk = w + (row * (K / 256) + sb) * 144;
+    const uint32_t v = reinterpret_cast<const uint32_t*>(blk + 16)[wq];
+    float A0, A1, B0, B1;
+    if (plane) {
+      const int c0 = sb * 8 + 2 * pp;
+      const float2 P0 = reinterpret_cast<const float2*>(plane)[static_cast<long long>(c0) * N + row];
+      const float2 P1 = reinterpret_cast<const float2*>(plane)[static_cast<long long>(c0 + 1) * N + row];
+      A0 = P0.x; B0 = P0.y; A1 = P1.x; B1 = P1.y;
+    } else {
+      const uint32_t* hw = reinterpret_cast<const uint32_t*>(blk);
+      uint32_t sc2, mn2;
+      q4k_scale_min_pair(hw[1], hw[2], hw[3], static_cast<uint32_t>(pp & 1), static_cast<uint32_t>(pp >> 1), sc2,
+                         mn2);
+      const float d = h16_to_f32(hw[0]);
+      const float dmin = h16_to_f32(hw[0] >> 16);
+      A0 = __fmul_rn(d, static_cast<float>(sc2 & 0xFFu));
+      A1 = __fmul_rn(d, static_cast<float>(sc2 >> 8));
+      B0 = -__fmul_rn(dmin, static_cast<float>(mn2 & 0xFFu));
+      B1 = -__fmul_rn(dmin, static_cast<float>(mn2 >> 8));
+    }
+    // pairs: lo4(v) = (c0[i], c0[i+2]); hi4(v) = (c1[i], c1[i+2]);
+    //        lo4(v>>8) = (c0[i+1], c0[i+3]); hi4(v>>8) = (c1[i+1], c1[i+3])
+    const uint32_t p0 = lo4(v), p1 = hi4(v), p2 = lo4(v >> 8), p3 = hi4(v >> 8);
+    float* o0 = out + row * K + sb * 256 + 64 * pp + i;  // chunk 2p
+    float* o1 = o0 + 32;                                 // chunk 2p+1
+    o0[0] = fmaf(A0, code_of(p0, 0, false), B0);
+    o0[2] = fmaf(A0, code_of(p0, 1, false), B0);
+    o0[1] = fmaf(A0, code_of(p2, 0, false), B0);
+    o0[3] = fmaf(A0, code_of(p2, 1, false), B0);
+    o1[0] = fmaf(A1, code_of(p1, 0, true), B1);
+    o1[2] = fmaf(A1, code_of(p1, 1, true), B1);
+    o1[1] = fmaf(A1, code_of(p3, 0, true), B1);
+    o1[3] = fmaf(A1, code_of(p3, 1, true), B1);
+  }
+}
+
+// W_dsc plane on the device (minfer doc 62, §2.2-§2.3): thread per (chunk, row).
+__global__ void build_q4k_dsc_kernel(const uint8_t* w, float2* plane, int N, int K) {
+  const long long n_chunks = K / 32;
+  const long long total = n_chunks * N;
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = t / N;
+    const long long row = t - c * N;
+    const uint32_t* hw = reinterpret_cast<const uint32_t*>(w + (row * (K / 256) + c / 8) * 144);
+    uint32_t sc, mn;
+    q4k_scale_min(hw[1], hw[2], hw[3], static_cast<int>(c & 7), sc, mn);
+    const float px = __fmul_rn(h16_to_f32(hw[0]), static_cast<float>(sc));
+    const float py = -__fmul_rn(h16_to_f32(hw[0] >> 16), static_cast<float>(mn));
+    plane[t] = make_float2(px, py);
+  }
+}
+
+}  // namespace wq
