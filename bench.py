@@ -36,8 +36,9 @@ from weight_only_quantized_q4_b200 import synth  # noqa: E402
 # ---------------------------------------------------------------- workloads
 
 
-def _int4(M, N, K, bs, zeros, workload, s_lo, s_hi):
-    return dict(fmt="int4", M=M, N=N, K=K, bs=bs, zeros=zeros, workload=workload, s_lo=s_lo, s_hi=s_hi)
+def _int4(M, N, K, bs, zeros, workload, s_lo, s_hi, layout=0):
+    return dict(fmt="int4", M=M, N=N, K=K, bs=bs, zeros=zeros, workload=workload, s_lo=s_lo, s_hi=s_hi,
+                layout=layout)
 
 
 WORKLOADS = {
@@ -57,9 +58,14 @@ for _M in (1, 3, 8):
         WORKLOADS[f"bf16_m{_M}_{_N}x{_K}"] = dict(fmt="bf16", M=_M, N=_N, K=_K, workload=2)
 for _M in (2, 4, 8):
     WORKLOADS[f"int4_b128_zp_m{_M}_4096x14336"] = _int4(_M, 4096, 14336, 128, True, 3, 0.002, 0.01)
+for _M in (1, 2, 4, 8):
+    for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336)):
+        WORKLOADS[f"int4_b128_zp_v1_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 3, 0.002, 0.01, layout=1)
 
 DEFAULT_WORKLOAD = "int4_b128_zp_m1_4096x14336"
-SWEEP = ["int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
+SWEEP = ["int4_b128_zp_v1_m1_4096x14336", "int4_b128_zp_v1_m2_4096x14336", "int4_b128_zp_v1_m4_4096x14336", "int4_b128_zp_v1_m8_4096x14336",
+         "int4_b128_zp_v1_m1_14336x4096", "int4_b128_zp_v1_m1_4096x4096",
+         "int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
          "int4_b32_m1_256x1024", "q4k_m1_4096x11008", "q4k_dsc_m1_4096x11008", "q4k_m4_11008x4096",
          "q4k_m8_4096x4096", "bf16_m1_1536x6912", "bf16_m3_1536x6912", "bf16_m8_1536x6912", "bf16_m1_151936x1536"]
 
@@ -154,7 +160,7 @@ class ClockSampler:
 class DeviceWorkload:
     """Device buffers for one workload plus a callable that issues one call on copy i."""
 
-    def __init__(self, w, host, torch, wq, l2_bytes):
+    def __init__(self, w, host, torch, wq, l2_bytes, copies=0):
         self.w, self.torch, self.wq = w, torch, wq
         dev = torch.device("cuda", torch.cuda.current_device())
         M, N, K = w["M"], w["N"], w["K"]
@@ -163,10 +169,16 @@ class DeviceWorkload:
         # enough weight copies that a round trip exceeds 3x L2
         self.R = max(1, -(-3 * l2_bytes // max(self.bytes, 1)))
         self.R = min(self.R, max(1, int(8e9 // max(self.bytes, 1))))
+        if copies > 0:
+            self.R = copies
         self.copies = []
         if w["fmt"] == "int4":
             base = [torch.from_numpy(host["w_packed"]).to(dev), torch.from_numpy(host["scales"]).to(dev),
                     torch.from_numpy(host["zeros"]).to(dev) if host["zeros"] is not None else None]
+            if w.get("layout", 0) == 1:  # offline repack to the B200_V1 stream (codes + scales + zero-points)
+                packed = torch.empty(wq.wq_int4_packed_bytes(N, K, w["bs"], 1), dtype=torch.uint8, device=dev)
+                wq.wq_repack_int4(base[0], base[1], base[2], packed, N, K, w["bs"], 1)
+                base = [packed, None, None]
             for _ in range(self.R):
                 self.copies.append([t.clone() if t is not None else None for t in base])
             self.x = torch.from_numpy(host["x"]).to(dev)
@@ -196,7 +208,8 @@ class DeviceWorkload:
         y = self.y if y is None else y
         w, wq = self.w, self.wq
         if w["fmt"] == "int4":
-            wq.gemv_int4_blockwise(x, c[0], c[1], c[2], y, self.M, self.N, self.K, w["bs"], stream=stream)
+            wq.gemv_int4_blockwise(x, c[0], c[1], c[2], y, self.M, self.N, self.K, w["bs"],
+                                   layout=w.get("layout", 0), stream=stream)
         elif w["fmt"] == "q4k":
             if w["dsc"]:
                 wq.gemv_q4k_dsc(x, c[0], c[1], y, self.M, self.N, self.K, stream=stream)
@@ -246,7 +259,7 @@ def run_ours(args, w, wname, rank, world, dist):
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
     host = host_inputs(w)
-    d = DeviceWorkload(w, host, torch, wq, l2)
+    d = DeviceWorkload(w, host, torch, wq, l2, copies=args.copies)
     stream = torch.cuda.Stream()
 
     # configure every kernel once outside capture, then capture a graph of G calls
@@ -358,6 +371,7 @@ def run_ours(args, w, wname, rank, world, dist):
         "dtype": dtype_of(w),
         "data": "synthetic (seeded; value distributions of the workload definition)",
         "config": {"workload": wname, "fmt": w["fmt"], "M": w["M"], "N": w["N"], "K": w["K"],
+                   "layout": {0: "canonical", 1: "B200_V1 (offline repack)"}[w.get("layout", 0)],
                    "weight_bytes_per_call": bytes_call, "weight_copies_rotated": d.R,
                    "l2": f"inputs larger than L2: {d.R} rotating weight copies, {d.R * bytes_call / 1e6:.0f} MB "
                          f">= 3x L2 ({l2 / 1e6:.0f} MB)",
@@ -460,6 +474,8 @@ def main():
     ap.add_argument("--graph-calls", type=int, default=1000)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="weight copies to rotate (0: enough to exceed 3x L2); small values only for profiling")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -65,6 +65,26 @@ extern "C" {
 
 /* Weight layout versions. */
 #define WQ_LAYOUT_CANONICAL 0
+/* B200_V1 (int4): the codes, scales and zero-points of 16-row bands stored as
+ * one contiguous stream per band, read front to back.  Rows are grouped in
+ * bands of 16 (the last band padded with zero codes, scale 0, zero-point 8).
+ * A band is K/128 consecutive tiles of WQ_INT4_V1_TILE_BYTES(block_size)
+ * bytes; tile s covers k = 128s .. 128s+127 of the band's 16 rows:
+ *   bytes [0, 1024): codes in warp-MMA fragment order: offset h·512 + lane·16
+ *     + 4·(2·(gi & 1) + r8) holds the 32-bit code word of band row
+ *     (lane / 4) + 8·r8 for k = 128s + 32·gi + 8·(lane % 4) + e, e = 0..7
+ *     (gi = 2h + (0|1)), code e in nibble position (e >> 1) | ((e & 1) << 2);
+ *   then bpt = max(1, 128 / block_size) scale rows [bpt][16] fp16 (for
+ *     block 256 each tile repeats its block's scales);
+ *   then zero-points [bpt][8] bytes (row 2i low nibble, row 2i+1 high);
+ *   padded to a multiple of 16 bytes.
+ * Needs K % 128 == 0 and block_size >= 32.  Built on the device by
+ * wq_repack_int4 (onnx-genai PR #1000, "Roadmap recommendation": an offline
+ * interleaving repack behind a versioned layout flag).  With this layout the
+ * GEMV ignores its scales and zeros arguments (they may be NULL). */
+#define WQ_INT4_V1_TILE_BYTES(bs) \
+  ((1024 + ((bs) >= 128 ? 1 : 128 / (bs)) * 40 + 15) / 16 * 16)
+#define WQ_LAYOUT_B200_V1 1
 
 /* ---------------------------------------------------------------------------
  * GEMV / GEMM entry points.  All device pointers; y is written, never read.
@@ -72,7 +92,9 @@ extern "C" {
 
 /* y[M,N] fp16 = x[M,K] fp16 · dequant(int4)ᵀ.
  * block_size: a power of two in [16, 256] with K % block_size == 0.
- * zeros_u4 may be NULL (z = 8).  layout must be WQ_LAYOUT_CANONICAL.
+ * zeros_u4 may be NULL (z = 8).  layout: WQ_LAYOUT_CANONICAL, or
+ * WQ_LAYOUT_B200_V1 for weights rewritten by wq_repack_int4 (then w_packed is
+ * the repacked buffer and scales_f16 / zeros_u4 are ignored).
  * M >= 1, N >= 1, K >= 1.  Errors: WQ_ERR_ARG, WQ_ERR_ALIGN, WQ_ERR_LAYOUT,
  * WQ_ERR_DEVICE, WQ_ERR_CUDA. */
 int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* scales_f16,
@@ -102,6 +124,7 @@ int gemv_bf16(const void* x_bf16, const void* w_bf16, void* y_bf16, int M, int N
  * ------------------------------------------------------------------------- */
 int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const void* zeros_u4,
                            float* w_out, int N, int K, int block_size, int layout, void* stream);
+/* (layout selects how w_packed is read: canonical or B200_V1.) */
 
 /* w_dsc NULL: coefficients decoded from the packed fields; else taken from the plane. */
 int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K, int layout,
@@ -111,9 +134,23 @@ int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K
  * Weight packing (load time).
  * ------------------------------------------------------------------------- */
 
-/* Bytes of each canonical int4 array (codes + scales + zero-points) for a
- * layout; 0 for invalid arguments. */
+/* Bytes of the int4 arrays (codes + scales + zero-points) for a layout; 0 for
+ * invalid arguments. */
 size_t wq_int4_bytes(int N, int K, int block_size, int layout);
+
+/* Bytes of the canonical int4 code array ([N][K/2]); 0 if invalid. */
+size_t wq_int4_codes_bytes(int N, int K, int layout);
+
+/* Rewrite canonical int4 weights (codes [N][K/2], scales, zeros or NULL)
+ * into layout `to_layout` at w_out (wq_int4_packed_bytes(N, K, block_size,
+ * to_layout) bytes, device, must not overlap the sources).  Errors:
+ * WQ_ERR_ARG (K % 128 != 0 or block_size < 32 for B200_V1), WQ_ERR_LAYOUT,
+ * WQ_ERR_ALIGN, WQ_ERR_CUDA. */
+int wq_repack_int4(const void* w_canonical, const void* scales_f16, const void* zeros_u4, void* w_out,
+                   int N, int K, int block_size, int to_layout, void* stream);
+
+/* Bytes of the buffer wq_repack_int4 writes (B200_V1), 0 if invalid. */
+size_t wq_int4_packed_bytes(int N, int K, int block_size, int layout);
 
 /* Bytes of a q4_K tensor and of its W_dsc plane; 0 for invalid arguments. */
 size_t wq_q4k_bytes(int N, int K);

@@ -38,18 +38,24 @@ def check(y_dev: np.ndarray, W: np.ndarray, x: np.ndarray, what: str) -> None:
 # ----------------------------------------------------------------- int4
 
 class Int4Case:
-    def __init__(self, M, N, K, bs, zeros, workload=3, s_lo=0.002, s_hi=0.01):
-        self.M, self.N, self.K, self.bs = M, N, K, bs
+    def __init__(self, M, N, K, bs, zeros, workload=3, s_lo=0.002, s_hi=0.01, layout=0):
+        self.M, self.N, self.K, self.bs, self.layout = M, N, K, bs, layout
         t = synth.int4_weights(N, K, bs, scale_lo=s_lo, scale_hi=s_hi, with_zeros=zeros, workload=workload)
         self.w, self.s, self.z = t["w_packed"], t["scales"], t["zeros"]
         self.x = synth.activations_f16(M, K, workload=workload)
         self.dw, self.ds = dev(self.w), dev(self.s)
         self.dz = dev(self.z) if self.z is not None else None
+        if layout == wq.WQ_LAYOUT_B200_V1:
+            packed = torch.full((wq.wq_int4_packed_bytes(N, K, bs, layout),), 0x5A, dtype=torch.uint8, device=DEV)
+            wq.wq_repack_int4(self.dw, self.ds, self.dz, packed, N, K, bs, layout)
+            torch.cuda.synchronize()
+            self.dw = packed
         self.dx = dev(self.x)
 
     def run(self, stream=None) -> np.ndarray:
         y = torch.empty((self.M, self.N), dtype=torch.float16, device=DEV)
-        wq.gemv_int4_blockwise(self.dx, self.dw, self.ds, self.dz, y, self.M, self.N, self.K, self.bs, stream=stream)
+        wq.gemv_int4_blockwise(self.dx, self.dw, self.ds, self.dz, y, self.M, self.N, self.K, self.bs,
+                               layout=self.layout, stream=stream)
         torch.cuda.synchronize()
         return f16_of(y).astype(np.float64)
 
@@ -120,6 +126,33 @@ class BF16Case:
 
     def X(self):
         return oracle.dequant_bf16(self.xb, self.M, self.K)
+
+
+VARIANTS = ("tc", "cc", "simple", None)
+
+
+def each_variant(run, W, x, what):
+    """Run `run()` under every forced GEMV variant (and the default); check each
+    against the oracle; return the liveness labels seen."""
+    import os
+
+    labels = {}
+    old = os.environ.get("WQ_FORCE_KERNEL")
+    try:
+        for v in VARIANTS:
+            if v is None:
+                os.environ.pop("WQ_FORCE_KERNEL", None)
+            else:
+                os.environ["WQ_FORCE_KERNEL"] = v
+            y = run()
+            labels[v or "default"] = wq.last_kernel()
+            check(y, W, x, f"{what} [{v or 'default'} -> {labels[v or 'default']}]")
+    finally:
+        if old is None:
+            os.environ.pop("WQ_FORCE_KERNEL", None)
+        else:
+            os.environ["WQ_FORCE_KERNEL"] = old
+    return labels
 
 
 def sample_rows(N: int, count: int = 48, seed: int = 0) -> np.ndarray:

@@ -55,7 +55,7 @@ def test_int4_argument_errors():
     assert rc_int4(bs=8) == _lib.WQ_ERR_ARG
     assert rc_int4(bs=512) == _lib.WQ_ERR_ARG
     assert rc_int4(K=250) == _lib.WQ_ERR_ARG
-    assert rc_int4(layout=1) == _lib.WQ_ERR_LAYOUT
+    assert rc_int4(layout=3) == _lib.WQ_ERR_LAYOUT
     assert rc_int4(x=None) == _lib.WQ_ERR_ARG
     assert rc_int4(w=A16 + 8) == _lib.WQ_ERR_ALIGN
     assert rc_int4(z=A16 + 4) == _lib.WQ_ERR_ALIGN
@@ -74,7 +74,27 @@ def test_q4k_and_bf16_argument_errors():
     assert L.wq_build_q4k_dsc(None, 4, 256, None) == _lib.WQ_ERR_ARG
 
 
+def test_v1_layout_argument_errors():
+    assert rc_int4(layout=1, K=192, bs=64) == _lib.WQ_ERR_ARG   # K % 128 != 0
+    assert rc_int4(layout=2) == _lib.WQ_ERR_LAYOUT
+    assert rc_int4(layout=1, K=256, bs=16) == _lib.WQ_ERR_ARG   # B200_V1 needs block >= 32
+    L = _lib.lib()
+    assert L.wq_repack_int4(A16, A16, None, A16, 16, 192, 64, 1, None) == _lib.WQ_ERR_ARG
+    assert L.wq_repack_int4(A16, A16, None, A16, 16, 256, 16, 1, None) == _lib.WQ_ERR_ARG
+    assert L.wq_repack_int4(A16, A16, None, A16, 16, 256, 128, 0, None) == _lib.WQ_ERR_LAYOUT
+    assert L.wq_repack_int4(A16 + 4, A16, None, A16, 16, 256, 128, 1, None) == _lib.WQ_ERR_ALIGN
+    assert L.wq_repack_int4(A16, None, None, A16, 16, 256, 128, 1, None) == _lib.WQ_ERR_ARG
+
+
 def test_size_queries():
+    assert wq.wq_int4_codes_bytes(21, 256, 0) == 21 * 128
+    assert wq.wq_int4_codes_bytes(21, 256, 1) == 0
+    assert wq.wq_int4_packed_bytes(21, 256, 128) == 2 * 2 * 1072
+    assert wq.wq_int4_packed_bytes(21, 256, 64) == 2 * 2 * 1104
+    assert wq.wq_int4_packed_bytes(21, 256, 32) == 2 * 2 * 1184
+    assert wq.wq_int4_packed_bytes(21, 192, 64) == 0
+    assert wq.wq_int4_packed_bytes(21, 256, 16) == 0
+    assert wq.wq_int4_bytes(4096, 14336, 128, 1) == 256 * 112 * 1072
     assert wq.wq_int4_bytes(256, 1024, 32) == 256 * 512 + 256 * 32 * 2 + 256 * 16
     assert wq.wq_int4_bytes(4, 96, 32) == 4 * 48 + 4 * 3 * 2 + 4 * 2  # odd block count: zero-point bytes round up
     assert wq.wq_int4_bytes(4, 100, 32) == 0

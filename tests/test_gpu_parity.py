@@ -16,7 +16,7 @@ else:
 
 import oracle  # noqa: E402
 import weight_only_quantized_q4_b200 as wq  # noqa: E402
-from _gpu import DEV, BF16Case, Int4Case, Q4KCase, check, dev, sample_rows  # noqa: E402
+from _gpu import DEV, BF16Case, Int4Case, Q4KCase, check, dev, each_variant, sample_rows  # noqa: E402
 from weight_only_quantized_q4_b200 import synth  # noqa: E402
 
 gpu = pytest.mark.gpu
@@ -62,7 +62,80 @@ def test_plane_device_host_oracle_identical(N, K):
     assert np.array_equal(host.view(np.uint32), ref.view(np.uint32))
 
 
+@gpu
+@pytest.mark.parametrize("bs,zeros,N,K", [(32, False, 5, 1024), (128, True, 23, 1024), (64, True, 16, 384),
+                                          (256, True, 33, 512)])
+def test_dequant_int4_v1_layout_bit_exact(bs, zeros, N, K):
+    """Codes repacked to B200_V1 read back (through the layout's addressing) bit-exactly."""
+    c = Int4Case(1, N, K, bs, zeros, workload=14, layout=wq.WQ_LAYOUT_B200_V1)
+    out = torch.empty((N, K), dtype=torch.float32, device=DEV)
+    wq.dequant_int4_blockwise(c.dw, c.ds, c.dz, out, N, K, bs, layout=wq.WQ_LAYOUT_B200_V1)
+    torch.cuda.synchronize()
+    assert wq.last_kernel() == "int4.dequant.v1"
+    ref = c.W().astype(np.float32)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def decode_v1(buf, N, K, bs):
+    """Read a B200_V1 int4 stream back into (q, s, z) per the layout the header
+    documents (pure Python/numpy, independent of the device code)."""
+    bpt = 1 if bs >= 128 else 128 // bs
+    tb = (1024 + bpt * 40 + 15) // 16 * 16
+    nbands = (N + 15) // 16
+    q = np.zeros((nbands * 16, K), dtype=np.int64)
+    sc = np.zeros((nbands * 16, K // bs), dtype=np.float64)
+    zp = np.zeros((nbands * 16, K // bs), dtype=np.int64)
+    for band in range(nbands):
+        for s_ in range(K // 128):
+            tile = buf[(band * (K // 128) + s_) * tb:(band * (K // 128) + s_ + 1) * tb]
+            for h in range(2):
+                for lane in range(32):
+                    g, t = lane // 4, lane % 4
+                    for j in range(4):
+                        gi, r8 = 2 * h + j // 2, j % 2
+                        word = int(tile[h * 512 + lane * 16 + 4 * j:h * 512 + lane * 16 + 4 * j + 4].view(np.uint32)[0])
+                        row = band * 16 + g + 8 * r8
+                        for e in range(8):
+                            pos = (e >> 1) | ((e & 1) << 2)
+                            q[row, 128 * s_ + 32 * gi + 8 * t + e] = (word >> (4 * pos)) & 15
+            for bt in range(bpt):
+                blk = (128 * s_ + bt * bs) // bs if bs < 128 else (128 * s_) // bs
+                svals = tile[1024 + bt * 32:1024 + bt * 32 + 32].view(np.float16).astype(np.float64)
+                zbytes = tile[1024 + 32 * bpt + bt * 8:1024 + 32 * bpt + bt * 8 + 8]
+                for r in range(16):
+                    sc[band * 16 + r, blk] = svals[r]
+                    zp[band * 16 + r, blk] = (int(zbytes[r // 2]) >> (4 * (r % 2))) & 15
+    return q, sc, zp
+
+
+@gpu
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+def test_repack_v1_layout_matches_header(bs):
+    """The repacked bytes, decoded by a plain reading of the documented layout,
+    give the oracle's weights; pad rows hold codes 0, scale 0, zero-point 8."""
+    N, K = 21, 256
+    t = synth.int4_weights(N, K, bs, scale_lo=0.01, scale_hi=0.02, with_zeros=True, workload=15)
+    packed = torch.full((wq.wq_int4_packed_bytes(N, K, bs),), 0xA5, dtype=torch.uint8, device=DEV)
+    wq.wq_repack_int4(dev(t["w_packed"]), dev(t["scales"]), dev(t["zeros"]), packed, N, K, bs)
+    torch.cuda.synchronize()
+    q, sc, zp = decode_v1(packed.cpu().numpy(), N, K, bs)
+    blk = np.arange(K) // bs
+    W = (q[:N] - zp[:N][:, blk]).astype(np.float64) * sc[:N][:, blk]
+    assert np.array_equal(W, oracle.dequant_int4(t["w_packed"], t["scales"], t["zeros"], N, K, bs))
+    assert np.all(q[N:] == 0) and np.all(sc[N:] == 0) and np.all(zp[N:] == 8)
+
+
 # ----------------------------------------------------------- GEMV, whole outputs
+
+@gpu
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8, 11])
+@pytest.mark.parametrize("N,K,bs,zeros", [(256, 1024, 32, False), (37, 2048, 128, True), (64, 4096, 64, True),
+                                          (1000, 1536, 256, False), (5, 128, 128, True)])
+def test_gemv_int4_v1_layout(M, N, K, bs, zeros):
+    c = Int4Case(M, N, K, bs, zeros, workload=16, layout=wq.WQ_LAYOUT_B200_V1)
+    labels = each_variant(c.run, c.W(), c.x, f"int4 v1 M={M} N={N} K={K} bs={bs} zp={zeros}")
+    assert ".tc." in labels["tc"] and ".v1" in labels["tc"], labels
+    assert ".simple." in labels["cc"] and ".simple." in labels["simple"], labels
 
 @gpu
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
@@ -70,7 +143,10 @@ def test_plane_device_host_oracle_identical(N, K):
                                           (64, 4096, 64, True), (1000, 1536, 256, False)])
 def test_gemv_int4_small(M, N, K, bs, zeros):
     c = Int4Case(M, N, K, bs, zeros, workload=21)
-    check(c.run(), c.W(), c.x, f"int4 M={M} N={N} K={K} bs={bs} zp={zeros}")
+    labels = each_variant(c.run, c.W(), c.x, f"int4 M={M} N={N} K={K} bs={bs} zp={zeros}")
+    if bs >= 32:
+        assert ".tc." in labels["tc"], labels
+    assert (".cc." in labels["cc"] or ".simple." in labels["cc"]) and ".simple." in labels["simple"], labels
 
 
 @gpu
@@ -79,7 +155,8 @@ def test_gemv_int4_small(M, N, K, bs, zeros):
 @pytest.mark.parametrize("dsc", [False, True])
 def test_gemv_q4k_small(M, N, K, dsc):
     c = Q4KCase(M, N, K, workload=22)
-    check(c.run(dsc), c.W(), c.x, f"q4k dsc={dsc} M={M} N={N} K={K}")
+    labels = each_variant(lambda: c.run(dsc), c.W(), c.x, f"q4k dsc={dsc} M={M} N={N} K={K}")
+    assert ".tc." in labels["tc"] and (".cc." in labels["cc"] or ".simple." in labels["cc"]), labels
 
 
 @gpu
@@ -87,7 +164,8 @@ def test_gemv_q4k_small(M, N, K, dsc):
 @pytest.mark.parametrize("N,K", [(256, 1536), (77, 6912), (300, 64)])
 def test_gemv_bf16_small(M, N, K):
     c = BF16Case(M, N, K, workload=23)
-    check(c.run(), c.W(), c.X(), f"bf16 M={M} N={N} K={K}")
+    labels = each_variant(c.run, c.W(), c.X(), f"bf16 M={M} N={N} K={K}")
+    assert ".tc." in labels["tc"] and (".cc." in labels["cc"] or ".simple." in labels["cc"]), labels
 
 
 @gpu
@@ -97,18 +175,19 @@ def test_gemv_bf16_small(M, N, K):
 @pytest.mark.parametrize("offset", [0, 1])
 def test_gemv_bf16_odd_k_and_offsets(K, M, N, offset):
     c = BF16Case(M, N, K, offset=offset, workload=24)
-    check(c.run(), c.W(), c.X(), f"bf16 odd-K M={M} N={N} K={K} offset={offset}")
+    each_variant(c.run, c.W(), c.X(), f"bf16 odd-K M={M} N={N} K={K} offset={offset}")
 
 
 @gpu
 @pytest.mark.parametrize("M", [9, 16, 17])
 def test_gemv_larger_batches(M):
     c = Int4Case(M, 96, 1024, 128, True, workload=25)
-    check(c.run(), c.W(), c.x, f"int4 M={M}")
+    each_variant(c.run, c.W(), c.x, f"int4 M={M}")
     q = Q4KCase(M, 40, 512, workload=25)
-    check(q.run(False), q.W(), q.x, f"q4k M={M}")
+    each_variant(lambda: q.run(False), q.W(), q.x, f"q4k M={M}")
+    each_variant(lambda: q.run(True), q.W(), q.x, f"q4k dsc M={M}")
     b = BF16Case(M, 50, 256, workload=25)
-    check(b.run(), b.W(), b.X(), f"bf16 M={M}")
+    each_variant(b.run, b.W(), b.X(), f"bf16 M={M}")
 
 
 # ----------------------------------------------------------- closed forms on the device
@@ -153,7 +232,7 @@ def test_uses_given_stream_and_labels():
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         y = c.run()
-    assert "int4.gemv.cc" in wq.last_kernel()
+    assert "int4.gemv.tc" in wq.last_kernel()
     check(y, c.W(), c.x, "int4 on a side stream")
     wq.wq_device_status()
 
@@ -168,12 +247,12 @@ FULL_BF16 = [(1536, 1536), (256, 1536), (1536, 6912), (151936, 1536)]
 @gpu
 @pytest.mark.parametrize("M", [1, 4])
 @pytest.mark.parametrize("N,K", FULL_INT4)
-def test_full_int4_b128_sampled(M, N, K):
-    c = Int4Case(M, N, K, 128, True, workload=3)
-    y = c.run()
-    assert ".gemv." in wq.last_kernel()
+@pytest.mark.parametrize("layout", [0, 1])
+def test_full_int4_b128_sampled(M, N, K, layout):
+    c = Int4Case(M, N, K, 128, True, workload=3, layout=layout)
     rows = sample_rows(N)
-    check(y[:, rows], c.W(rows), c.x, f"int4 full {N}x{K} M={M}")
+    Wr = c.W(rows)
+    each_variant(lambda: c.run()[:, rows], Wr, c.x, f"int4 full {N}x{K} M={M}")
 
 
 @gpu
@@ -188,9 +267,9 @@ def test_full_int4_b32_config():
 @pytest.mark.parametrize("dsc", [False, True])
 def test_full_q4k_sampled(M, N, K, dsc):
     c = Q4KCase(M, N, K, workload=4)
-    y = c.run(dsc)
     rows = sample_rows(N)
-    check(y[:, rows], c.W(rows), c.x, f"q4k dsc={dsc} full {N}x{K} M={M}")
+    Wr = c.W(rows)
+    each_variant(lambda: c.run(dsc)[:, rows], Wr, c.x, f"q4k dsc={dsc} full {N}x{K} M={M}")
 
 
 @gpu
@@ -198,6 +277,6 @@ def test_full_q4k_sampled(M, N, K, dsc):
 @pytest.mark.parametrize("N,K", FULL_BF16)
 def test_full_bf16_sampled(M, N, K):
     c = BF16Case(M, N, K, workload=2)
-    y = c.run()
     rows = sample_rows(N)
-    check(y[:, rows], c.W(rows), c.X(), f"bf16 full {N}x{K} M={M}")
+    Wr = c.W(rows)
+    each_variant(lambda: c.run()[:, rows], Wr, c.X(), f"bf16 full {N}x{K} M={M}")

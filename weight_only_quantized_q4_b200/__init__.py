@@ -6,6 +6,8 @@ The kernels live in libwq.so (C ABI in include/wq.h); this package is a thin
 ctypes binding with the same entry-point names.
 """
 from .api import (  # noqa: F401
+    WQ_LAYOUT_B200_V1,
+    WQ_LAYOUT_CANONICAL,
     WQError,
     dequant_int4_blockwise,
     dequant_q4k,
@@ -19,6 +21,9 @@ from .api import (  # noqa: F401
     wq_build_q4k_dsc_device,
     wq_device_status,
     wq_int4_bytes,
+    wq_int4_codes_bytes,
+    wq_int4_packed_bytes,
+    wq_repack_int4,
     wq_layout_version,
     wq_q4k_bytes,
     wq_q4k_dsc_bytes,

@@ -22,6 +22,7 @@ WQ_ERR_DEVICE = -5
 WQ_ERR_TIMEOUT = -6
 WQ_ERR_UNSUPPORTED = -7
 WQ_LAYOUT_CANONICAL = 0
+WQ_LAYOUT_B200_V1 = 1
 
 _ERRNAMES = {v: k for k, v in dict(globals()).items() if k.startswith("WQ_ERR_")}
 
@@ -35,6 +36,9 @@ SIGNATURES = {
     "dequant_int4_blockwise": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "dequant_q4k": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "wq_int4_bytes": (_sz, [_i, _i, _i, _i]),
+    "wq_int4_codes_bytes": (_sz, [_i, _i, _i]),
+    "wq_repack_int4": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "wq_int4_packed_bytes": (_sz, [_i, _i, _i, _i]),
     "wq_q4k_bytes": (_sz, [_i, _i]),
     "wq_q4k_dsc_bytes": (_sz, [_i, _i]),
     "wq_build_q4k_dsc": (_i, [_vp, _i, _i, _vp]),

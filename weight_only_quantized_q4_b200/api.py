@@ -11,7 +11,7 @@ import ctypes
 
 import numpy as np
 
-from ._lib import WQ_LAYOUT_CANONICAL, WQError, _check, last_error, last_kernel, lib  # noqa: F401
+from ._lib import WQ_LAYOUT_B200_V1, WQ_LAYOUT_CANONICAL, WQError, _check, last_error, last_kernel, lib  # noqa: F401
 
 
 def _ptr(t):
@@ -63,6 +63,19 @@ def dequant_q4k(w_q4k, w_dsc, w_out, N, K, layout=WQ_LAYOUT_CANONICAL, stream=No
 
 def wq_int4_bytes(N, K, block_size, layout=WQ_LAYOUT_CANONICAL) -> int:
     return int(lib().wq_int4_bytes(N, K, block_size, layout))
+
+
+def wq_int4_codes_bytes(N, K, layout=WQ_LAYOUT_CANONICAL) -> int:
+    return int(lib().wq_int4_codes_bytes(N, K, layout))
+
+
+def wq_int4_packed_bytes(N, K, block_size, layout=WQ_LAYOUT_B200_V1) -> int:
+    return int(lib().wq_int4_packed_bytes(N, K, block_size, layout))
+
+
+def wq_repack_int4(w_canonical, scales, zeros, w_out, N, K, block_size, to_layout=WQ_LAYOUT_B200_V1, stream=None):
+    _check(lib().wq_repack_int4(_ptr(w_canonical), _ptr(scales), _ptr(zeros), _ptr(w_out), N, K, block_size,
+                                to_layout, _stream(stream)), "wq_repack_int4")
 
 
 def wq_q4k_bytes(N, K) -> int:

@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -16,6 +17,7 @@
 #include "../../include/wq.h"
 #include "gemv_cc.cuh"
 #include "gemv_simple.cuh"
+#include "gemv_tc.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -299,6 +301,161 @@ std::string cc_label(const char* fmt, int M, int KS, const char* extra) {
   return buf;
 }
 
+// ---------------------------------------------------------------------------
+// tensor-pipe GEMV (warp MMA, register operands): planner and launcher
+// ---------------------------------------------------------------------------
+struct TCPlan {
+  TCParams p{};
+  int threads = 0, grid = 0, smem = 0;
+};
+
+bool plan_tc(Fmt f, int M, int N, int K, long long row_bytes, int nb, int zb, int block_size, int layout,
+             int sms, TCPlan* plan) {
+  if (M < 1 || M > 8) return false;
+  int Kc = 0;
+  long long seg_full = 0;  // weight bytes per row of a full stage
+  // WQ_TC_KC overrides the k-extent of a stage (tuning; rounded to the format's unit)
+  const char* kc_env = std::getenv("WQ_TC_KC");
+  const int kc_req = kc_env ? std::atoi(kc_env) : 0;
+  int v1_tb = 0, v1_tpb = 0, v1_tps = 0;
+  if (f == Fmt::Int4 && layout == WQ_LAYOUT_B200_V1) {
+    if (block_size < 32 || K % 128) return false;
+    v1_tb = int4_v1_tile_bytes(block_size);
+    v1_tpb = K / 128;
+    // tiles per stage: the largest divisor of the band's tile count within
+    // the stage budget (WQ_TC_KC, in k, overrides the budget)
+    const int cap_tiles = std::max(1, kc_req > 0 ? kc_req / 128 : (24 * 1024) / v1_tb);
+    for (int d = 1; d <= v1_tpb; ++d)
+      if (v1_tpb % d == 0 && d <= cap_tiles) v1_tps = d;
+    Kc = 128 * v1_tps;
+    seg_full = 0;
+  } else if (f == Fmt::Int4) {
+    if (block_size < 32 || K % 128) return false;
+    Kc = std::max(std::max(block_size, 128), kc_req > 0 ? kc_req / 256 * 256 : 1024);
+    Kc = std::min(Kc, K);
+    seg_full = Kc / 2;
+  } else if (f == Fmt::BF16) {
+    if (K % 64) return false;
+    Kc = std::min(kc_req > 0 ? std::max(64, kc_req / 64 * 64) : 2048, K);
+    seg_full = 2ll * Kc;
+  } else {
+    if (K % 256) return false;
+    Kc = std::min(kc_req > 0 ? std::max(256, kc_req / 256 * 256) : 1024, K);
+    seg_full = (Kc / 256) * 144;
+  }
+  TCParams& p = plan->p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nb = nb;
+  p.zb = zb;
+  p.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
+  p.row_bytes = row_bytes;
+  p.rpb = (f == Fmt::Q4K || f == Fmt::Q4KDsc) ? 15 : 16;
+  p.n_bands = (N + p.rpb - 1) / p.rpb;
+  p.Kc = Kc;
+  p.pitch = static_cast<int>(seg_full + 16);
+  p.n_kst = (K + Kc - 1) / Kc;
+  p.v1_tb = v1_tb;
+  p.v1_tpb = v1_tpb;
+  p.v1_tps = v1_tps;
+  long long off = layout == WQ_LAYOUT_B200_V1 ? round16(1ll * v1_tps * v1_tb) : round16(16ll * p.pitch);
+  p.off_x = static_cast<int>(off);
+  // Activations resident for the whole kernel when small (one copy per CTA
+  // instead of one per stage); WQ_TC_XRES=0/1 overrides (tuning).
+  const char* xr_env = std::getenv("WQ_TC_XRES");
+  const long long x_bytes = 2ll * M * K;
+  p.x_res = xr_env ? (std::atoi(xr_env) != 0 && x_bytes <= 96 * 1024) : (x_bytes <= 64 * 1024);
+  if (!p.x_res) off += round16(2ll * M * Kc);
+  p.off_plane = static_cast<int>(off);
+  p.plane_stride = round16(8ll * p.rpb + 16);
+  if (f == Fmt::Q4KDsc) off += static_cast<long long>(p.plane_stride) * (Kc / 32);
+  p.stage_bytes = static_cast<int>(round16(off));
+  // WQ_TC_W overrides the number of consumer warps (tuning)
+  // one CTA per SM for the B200_V1 stream needs 16 consumer warps (4 per
+  // scheduler) to cover the load / MMA latency chains of the tile loop
+  const char* w_env = std::getenv("WQ_TC_W");
+  const int W = w_env ? std::max(1, std::min(16, std::atoi(w_env))) : (layout == WQ_LAYOUT_B200_V1 ? 16 : 8);
+  p.W = W;
+  long long meta = 0;
+  if (f == Fmt::Int4 && layout == WQ_LAYOUT_B200_V1) {
+    meta = 0;  // scales and zero-points travel inside the tiles
+  } else if (f == Fmt::Int4 && block_size >= 128) {
+    meta = 16ll * 16 * nb;  // one 16-byte entry per (block, row)
+  } else if (f == Fmt::Int4) {
+    p.meta_zoff = round16(2ll * 16 * nb);
+    meta = p.meta_zoff + round16(16ll * zb);
+  }
+  const long long xres = p.x_res ? round16(x_bytes) : 0;
+  const long long tail = meta + xres + 2ll * W * 16 * 8 * 4 + 2 * 16 * 8 + 16;
+  // WQ_TC_NS overrides the ring depth (tuning); WQ_TC_CTAS the CTAs per SM (1 or 2)
+  const char* ns_env = std::getenv("WQ_TC_NS");
+  const char* cps_env = std::getenv("WQ_TC_CTAS");
+  const int ns_cap = ns_env ? std::max(2, std::atoi(ns_env)) : 8;
+  // B200_V1 streams want one CTA per SM with the deepest ring (the CTA's data is
+  // one contiguous range, so almost all of it can be requested at once).
+  int ctas_per_sm = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : (layout == WQ_LAYOUT_B200_V1 ? 1 : 2);
+  int NS = static_cast<int>(std::min<long long>(ns_cap, (kSmemPerSm / ctas_per_sm - tail) / p.stage_bytes));
+  if (layout == WQ_LAYOUT_B200_V1 && ctas_per_sm == 1 && !ns_env)
+    NS = static_cast<int>(std::min<long long>(16, (kSmemPerSm - tail) / p.stage_bytes));
+  if (NS < 4 && ctas_per_sm == 2) {
+    ctas_per_sm = 1;
+    NS = static_cast<int>(std::min<long long>(std::max(ns_cap, 16), (kSmemPerSm - tail) / p.stage_bytes));
+  }
+  if (NS < 2) return false;
+  p.NS = NS;
+  p.off_meta = NS * p.stage_bytes;
+  p.off_xres = static_cast<int>(p.off_meta + meta);
+  p.off_red = static_cast<int>(p.off_xres + xres);
+  plan->threads = (W + 1) * 32;
+  plan->grid = std::max(1, std::min(p.n_bands, ctas_per_sm * sms));
+  plan->smem = static_cast<int>(p.off_red + tail - meta - xres);
+  return true;
+}
+
+using TCKernel = void (*)(const TCParams);
+
+TCKernel tc_kernel(Fmt f, int layout, bool bigb) {
+  const bool v1 = layout == WQ_LAYOUT_B200_V1;
+  switch (f) {
+    case Fmt::Int4:
+      if (v1) return bigb ? &gemv_tc_kernel<Fmt::Int4, true, true> : &gemv_tc_kernel<Fmt::Int4, true, false>;
+      return bigb ? &gemv_tc_kernel<Fmt::Int4, false, true> : &gemv_tc_kernel<Fmt::Int4, false, false>;
+    case Fmt::Q4K: return &gemv_tc_kernel<Fmt::Q4K, false, false>;
+    case Fmt::Q4KDsc: return &gemv_tc_kernel<Fmt::Q4KDsc, false, false>;
+    case Fmt::BF16: return &gemv_tc_kernel<Fmt::BF16, false, false>;
+  }
+  return nullptr;
+}
+
+int launch_tc(Fmt f, int layout, const TCPlan& plan, cudaStream_t st) {
+  static std::mutex mu;
+  static bool configured[8][64] = {};
+  const bool bigb = f == Fmt::Int4 && plan.p.block_shift >= 7;
+  TCKernel fn = tc_kernel(f, layout, bigb);
+  const int slot = f == Fmt::Int4 ? 4 + (layout == WQ_LAYOUT_B200_V1 ? 2 : 0) + (bigb ? 1 : 0) : static_cast<int>(f);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[slot][dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[slot][dev] = true;
+    }
+  }
+  fn<<<plan.grid, plan.threads, plan.smem, st>>>(plan.p);
+  return launch_check("gemv_tc launch");
+}
+
+// WQ_FORCE_KERNEL = "cc" | "tc" | "simple" pins the GEMV variant (A/B runs and
+// per-variant parity tests); unset means the default choice below.
+const char* forced_variant() {
+  const char* v = std::getenv("WQ_FORCE_KERNEL");
+  return (v && *v) ? v : nullptr;
+}
+
 template <Fmt F>
 int launch_simple(const SimpleParams& sp, int M, int sms, cudaStream_t st) {
   const int threads = 256;
@@ -322,7 +479,7 @@ int launch_simple(const SimpleParams& sp, int M, int sms, cudaStream_t st) {
 template <Fmt F>
 int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros,
              const uint8_t* plane, void* y, int M, int N, int K, long long row_bytes, int nb, int zb,
-             int block_size, bool fast_ok, cudaStream_t st) {
+             int block_size, bool fast_ok, cudaStream_t st, int layout = WQ_LAYOUT_CANONICAL) {
   DeviceInfo di;
   int rc = device_info(&di);
   if (rc) return rc;
@@ -332,8 +489,28 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     const int mc = std::min(8, M - m0);
     const void* xc = static_cast<const uint8_t*>(x) + static_cast<long long>(m0) * K * x_elt;
     void* yc = static_cast<uint8_t*>(y) + static_cast<long long>(m0) * N * 2;
+    const char* force = forced_variant();
+    const bool want_tc = force ? std::strcmp(force, "tc") == 0 : true;
+    const bool want_cc = force ? std::strcmp(force, "cc") == 0 : true;
+    TCPlan tplan;
+    if (want_tc && fast_ok && aligned16(xc) &&
+        plan_tc(F, mc, N, K, row_bytes, nb, zb, block_size, layout, di.sms, &tplan)) {
+      tplan.p.x = xc;
+      tplan.p.w = w;
+      tplan.p.scales = scales;
+      tplan.p.zeros = zeros;
+      tplan.p.plane = plane;
+      tplan.p.y = yc;
+      rc = launch_tc(F, layout, tplan, st);
+      if (rc) return rc;
+      char buf[64];
+      std::snprintf(buf, sizeof(buf), "%s.gemv.tc.m%d%s%s", fmt_name, mc, layout == WQ_LAYOUT_B200_V1 ? ".v1" : "",
+                    M > 8 ? ".chunked" : "");
+      label = buf;
+      continue;
+    }
     CCPlan plan;
-    const bool use_cc = fast_ok && aligned16(xc) &&
+    const bool use_cc = want_cc && fast_ok && layout == WQ_LAYOUT_CANONICAL && aligned16(xc) &&
                         plan_cc(F, mc, N, K, row_bytes, nb, zb, block_size, zeros != nullptr, di.sms, &plan);
     if (use_cc) {
       plan.p.x = xc;
@@ -359,6 +536,7 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
       sp.nb = nb;
       sp.zb = zb;
       sp.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
+      sp.layout = layout;
       rc = launch_simple<F>(sp, mc, di.sms, st);
       if (rc) return rc;
       char buf[64];
@@ -376,10 +554,13 @@ int check_dims(int M, int N, int K) {
 }
 
 int check_int4(int K, int block_size, int layout) {
-  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown int4 layout version");
+  if (layout != WQ_LAYOUT_CANONICAL && layout != WQ_LAYOUT_B200_V1)
+    return fail(WQ_ERR_LAYOUT, "unknown int4 layout version");
   if (block_size < 16 || block_size > 256 || (block_size & (block_size - 1)))
     return fail(WQ_ERR_ARG, "block_size must be a power of two in [16, 256]");
   if (K % block_size) return fail(WQ_ERR_ARG, "K must be a multiple of block_size");
+  if (layout == WQ_LAYOUT_B200_V1 && (K % 128 || block_size < 32))
+    return fail(WQ_ERR_ARG, "the B200_V1 int4 layout needs K % 128 == 0 and block_size >= 32");
   return WQ_OK;
 }
 
@@ -403,8 +584,14 @@ int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* sca
   int rc = check_dims(M, N, K);
   if (rc) return rc;
   if ((rc = check_int4(K, block_size, layout))) return rc;
-  if (!x_f16 || !w_packed || !scales_f16 || !y_f16) return fail(WQ_ERR_ARG, "gemv_int4_blockwise: null pointer");
-  if (!aligned16(x_f16) || !aligned16(w_packed) || !aligned16(scales_f16) || !aligned16(y_f16) ||
+  const bool v1 = layout == WQ_LAYOUT_B200_V1;
+  if (v1) {
+    scales_f16 = nullptr;  // carried inside the repacked stream
+    zeros_u4 = nullptr;
+  }
+  if (!x_f16 || !w_packed || (!v1 && !scales_f16) || !y_f16)
+    return fail(WQ_ERR_ARG, "gemv_int4_blockwise: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_packed) || (scales_f16 && !aligned16(scales_f16)) || !aligned16(y_f16) ||
       (zeros_u4 && !aligned16(zeros_u4)))
     return fail(WQ_ERR_ALIGN, "gemv_int4_blockwise: device pointers must be 16-byte aligned");
   const int nb = K / block_size;
@@ -413,7 +600,8 @@ int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* sca
   const bool fast = (row_bytes % 16) == 0;
   return run_gemv<Fmt::Int4>("int4", x_f16, static_cast<const uint8_t*>(w_packed),
                              static_cast<const uint8_t*>(scales_f16), static_cast<const uint8_t*>(zeros_u4), nullptr,
-                             y_f16, M, N, K, row_bytes, nb, zb, block_size, fast, static_cast<cudaStream_t>(stream));
+                             y_f16, M, N, K, row_bytes, nb, zb, block_size, fast, static_cast<cudaStream_t>(stream),
+                             layout);
 }
 
 int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K, int layout, void* stream) {
@@ -460,8 +648,14 @@ int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const v
   int rc = check_dims(1, N, K);
   if (rc) return rc;
   if ((rc = check_int4(K, block_size, layout))) return rc;
-  if (!w_packed || !scales_f16 || !w_out) return fail(WQ_ERR_ARG, "dequant_int4_blockwise: null pointer");
-  if (!aligned16(w_packed) || !aligned16(scales_f16) || (zeros_u4 && !aligned16(zeros_u4)) || !aligned16(w_out))
+  const bool v1 = layout == WQ_LAYOUT_B200_V1;
+  if (v1) {
+    scales_f16 = nullptr;
+    zeros_u4 = nullptr;
+  }
+  if (!w_packed || (!v1 && !scales_f16) || !w_out) return fail(WQ_ERR_ARG, "dequant_int4_blockwise: null pointer");
+  if (!aligned16(w_packed) || (scales_f16 && !aligned16(scales_f16)) || (zeros_u4 && !aligned16(zeros_u4)) ||
+      !aligned16(w_out))
     return fail(WQ_ERR_ALIGN, "dequant_int4_blockwise: device pointers must be 16-byte aligned");
   DeviceInfo di;
   if ((rc = device_info(&di))) return rc;
@@ -470,9 +664,9 @@ int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const v
   const int grid = static_cast<int>(std::min<long long>((words + 255) / 256, di.sms * 32ll));
   dequant_int4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t*>(w_packed), static_cast<const uint8_t*>(scales_f16),
-      static_cast<const uint8_t*>(zeros_u4), w_out, N, K, nb, (nb + 1) / 2, ilog2_int(block_size));
+      static_cast<const uint8_t*>(zeros_u4), w_out, N, K, nb, (nb + 1) / 2, ilog2_int(block_size), layout);
   if ((rc = launch_check("dequant_int4 launch"))) return rc;
-  set_last_kernel("int4.dequant");
+  set_last_kernel(layout == WQ_LAYOUT_B200_V1 ? "int4.dequant.v1" : "int4.dequant");
   return WQ_OK;
 }
 
@@ -492,6 +686,33 @@ int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K
       static_cast<const uint8_t*>(w_q4k), static_cast<const uint8_t*>(w_dsc), w_out, N, K);
   if ((rc = launch_check("dequant_q4k launch"))) return rc;
   set_last_kernel(w_dsc ? "q4k_dsc.dequant" : "q4k.dequant");
+  return WQ_OK;
+}
+
+int wq_repack_int4(const void* w_canonical, const void* scales_f16, const void* zeros_u4, void* w_out, int N, int K,
+                   int block_size, int to_layout, void* stream) {
+  if (N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "wq_repack_int4: need N, K > 0");
+  if (!w_canonical || !scales_f16 || !w_out) return fail(WQ_ERR_ARG, "wq_repack_int4: null pointer");
+  if (to_layout != WQ_LAYOUT_B200_V1) return fail(WQ_ERR_LAYOUT, "wq_repack_int4: target layout must be B200_V1");
+  if (block_size < 32 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size)
+    return fail(WQ_ERR_ARG, "wq_repack_int4: B200_V1 needs a power-of-two block in [32, 256] and K % 128 == 0");
+  if (!aligned16(w_canonical) || !aligned16(scales_f16) || (zeros_u4 && !aligned16(zeros_u4)) || !aligned16(w_out))
+    return fail(WQ_ERR_ALIGN, "wq_repack_int4: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const long long tiles = static_cast<long long>((N + 15) / 16) * (K / 128);
+  const int g1 = static_cast<int>(std::min<long long>((tiles * 64 + 255) / 256, di.sms * 32ll));
+  repack_int4_v1_codes_kernel<<<g1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_canonical), static_cast<uint8_t*>(w_out), N, K, block_size);
+  if ((rc = launch_check("repack_int4 codes launch"))) return rc;
+  const long long items = tiles * int4_v1_bpt(block_size) * 8;
+  const int g2 = static_cast<int>(std::min<long long>((items + 255) / 256, di.sms * 32ll));
+  repack_int4_v1_meta_kernel<<<g2, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(scales_f16), static_cast<const uint8_t*>(zeros_u4), static_cast<uint8_t*>(w_out), N,
+      K, block_size);
+  if ((rc = launch_check("repack_int4 meta launch"))) return rc;
+  set_last_kernel("int4.repack.v1");
   return WQ_OK;
 }
 

@@ -137,7 +137,7 @@ __device__ __forceinline__ void issue_stage(const CCParams& p, uint8_t* dst, uin
     total += (n_chunks - n_pl8) * pl_len0 + n_pl8 * pl_len8;
   }
   if (lane == 0) {
-    fence_proxy_async_smem();
+    // slot reuse is ordered by the __syncthreads that ended its last use
     mbar_arrive_expect_tx(bar, total);
     bulk_g2s_stream(dst, p.w + static_cast<long long>(r0) * p.row_bytes, wbytes, bar, policy);
     if constexpr (F == Fmt::Int4) {

@@ -14,6 +14,40 @@
 
 namespace wq {
 
+// B200_V1 stores the eight codes of a word in the order k0 k2 k4 k6 k1 k3 k5 k7
+// (nibble positions 0..7), so that the pair extractions lo4 / hi4 / lo4(>>8) /
+// hi4(>>8) yield (k0,k1) (k2,k3) (k4,k5) (k6,k7): consecutive activation
+// pairs.  Nibble position of code k (0..7) inside such a word:
+__host__ __device__ __forceinline__ int int4_v1_nibble_pos(int k) { return (k >> 1) | ((k & 1) << 2); }
+
+// B200_V1 int4 stream geometry (see include/wq.h): bands of 16 rows, K/128
+// tiles per band, each tile = 1024 code bytes + bpt·16 fp16 scales + bpt·8
+// zero-point bytes, padded to 16 bytes.
+__host__ __device__ __forceinline__ int int4_v1_bpt(int bs) { return bs >= 128 ? 1 : 128 / bs; }
+__host__ __device__ __forceinline__ int int4_v1_tile_bytes(int bs) {
+  return (1024 + int4_v1_bpt(bs) * 40 + 15) / 16 * 16;
+}
+__host__ __device__ __forceinline__ long long int4_v1_tile_offset(long long row, int k, int K, int bs) {
+  return ((row >> 4) * (K / 128) + (k >> 7)) * static_cast<long long>(int4_v1_tile_bytes(bs));
+}
+// Byte offset of the 32-bit code word covering k = k8 .. k8+7 (k8 % 8 == 0) of `row`.
+__host__ __device__ __forceinline__ long long int4_v1_word_offset(long long row, int k8, int K, int bs) {
+  const int r = static_cast<int>(row & 15);
+  const int g = r & 7, r8 = r >> 3;
+  const int kk = k8 & 127;
+  const int gi = kk >> 5, t = (kk & 31) >> 3;
+  return int4_v1_tile_offset(row, k8, K, bs) + (gi >> 1) * 512 + (4 * g + t) * 16 + 4 * (2 * (gi & 1) + r8);
+}
+// Block slot inside a tile for k (0 when blocks span >= 128 k).
+__host__ __device__ __forceinline__ int int4_v1_block_in_tile(int k, int bs) { return bs >= 128 ? 0 : (k & 127) / bs; }
+__host__ __device__ __forceinline__ long long int4_v1_scale_offset(long long row, int k, int K, int bs) {
+  return int4_v1_tile_offset(row, k, K, bs) + 1024 + (int4_v1_block_in_tile(k, bs) * 16 + (row & 15)) * 2;
+}
+__host__ __device__ __forceinline__ long long int4_v1_zero_offset(long long row, int k, int K, int bs) {
+  return int4_v1_tile_offset(row, k, K, bs) + 1024 + 32 * int4_v1_bpt(bs) + int4_v1_block_in_tile(k, bs) * 8 +
+         ((row & 15) >> 1);
+}
+
 struct SimpleParams {
   const void* x;
   const uint8_t* w;
@@ -23,6 +57,7 @@ struct SimpleParams {
   void* y;
   int M, N, K;
   int nb, zb, block_shift;
+  int layout;  // int4: 0 canonical, 1 B200_V1 (codes, scales and zero-points all in w)
 };
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float((b16 & 0xFFFFu) << 16); }
@@ -31,14 +66,24 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_
 template <Fmt F>
 __device__ __forceinline__ float weight_scalar(const SimpleParams& p, int row, int k) {
   if constexpr (F == Fmt::Int4) {
-    const uint32_t byte = p.w[static_cast<long long>(row) * (p.K / 2) + (k >> 1)];
-    const uint32_t q = (k & 1) ? (byte >> 4) : (byte & 15u);
-    const int b = k >> p.block_shift;
-    const uint32_t sb = reinterpret_cast<const uint16_t*>(p.scales)[static_cast<long long>(row) * p.nb + b];
-    uint32_t z = 8u;
-    if (p.zeros) {
-      const uint32_t zb = p.zeros[static_cast<long long>(row) * p.zb + (b >> 1)];
-      z = (b & 1) ? (zb >> 4) : (zb & 15u);
+    uint32_t q, sb, z = 8u;
+    if (p.layout == 1) {
+      const int bs = 1 << p.block_shift;
+      const int pos = int4_v1_nibble_pos(k & 7);
+      const uint32_t byte = p.w[int4_v1_word_offset(row, k & ~7, p.K, bs) + (pos >> 1)];
+      q = (pos & 1) ? (byte >> 4) : (byte & 15u);
+      sb = *reinterpret_cast<const uint16_t*>(p.w + int4_v1_scale_offset(row, k, p.K, bs));
+      const uint32_t zbyte = p.w[int4_v1_zero_offset(row, k, p.K, bs)];
+      z = (row & 1) ? (zbyte >> 4) : (zbyte & 15u);
+    } else {
+      const uint32_t byte = p.w[static_cast<long long>(row) * (p.K / 2) + (k >> 1)];
+      q = (k & 1) ? (byte >> 4) : (byte & 15u);
+      const int b = k >> p.block_shift;
+      sb = reinterpret_cast<const uint16_t*>(p.scales)[static_cast<long long>(row) * p.nb + b];
+      if (p.zeros) {
+        const uint32_t zb = p.zeros[static_cast<long long>(row) * p.zb + (b >> 1)];
+        z = (b & 1) ? (zb >> 4) : (zb & 15u);
+      }
     }
     return static_cast<float>(static_cast<int>(q) - static_cast<int>(z)) * h16_to_f32(sb);
   } else if constexpr (F == Fmt::Q4K || F == Fmt::Q4KDsc) {
@@ -119,30 +164,42 @@ __device__ __forceinline__ float code_of(uint32_t pair, int h, bool high_class) 
 }
 
 __global__ void dequant_int4_kernel(const uint8_t* w, const uint8_t* scales, const uint8_t* zeros, float* out,
-                                    int N, int K, int nb, int zb, int block_shift) {
+                                    int N, int K, int nb, int zb, int block_shift, int layout) {
   const long long words_per_row = K / 8;
   const long long total = static_cast<long long>(N) * words_per_row;
   for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long row = t / words_per_row;
     const int wd = static_cast<int>(t - row * words_per_row);
-    const uint32_t v = reinterpret_cast<const uint32_t*>(w + row * (K / 2))[wd];
-    const uint32_t pr[4] = {lo4(v), hi4(v), lo4(v >> 8), hi4(v >> 8)};  // (n0,n4) (n1,n5) (n2,n6) (n3,n7)
+    const int bs = 1 << block_shift;
+    const uint32_t v = layout == 1 ? *reinterpret_cast<const uint32_t*>(w + int4_v1_word_offset(row, 8 * wd, K, bs))
+                                   : reinterpret_cast<const uint32_t*>(w + row * (K / 2))[wd];
+    // pairs by nibble position: (p0,p4) (p1,p5) (p2,p6) (p3,p7)
+    const uint32_t pr[4] = {lo4(v), hi4(v), lo4(v >> 8), hi4(v >> 8)};
     const int k0 = 8 * wd;
     const int b = k0 >> block_shift;  // a word never straddles a block (block >= 16)
-    const float s = h16_to_f32(reinterpret_cast<const uint16_t*>(scales)[row * nb + b]);
-    float z = 8.f;
-    if (zeros) {
-      const uint32_t zbyte = zeros[row * zb + (b >> 1)];
-      z = static_cast<float>((b & 1) ? (zbyte >> 4) : (zbyte & 15u));
+    float s, z = 8.f;
+    if (layout == 1) {
+      s = h16_to_f32(*reinterpret_cast<const uint16_t*>(w + int4_v1_scale_offset(row, k0, K, bs)));
+      const uint32_t zbyte = w[int4_v1_zero_offset(row, k0, K, bs)];
+      z = static_cast<float>((row & 1) ? (zbyte >> 4) : (zbyte & 15u));
+    } else {
+      s = h16_to_f32(reinterpret_cast<const uint16_t*>(scales)[row * nb + b]);
+      if (zeros) {
+        const uint32_t zbyte = zeros[row * zb + (b >> 1)];
+        z = static_cast<float>((b & 1) ? (zbyte >> 4) : (zbyte & 15u));
+      }
     }
     float* o = out + row * K + k0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const bool high = (i & 1) != 0;
-      const int e0 = (i >> 1) * 2 + (high ? 1 : 0);  // nibble index of the pair's low half
+      const int p0 = (i >> 1) * 2 + (high ? 1 : 0);  // nibble position of the pair's low half
+      // canonical: position == k; B200_V1: position p holds k = 2·(p & 3) + (p >> 2)
+      const int e0 = layout == 1 ? 2 * (p0 & 3) + (p0 >> 2) : p0;
+      const int e1 = layout == 1 ? 2 * ((p0 + 4) & 3) + ((p0 + 4) >> 2) : p0 + 4;
       o[e0] = (code_of(pr[i], 0, high) - z) * s;
-      o[e0 + 4] = (code_of(pr[i], 1, high) - z) * s;
+      o[e1] = (code_of(pr[i], 1, high) - z) * s;
     }
   }
 }
@@ -193,6 +250,78 @@ __global__ void dequant_q4k_kernel(const uint8_t* w, const uint8_t* plane, float
     o1[2] = fmaf(A1, code_of(p1, 1, true), B1);
     o1[1] = fmaf(A1, code_of(p3, 0, true), B1);
     o1[3] = fmaf(A1, code_of(p3, 1, true), B1);
+  }
+}
+
+// Canonical int4 -> B200_V1, codes: thread per 16-byte code chunk of a tile
+// (rows past N get zero codes).
+__global__ void repack_int4_v1_codes_kernel(const uint8_t* w, uint8_t* out, int N, int K, int bs) {
+  const long long n_bands = (N + 15) / 16;
+  const int tpb = K / 128;
+  const int tb = int4_v1_tile_bytes(bs);
+  const long long chunks = n_bands * tpb * 64;
+  for (long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
+       c += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long tile = c >> 6;  // band * tpb + s
+    const int q = static_cast<int>(c & 63);
+    const long long band = tile / tpb;
+    const int s = static_cast<int>(tile - band * tpb);
+    const int h = q >> 5, lane = q & 31;
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gi = 2 * h + (j >> 1), r8 = j & 1;
+      const long long row = 16 * band + g + 8 * r8;
+      const int k = 128 * s + 32 * gi + 8 * t;
+      const uint32_t cw = row < N ? *reinterpret_cast<const uint32_t*>(w + row * (K / 2) + k / 2) : 0u;
+      uint32_t o = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o |= ((cw >> (4 * e)) & 15u) << (4 * int4_v1_nibble_pos(e));
+      v[j] = o;
+    }
+    *reinterpret_cast<uint4*>(out + tile * tb + q * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+// Canonical int4 -> B200_V1, metadata: thread per (tile, block slot, row pair):
+// the two rows' fp16 scales and their shared zero-point byte (pads: scale 0,
+// zero-point 8); the 16-byte tail padding of a tile is zeroed by slot 0.
+__global__ void repack_int4_v1_meta_kernel(const uint8_t* scales, const uint8_t* zeros, uint8_t* out, int N, int K,
+                                           int bs) {
+  const long long n_bands = (N + 15) / 16;
+  const int tpb = K / 128;
+  const int bpt = int4_v1_bpt(bs);
+  const int tb = int4_v1_tile_bytes(bs);
+  const int nb = K / bs, zb = (nb + 1) / 2;
+  const long long items = n_bands * tpb * bpt * 8;
+  for (long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
+       it += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int rp = static_cast<int>(it & 7);
+    const long long rest = it >> 3;
+    const int bt = static_cast<int>(rest % bpt);
+    const long long tile = rest / bpt;
+    const long long band = tile / tpb;
+    const int s = static_cast<int>(tile - band * tpb);
+    const int blk = (128 * s + bt * (bs < 128 ? bs : 0)) / bs;
+    uint8_t* tp = out + tile * tb;
+    uint32_t zbyte = 0;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * rp + e;
+      const long long row = 16 * band + r;
+      uint16_t sv = 0;
+      uint32_t z = 8u;
+      if (row < N) {
+        sv = reinterpret_cast<const uint16_t*>(scales)[row * nb + blk];
+        if (zeros) z = (zeros[row * zb + (blk >> 1)] >> ((blk & 1) * 4)) & 15u;
+      }
+      reinterpret_cast<uint16_t*>(tp + 1024)[bt * 16 + r] = sv;
+      zbyte |= z << (4 * e);
+    }
+    tp[1024 + 32 * bpt + bt * 8 + rp] = static_cast<uint8_t>(zbyte);
+    if (bt == 0 && rp == 0)
+      for (int o = 1024 + 40 * bpt; o < tb; ++o) tp[o] = 0;
   }
 }
 
