@@ -62,7 +62,14 @@ for _M in (1, 2, 4, 8):
     for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336)):
         WORKLOADS[f"int4_b128_zp_v1_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 3, 0.002, 0.01, layout=1)
 
+for _M in (16, 32, 64, 128):
+    for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336), (32000, 4096)):
+        WORKLOADS[f"batched_int4_b128_zp_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 5, 0.002, 0.01)
+        WORKLOADS[f"batched_q4k_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=False, workload=5)
+
 DEFAULT_WORKLOAD = "int4_b128_zp_m1_4096x14336"
+SWEEP_BATCHED = [f"batched_{f}_m{m}_{n}x{k}" for f in ("int4_b128_zp", "q4k") for m in (16, 64, 128)
+                 for n, k in ((4096, 4096), (14336, 4096), (32000, 4096))]
 SWEEP = ["int4_b128_zp_v1_m1_4096x14336", "int4_b128_zp_v1_m2_4096x14336", "int4_b128_zp_v1_m4_4096x14336", "int4_b128_zp_v1_m8_4096x14336",
          "int4_b128_zp_v1_m1_14336x4096", "int4_b128_zp_v1_m1_4096x4096",
          "int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
@@ -471,6 +478,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--sweep", action="store_true", help="one JSON line per workload of the sweep list")
+    ap.add_argument("--sweep-batched", action="store_true", help="one JSON line per batched (M >= 16) workload")
     ap.add_argument("--graph-calls", type=int, default=1000)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -494,7 +502,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
-    names = SWEEP if args.sweep else [args.workload]
+    names = SWEEP if args.sweep else (SWEEP_BATCHED if args.sweep_batched else [args.workload])
     for name in names:
         out = run_ours(args, WORKLOADS[name], name, rank, world, dist)
         if rank == 0:

@@ -128,7 +128,7 @@ class BF16Case:
         return oracle.dequant_bf16(self.xb, self.M, self.K)
 
 
-VARIANTS = ("tc", "cc", "simple", None)
+VARIANTS = ("tc", "cc", "simple", "tc5", None)
 
 
 def each_variant(run, W, x, what):

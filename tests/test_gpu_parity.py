@@ -190,6 +190,24 @@ def test_gemv_larger_batches(M):
     each_variant(b.run, b.W(), b.X(), f"bf16 M={M}")
 
 
+@gpu
+@pytest.mark.parametrize("M", [9, 16, 32, 64, 128, 200, 300])
+@pytest.mark.parametrize("fmt", ["int4", "q4k"])
+def test_gemm_tcgen05_batched(M, fmt):
+    """The tcgen05 dequant-then-MMA path (default for M >= 9) on ragged row
+    tiles (N = 300) and batches that span one or two N tiles of the MMA."""
+    if fmt == "int4":
+        c = Int4Case(M, 300, 1024, 128, True, workload=29)
+        y = c.run()
+        W, x = c.W(), c.x
+    else:
+        c = Q4KCase(M, 300, 1024, workload=29)
+        y = c.run(False)
+        W, x = c.W(), c.x
+    assert ".gemm.tc5." in wq.last_kernel(), wq.last_kernel()
+    check(y, W, x, f"tcgen05 {fmt} M={M}")
+
+
 # ----------------------------------------------------------- closed forms on the device
 
 @gpu

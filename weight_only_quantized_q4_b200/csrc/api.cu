@@ -18,6 +18,7 @@
 #include "gemv_cc.cuh"
 #include "gemv_simple.cuh"
 #include "gemv_tc.cuh"
+#include "gemm_tc5.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -475,6 +476,54 @@ int launch_simple(const SimpleParams& sp, int M, int sms, cudaStream_t st) {
   return launch_check("gemv_simple launch");
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 batched path (M >= 9): planner and launcher
+// ---------------------------------------------------------------------------
+template <Fmt F>
+int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros, void* y, int M, int N,
+               int K, int nb, int zb, int block_size, cudaStream_t st, std::string* label) {
+  TC5Params p{};
+  p.x = x;
+  p.w = w;
+  p.scales = scales;
+  p.zeros = zeros;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nb = nb;
+  p.zb = zb;
+  p.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
+  p.BN = std::min(256, (M + 15) / 16 * 16);
+  int cols = 32;
+  while (cols < p.BN) cols *= 2;
+  p.tmem_cols = cols;
+  const int bsz = (p.BN * 128 + 1023) / 1024 * 1024;
+  const int smem = 1024 + 32768 + 2 * bsz + 64;
+  static std::mutex mu;
+  static bool configured[2][64] = {};
+  const int fi = F == Fmt::Int4 ? 0 : 1;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[fi][dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemm_tc5_kernel<F>),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[fi][dev] = true;
+    }
+  }
+  dim3 grid((N + 127) / 128, (M + p.BN - 1) / p.BN);
+  gemm_tc5_kernel<F><<<grid, 128, smem, st>>>(p);
+  int rc = launch_check("gemm_tc5 launch");
+  if (rc) return rc;
+  char buf[64];
+  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.bn%d", F == Fmt::Int4 ? "int4" : "q4k", p.BN);
+  *label = buf;
+  return WQ_OK;
+}
+
 // Run one format over all M in chunks of at most 8 rows of x.
 template <Fmt F>
 int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros,
@@ -485,6 +534,21 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
   if (rc) return rc;
   std::string label;
   const int x_elt = 2;
+  {
+    // batches of 9 and more: one tcgen05 dequant-then-MMA launch (int4 canonical, q4_K)
+    const char* force = forced_variant();
+    const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 128 == 0 && (K / 2) % 16 == 0) ||
+                        (F == Fmt::Q4K && K % 256 == 0);
+    const bool want = force ? std::strcmp(force, "tc5") == 0 : M >= 9;
+    if (tc5_ok && want && aligned16(x)) {
+      if constexpr (F == Fmt::Int4 || F == Fmt::Q4K) {
+        rc = launch_tc5<F>(x, w, scales, zeros, y, M, N, K, nb, zb, block_size, st, &label);
+        if (rc) return rc;
+        set_last_kernel(label);
+        return WQ_OK;
+      }
+    }
+  }
   for (int m0 = 0; m0 < M; m0 += 8) {
     const int mc = std::min(8, M - m0);
     const void* xc = static_cast<const uint8_t*>(x) + static_cast<long long>(m0) * K * x_elt;
