@@ -537,7 +537,7 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
   {
     // batches of 9 and more: one tcgen05 dequant-then-MMA launch (int4 canonical, q4_K)
     const char* force = forced_variant();
-    const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 128 == 0 && (K / 2) % 16 == 0) ||
+    const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 128 == 0 && block_size >= 64) ||
                         (F == Fmt::Q4K && K % 256 == 0);
     const bool want = force ? std::strcmp(force, "tc5") == 0 : M >= 9;
     if (tc5_ok && want && aligned16(x)) {

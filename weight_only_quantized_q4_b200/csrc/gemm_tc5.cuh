@@ -76,6 +76,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ uint32_t lop3_or(uint32_t v, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(magic));  // (v & mask) | magic
+  return r;
+}
+__device__ __forceinline__ uint32_t hsub2_f(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2_f(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // swizzled byte offset of 16-byte chunk c (0..7) of row r in a 128-B-row tile
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
@@ -85,15 +101,94 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
+// Raw data of one 64-k stage of one weight row, fetched ahead into registers.
+struct RawStage {
+  uint4 c0, c1, c2;  // int4: codes in c0, c1; q4_K: header in c0, codes in c1, c2
+  uint32_t sz;       // int4: fp16 scale bits | zero-point << 16
+};
+
 template <Fmt F>
-__global__ void __launch_bounds__(128, 1) gemm_tc5_kernel(const TC5Params p) {
+__device__ __forceinline__ void fetch_stage(const TC5Params& p, int row, int s, RawStage& r) {
+  const int k0 = s * 64;
+  if (row >= p.N) {
+    r.c0 = r.c1 = r.c2 = make_uint4(0u, 0u, 0u, 0u);
+    r.sz = 8u << 16;
+    return;
+  }
+  if constexpr (F == Fmt::Int4) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.w + static_cast<long long>(row) * (p.K / 2) + k0 / 2);
+    r.c0 = __ldcs(src);
+    r.c1 = __ldcs(src + 1);
+    const int b = k0 >> p.block_shift;  // blocks of >= 64 k: one scale / zero-point per stage
+    uint32_t z = 8u;
+    if (p.zeros) z = (p.zeros[static_cast<long long>(row) * p.zb + (b >> 1)] >> ((b & 1) * 4)) & 15u;
+    r.sz = reinterpret_cast<const uint16_t*>(p.scales)[static_cast<long long>(row) * p.nb + b] | (z << 16);
+  } else {
+    const int sb = k0 >> 8, pp = (k0 & 255) >> 6;
+    const uint8_t* blk = p.w + (static_cast<long long>(row) * (p.K / 256) + sb) * 144;
+    r.c0 = __ldcs(reinterpret_cast<const uint4*>(blk));
+    r.c1 = __ldcs(reinterpret_cast<const uint4*>(blk + 16 + 32 * pp));
+    r.c2 = __ldcs(reinterpret_cast<const uint4*>(blk + 32 + 32 * pp));
+  }
+}
+
+// Dequantize one stage of one row into 32 fp16x2 words (8 chunks of 8).
+// int4 chunk c holds codes of k = 8c + {0,4,1,5,2,6,3,7} (the activation tile
+// is permuted the same way); q4_K chunks are in natural k order.
+template <Fmt F>
+__device__ __forceinline__ void dequant_stage(const TC5Params& p, int s, const RawStage& r, uint32_t (&h)[32]) {
+  if constexpr (F == Fmt::Int4) {
+    const uint32_t sbits = r.sz & 0xFFFFu, z = r.sz >> 16;
+    const uint32_t s2 = sbits | (sbits << 16);
+    const uint32_t zl = (0x6400u | z) * 0x00010001u, zh = (0x5400u | (z << 4)) * 0x00010001u;
+    const uint32_t words[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
+#pragma unroll
+    for (int wd = 0; wd < 8; ++wd) {
+      const uint32_t v = words[wd], v8 = v >> 8;
+      uint32_t q[4];
+      q[0] = hsub2_f(lop3_or(v, 0x000F000Fu, 0x64006400u), zl);   // (n0, n4) - z, exact
+      q[1] = hsub2_f(lop3_or(v, 0x00F000F0u, 0x54005400u), zh);   // (n1, n5) - z
+      q[2] = hsub2_f(lop3_or(v8, 0x000F000Fu, 0x64006400u), zl);  // (n2, n6) - z
+      q[3] = hsub2_f(lop3_or(v8, 0x00F000F0u, 0x54005400u), zh);  // (n3, n7) - z
+#pragma unroll
+      for (int e = 0; e < 4; ++e) h[wd * 4 + e] = hmul2_f(q[e], s2);  // RN16((q - z)·s): one rounding
+    }
+  } else {
+    const int pp = ((s * 64) & 255) >> 6;
+    uint32_t sc2, mn2;
+    q4k_scale_min_pair(r.c0.y, r.c0.z, r.c0.w, static_cast<uint32_t>(pp & 1), static_cast<uint32_t>(pp >> 1), sc2, mn2);
+    const float d = h16_to_f32(r.c0.x), dm = h16_to_f32(r.c0.x >> 16);
+    const float A0 = __fmul_rn(d, static_cast<float>(sc2 & 0xFFu)), A1 = __fmul_rn(d, static_cast<float>(sc2 >> 8));
+    const float B0 = -__fmul_rn(dm, static_cast<float>(mn2 & 0xFFu)), B1 = -__fmul_rn(dm, static_cast<float>(mn2 >> 8));
+    const uint32_t words[8] = {r.c1.x, r.c1.y, r.c1.z, r.c1.w, r.c2.x, r.c2.y, r.c2.z, r.c2.w};
+#pragma unroll
+    for (int wd = 0; wd < 8; ++wd) {
+      const uint32_t v = words[wd];
+      float lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        lo[e] = fmaf(A0, __uint_as_float(0x4B000000u | ((v >> (8 * e)) & 15u)) - 8388608.0f, B0);
+        hi[e] = fmaf(A1, __uint_as_float(0x4B000000u | ((v >> (8 * e + 4)) & 15u)) - 8388608.0f, B1);
+      }
+      h[wd * 2 + 0] = pack_f16x2(lo[0], lo[1]);
+      h[wd * 2 + 1] = pack_f16x2(lo[2], lo[3]);
+      h[16 + wd * 2 + 0] = pack_f16x2(hi[0], hi[1]);
+      h[16 + wd * 2 + 1] = pack_f16x2(hi[2], hi[3]);
+    }
+  }
+}
+
+constexpr int kTc5Prefetch = 4;  // stages of raw weights in flight per thread
+
+template <Fmt F>
+__global__ void __launch_bounds__(128, 2) gemm_tc5_kernel(const TC5Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* A[2] = {smem, smem + 16384};
   const int bsz = ((p.BN * 128) + 1023) & ~1023;
   uint8_t* B[2] = {smem + 32768, smem + 32768 + bsz};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 32768 + 2 * bsz);  // [2] stage done, [2] final
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 32768 + 2 * bsz);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -122,92 +217,55 @@ __global__ void __launch_bounds__(128, 1) gemm_tc5_kernel(const TC5Params p) {
   const int nks = p.K / 64;
   const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x);
 
-  for (int s = 0; s < nks; ++s) {
-    const int slot = s & 1;
-    if (s >= 2 && !*abort_flag) {
-      // the MMAs that read this slot two stages ago must be done
-      if (!mbar_wait_bounded(&bars[slot], static_cast<uint32_t>(((s - 2) >> 1) & 1))) *abort_flag = 1;
-    }
-    __syncthreads();
-    if (*abort_flag) break;
-    const int k0 = s * 64;
-    // ---- A: this row's 64 weights as fp16 (8 chunks of 8)
-    uint32_t h[32];
-    if (row < p.N) {
-      if constexpr (F == Fmt::Int4) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.w + static_cast<long long>(row) * (p.K / 2) + k0 / 2);
-        const uint4 c0 = src[0], c1 = src[1];
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  RawStage raw[kTc5Prefetch];
 #pragma unroll
-        for (int wd = 0; wd < 8; ++wd) {
-          const int b = (k0 + 8 * wd) >> p.block_shift;
-          const float sc = h16_to_f32(reinterpret_cast<const uint16_t*>(p.scales)[static_cast<long long>(row) * p.nb + b]);
-          uint32_t z = 8u;
-          if (p.zeros) z = (p.zeros[static_cast<long long>(row) * p.zb + (b >> 1)] >> ((b & 1) * 4)) & 15u;
-          const uint32_t v = words[wd];
-          float f[8];
+  for (int i = 0; i < kTc5Prefetch; ++i)
+    if (i < nks) fetch_stage<F>(p, row, i, raw[i]);
+
+  for (int s0 = 0; s0 < nks; s0 += kTc5Prefetch) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = static_cast<float>(static_cast<int>((v >> (4 * e)) & 15u) - static_cast<int>(z)) * sc;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) h[wd * 4 + e] = pack_f16x2(f[2 * e], f[2 * e + 1]);
-        }
-      } else {
-        // 64 k = one run (chunks 2p, 2p+1) of one super-block
-        const int sb = k0 >> 8, pp = (k0 & 255) >> 6;
-        const uint8_t* blk = p.w + (static_cast<long long>(row) * (p.K / 256) + sb) * 144;
-        const uint4 hd = *reinterpret_cast<const uint4*>(blk);
-        uint32_t sc2, mn2;
-        q4k_scale_min_pair(hd.y, hd.z, hd.w, static_cast<uint32_t>(pp & 1), static_cast<uint32_t>(pp >> 1), sc2, mn2);
-        const float d = h16_to_f32(hd.x), dm = h16_to_f32(hd.x >> 16);
-        const float A0 = __fmul_rn(d, static_cast<float>(sc2 & 0xFFu)), A1 = __fmul_rn(d, static_cast<float>(sc2 >> 8));
-        const float B0 = -__fmul_rn(dm, static_cast<float>(mn2 & 0xFFu)), B1 = -__fmul_rn(dm, static_cast<float>(mn2 >> 8));
-        const uint4* qs = reinterpret_cast<const uint4*>(blk + 16 + 32 * pp);
-        const uint4 q0 = qs[0], q1 = qs[1];
-        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        // element i of chunk 2p: low nibble of byte i; of chunk 2p+1: high nibble
-#pragma unroll
-        for (int wd = 0; wd < 8; ++wd) {
-          const uint32_t v = words[wd];
-          float lo[4], hi[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            lo[e] = fmaf(A0, static_cast<float>((v >> (8 * e)) & 15u), B0);
-            hi[e] = fmaf(A1, static_cast<float>((v >> (8 * e + 4)) & 15u), B1);
-          }
-          h[wd * 2 + 0] = pack_f16x2(lo[0], lo[1]);      // k = 64p + 4wd + 0,1
-          h[wd * 2 + 1] = pack_f16x2(lo[2], lo[3]);      // k = 64p + 4wd + 2,3
-          h[16 + wd * 2 + 0] = pack_f16x2(hi[0], hi[1]); // k = 64p + 32 + 4wd + 0,1
-          h[16 + wd * 2 + 1] = pack_f16x2(hi[2], hi[3]);
-        }
+    for (int i = 0; i < kTc5Prefetch; ++i) {
+      const int s = s0 + i;
+      if (s >= nks) break;
+      const int slot = s & 1;
+      if (s >= 2 && !*abort_flag) {
+        if (!mbar_wait_bounded(&bars[slot], static_cast<uint32_t>(((s - 2) >> 1) & 1))) *abort_flag = 1;
       }
-    } else {
+      __syncthreads();
+      if (*abort_flag) break;
+      const int k0 = s * 64;
+      uint32_t h[32];
+      dequant_stage<F>(p, s, raw[i], h);
+      if (s + kTc5Prefetch < nks) fetch_stage<F>(p, row, s + kTc5Prefetch, raw[i]);
+      uint8_t* a = A[slot];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) h[i] = 0u;
-    }
-    uint8_t* a = A[slot];
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(a + sw128(tid, c)) = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+      // ---- B: activation rows m0 .. m0+BN-1, k0 .. k0+63 (zero past M)
+      uint8_t* bt = B[slot];
+      for (int c = tid; c < p.BN * 8; c += 128) {
+        const int n = c >> 3, kc = c & 7;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (m0 + n < p.M) v = *reinterpret_cast<const uint4*>(xg + static_cast<long long>(m0 + n) * p.K + k0 + 8 * kc);
+        if constexpr (F == Fmt::Int4)  // same k order as the A chunks: x0 x4 x1 x5 x2 x6 x3 x7
+          v = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632), __byte_perm(v.y, v.w, 0x5410),
+                         __byte_perm(v.y, v.w, 0x7632));
+        *reinterpret_cast<uint4*>(bt + sw128(n, kc)) = v;
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint64_t ad = umma_smem_desc_sw128(smem_u32(a));
+        const uint64_t bd = umma_smem_desc_sw128(smem_u32(bt));
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<uint4*>(a + sw128(tid, c)) = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
-    // ---- B: activation rows m0 .. m0+BN-1, k0 .. k0+63 (zero past M)
-    uint8_t* bt = B[slot];
-    for (int c = tid; c < p.BN * 8; c += 128) {
-      const int n = c >> 3, kc = c & 7;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (m0 + n < p.M) v = *reinterpret_cast<const uint4*>(xg + static_cast<long long>(m0 + n) * p.K + k0 + 8 * kc);
-      *reinterpret_cast<uint4*>(bt + sw128(n, kc)) = v;
+        for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
+          umma_f16(tmem, ad + 2ull * j, bd + 2ull * j, idesc, (s > 0 || j > 0) ? 1u : 0u);
+        umma_commit(&bars[slot]);
+      }
     }
-    fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint64_t ad = umma_smem_desc_sw128(smem_u32(a));
-      const uint64_t bd = umma_smem_desc_sw128(smem_u32(bt));
-#pragma unroll
-      for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
-        umma_f16(tmem, ad + 2ull * j, bd + 2ull * j, idesc, (s > 0 || j > 0) ? 1u : 0u);
-      umma_commit(&bars[slot]);
-    }
+    if (*abort_flag) break;
   }
   // ---- wait for the last stage's MMAs, then read the accumulator
   const int last = nks - 1;
