@@ -128,7 +128,7 @@ class BF16Case:
         return oracle.dequant_bf16(self.xb, self.M, self.K)
 
 
-VARIANTS = ("tc", "cc", "simple", "tc5", None)
+VARIANTS = ("tc", "cc", "simple", "tc5", "v1s", "v1r", None)
 
 
 def each_variant(run, W, x, what):

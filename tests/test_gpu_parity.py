@@ -138,6 +138,54 @@ def test_gemv_int4_v1_layout(M, N, K, bs, zeros):
     assert ".simple." in labels["cc"] and ".simple." in labels["simple"], labels
 
 @gpu
+@pytest.mark.parametrize("C", [1, 2, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("N,K,bs,zeros", [(37, 2048, 128, True), (1000, 1536, 256, False), (300, 512, 128, True),
+                                          (4100, 1024, 128, True), (16, 4096, 256, True)])
+def test_gemv_int4_v1_cluster_split(C, M, N, K, bs, zeros, monkeypatch):
+    """The B200_V1 kernel with subnormal codes and a per-tile Σx zero-point term,
+    with the k-tiles of every band split over clusters of C CTAs (partials added
+    through distributed shared memory).  Two calls in a row must agree bit for bit."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1s")
+    monkeypatch.setenv("WQ_V1_C", str(C))
+    c = Int4Case(M, N, K, bs, zeros, workload=23, layout=wq.WQ_LAYOUT_B200_V1)
+    y1 = c.run()
+    label = wq.last_kernel()
+    assert ".gemv.v1s." in label and label.endswith(f".c{C}"), label
+    check(y1, c.W(), c.x, f"v1s C={C} M={M} N={N} K={K} bs={bs} zp={zeros}")
+    y2 = c.run()
+    assert np.array_equal(y1, y2)
+
+
+@gpu
+@pytest.mark.parametrize("P", [2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("N,K,bs,zeros", [(37, 2048, 128, True), (1000, 1536, 256, False), (300, 512, 128, True),
+                                          (4100, 1024, 128, True), (16, 4096, 256, True), (5, 128, 128, True)])
+def test_gemv_int4_v1_register_stream(P, M, N, K, bs, zeros, monkeypatch):
+    """The B200_V1 kernel that streams tiles straight into registers, P tiles
+    ahead per warp.  Two calls in a row must agree bit for bit."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1r")
+    monkeypatch.setenv("WQ_V1R_P", str(P))
+    c = Int4Case(M, N, K, bs, zeros, workload=24, layout=wq.WQ_LAYOUT_B200_V1)
+    y1 = c.run()
+    label = wq.last_kernel()
+    assert ".gemv.v1r." in label and f".p{P}" in label, label
+    check(y1, c.W(), c.x, f"v1r P={P} M={M} N={N} K={K} bs={bs} zp={zeros}")
+    assert np.array_equal(y1, c.run())
+
+
+@gpu
+def test_gemv_int4_v1_default_kernel_full_size():
+    c = Int4Case(1, 4096, 14336, 128, True, workload=3, layout=wq.WQ_LAYOUT_B200_V1)
+    rows = sample_rows(4096)
+    y = c.run()
+    assert ".gemv.v1s." in wq.last_kernel(), wq.last_kernel()
+    W = oracle.dequant_int4(c.w[rows], c.s[rows], c.z[rows], len(rows), 14336, 128)
+    check(y[:, rows], W, c.x, "B200_V1 4096x14336 sampled rows")
+
+
+@gpu
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
 @pytest.mark.parametrize("N,K,bs,zeros", [(256, 1024, 32, False), (37, 2048, 128, True), (301, 512, 16, True),
                                           (64, 4096, 64, True), (1000, 1536, 256, False)])

@@ -18,6 +18,7 @@
 #include "gemv_cc.cuh"
 #include "gemv_simple.cuh"
 #include "gemv_tc.cuh"
+#include "gemv_v1.cuh"
 #include "gemm_tc5.cuh"
 #include "wq_host.h"
 
@@ -450,6 +451,281 @@ int launch_tc(Fmt f, int layout, const TCPlan& plan, cudaStream_t st) {
   return launch_check("gemv_tc launch");
 }
 
+// ---------------------------------------------------------------------------
+// B200_V1 int4 GEMV (blocks >= 128 k): planner and launcher
+// ---------------------------------------------------------------------------
+struct V1Plan {
+  V1Params p;
+  int grid = 0, threads = 0, smem = 0;
+};
+
+constexpr int kV1XBudget = 120 * 1024;   // resident activations per CTA
+constexpr int kV1PartBudget = 16 * 1024;  // per-CTA band partials of a cluster split
+
+// Clusters of C CTAs (one CTA per SM) that can be resident at once, per device.
+int v1_max_clusters(int C, int smem, int threads, int sms) {
+  if (C == 1) return sms;
+  static std::mutex mu;
+  static int cache[64][5] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= 0 && dev < 64 && cache[dev][C] > 0) return cache[dev][C];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C * sms, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(&gemv_v1_kernel), &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  if (dev >= 0 && dev < 64) cache[dev][C] = n > 0 ? n : -1;
+  return n;
+}
+
+int v1_configure() {
+  static std::mutex mu;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemv_v1_kernel),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    configured[dev] = true;
+  }
+  return WQ_OK;
+}
+
+// Geometry for cluster size C over n_clusters clusters; false if it does not fit.
+bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clusters, V1Plan* plan, int stage_kb) {
+  const char* w_env = std::getenv("WQ_V1_W");  // consumer warps (tuning)
+  if (w_env) W = std::max(4, std::min(kV1MaxWarps - 2, std::atoi(w_env)));
+  const int tpb = K / 128;
+  if (C < 1 || tpb % C || n_clusters < 1) return false;
+  V1Params& p = plan->p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_bands = (N + 15) / 16;
+  p.tpb = tpb;
+  p.tpc = tpb / C;
+  p.tb = int4_v1_tile_bytes(block_size);
+  p.W = W;
+  // tiles per stage: a multiple of W, about stage_kb KB (larger bulk copies
+  // stream faster on B200; WQ_V1_STAGE_KB overrides, for tuning)
+  const char* sk_env = std::getenv("WQ_V1_STAGE_KB");
+  const int stage_budget = (sk_env ? std::max(1, std::atoi(sk_env)) : stage_kb) * 1024;
+  p.tps = W * std::max(1, stage_budget / (W * p.tb));
+  const char* pre_env = std::getenv("WQ_V1_PRE");  // stages requested before the x copy (tuning)
+  p.pre = pre_env ? std::max(0, std::atoi(pre_env)) : 2;
+  const char* h_env = std::getenv("WQ_V1_HINT");
+  p.hint = h_env ? (std::atoi(h_env) != 0) : 1;
+  p.stage_bytes = p.tps * p.tb;
+  p.C = C;
+  p.Mp = (M + 1) & ~1;
+  const int bpc = (p.n_bands + n_clusters - 1) / n_clusters;  // bands per cluster, at most
+  const long long x_bytes = 2ll * M * p.tpc * 128;
+  const long long xs_bytes = 32ll * p.tpc;
+  const long long red_bytes = 2ll * W * 16 * p.Mp * 4;
+  const long long part_bytes = C > 1 ? 4ll * bpc * 16 * M : 0;
+  if (x_bytes > kV1XBudget || part_bytes > kV1PartBudget) return false;
+  const long long fixed = round16(x_bytes) + 256 + round16(xs_bytes) + round16(red_bytes) + round16(part_bytes);
+  const char* cps_env = std::getenv("WQ_V1_CTAS");
+  const int cps = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : 1;
+  const long long room = kSmemPerSm / cps - 1024 - fixed - (2ll * 16 * 8 + 8 + 16);
+  const char* ns_env = std::getenv("WQ_V1_NS");
+  const int NS = static_cast<int>(
+      std::min<long long>(ns_env ? std::max(2, std::atoi(ns_env)) : 16, room / p.stage_bytes));
+  if (NS < 3) return false;
+  p.NS = NS;
+  p.pre = std::min(p.pre, NS);  // the x copy must not wait for a ring slot
+  long long off = static_cast<long long>(NS) * p.stage_bytes;
+  p.off_x = static_cast<int>(off);
+  off += round16(x_bytes);
+  p.off_zero = static_cast<int>(off);
+  off += 256;
+  p.off_xs = static_cast<int>(off);
+  off += round16(xs_bytes);
+  p.off_red = static_cast<int>(off);
+  off += round16(red_bytes);
+  p.off_part = static_cast<int>(off);
+  off += round16(part_bytes);
+  p.off_bar = static_cast<int>(off);
+  off += 2ll * NS * 8 + 8 + 16;
+  plan->smem = static_cast<int>(off);
+  plan->threads = (W + 2) * 32;
+  plan->grid = n_clusters * C;
+  return true;
+}
+
+// Pick the cluster size that minimises the tiles of the busiest CTA
+// (WQ_V1_C forces one, for tests and tuning).
+bool plan_v1(int M, int N, int K, int block_size, int sms, V1Plan* out) {
+  if (M < 1 || M > 8 || K % 128 || block_size < 128) return false;
+  if (v1_configure() != WQ_OK) return false;
+  const char* c_env = std::getenv("WQ_V1_C");
+  const int c_force = c_env ? std::atoi(c_env) : 0;
+  const int W = 16;
+  const int n_bands = (N + 15) / 16;
+  long long best_cost = -1;
+  // Cluster splits along K measured slower than whole bands per CTA on B200
+  // (smaller copies per band, an extra cluster reduction): only on request.
+  for (int C : {1, 2, 4}) {
+    if (c_force ? C != c_force : C != 1) continue;
+    const char* cps_env = std::getenv("WQ_V1_CTAS");
+    const int cps = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : 1;
+    int ncl = C == 1 ? cps * sms : v1_max_clusters(C, kSmemPerSm, (W + 2) * 32, sms);
+    if (ncl <= 0) continue;
+    ncl = std::min(ncl, n_bands);
+    V1Plan pl;
+    // shrink the stages until the ring holds three of them (large activations)
+    bool fits = false;
+    for (int kb : {52, 36, 24, 18}) {
+      if (plan_v1_geom(M, N, K, block_size, C, W, ncl, &pl, kb)) {
+        fits = true;
+        break;
+      }
+    }
+    if (!fits) continue;
+    const long long cost = static_cast<long long>((n_bands + ncl - 1) / ncl) * pl.p.tpc;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      *out = pl;
+    }
+  }
+  return best_cost >= 0;
+}
+
+// WQ_PDL=0 turns programmatic dependent launch off (A/B runs).
+bool pdl_enabled() {
+  const char* v = std::getenv("WQ_PDL");
+  return !(v && std::atoi(v) == 0);
+}
+
+// ---------------------------------------------------------------------------
+// B200_V1 int4 GEMV, register-streaming kernel: planner and launcher
+// ---------------------------------------------------------------------------
+struct V1RPlan {
+  V1RParams p;
+  int P = 4, grid = 0, threads = 0, smem = 0;
+};
+
+constexpr int kV1RXBudget = 200 * 1024;  // activations resident in shared memory
+
+bool plan_v1r(int M, int N, int K, int block_size, int sms, V1RPlan* out) {
+  if (M < 1 || M > 8 || K % 128 || block_size < 128) return false;
+  V1RParams& p = out->p;
+  const char* w_env = std::getenv("WQ_V1R_W");  // consumer warps (tuning)
+  const char* p_env = std::getenv("WQ_V1R_P");  // tiles in flight per warp (tuning)
+  p.W = w_env ? std::max(4, std::min(kV1RMaxWarps - 1, std::atoi(w_env))) : 16;
+  out->P = p_env ? std::atoi(p_env) : 4;
+  if (out->P != 2 && out->P != 3 && out->P != 4) out->P = 4;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_bands = (N + 15) / 16;
+  p.tpb = K / 128;
+  p.tb = int4_v1_tile_bytes(block_size);
+  p.Mp = (M + 1) & ~1;
+  const long long x_bytes = 2ll * M * K;
+  if (x_bytes > kV1RXBudget) return false;
+  long long off = 0;
+  p.off_x = 0;
+  off += round16(x_bytes);
+  p.off_zero = static_cast<int>(off);
+  off += 256;
+  p.off_xs = static_cast<int>(off);
+  off += round16(32ll * p.tpb);
+  p.off_red = static_cast<int>(off);
+  off += 2ll * p.W * 16 * p.Mp * 4;
+  if (off > kSmemPerSm) return false;
+  out->smem = static_cast<int>(off);
+  out->threads = (p.W + 1) * 32;
+  out->grid = std::max(1, std::min(p.n_bands, sms));
+  return true;
+}
+
+template <int P>
+int launch_v1r_p(const V1RPlan& plan, cudaStream_t st) {
+  static std::mutex mu;
+  static bool configured[64] = {};
+  {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemv_v1r_kernel<P>),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.grid, 1, 1);
+  cfg.blockDim = dim3(plan.threads, 1, 1);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemv_v1r_kernel<P>, plan.p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemv_v1r launch: ") + cudaGetErrorString(e));
+  return launch_check("gemv_v1r launch");
+}
+
+int launch_v1r(const V1RPlan& plan, cudaStream_t st) {
+  switch (plan.P) {
+    case 2: return launch_v1r_p<2>(plan, st);
+    case 3: return launch_v1r_p<3>(plan, st);
+    default: return launch_v1r_p<4>(plan, st);
+  }
+}
+
+
+int launch_v1(const V1Plan& plan, cudaStream_t st) {
+  int rc = v1_configure();
+  if (rc) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.grid, 1, 1);
+  cfg.blockDim = dim3(plan.threads, 1, 1);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl_enabled()) {
+    // programmatic dependent launch: the kernel requests its read-only weights
+    // while the previous kernel in the stream finishes (it waits for that
+    // kernel before it reads x or writes y)
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (plan.p.C > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = plan.p.C;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemv_v1_kernel, plan.p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemv_v1 launch: ") + cudaGetErrorString(e));
+  return launch_check("gemv_v1 launch");
+}
+
 // WQ_FORCE_KERNEL = "cc" | "tc" | "simple" pins the GEMV variant (A/B runs and
 // per-variant parity tests); unset means the default choice below.
 const char* forced_variant() {
@@ -554,6 +830,37 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     const void* xc = static_cast<const uint8_t*>(x) + static_cast<long long>(m0) * K * x_elt;
     void* yc = static_cast<uint8_t*>(y) + static_cast<long long>(m0) * N * 2;
     const char* force = forced_variant();
+    if constexpr (F == Fmt::Int4) {
+      V1RPlan rplan;
+      // (the register-streaming kernel measured slower than the bulk-copy ring
+      // on B200 for the 4096x14336-class shapes: it runs on request only)
+      const bool want_v1r = force ? std::strcmp(force, "v1r") == 0 : false;
+      if (want_v1r && layout == WQ_LAYOUT_B200_V1 && aligned16(xc) && plan_v1r(mc, N, K, block_size, di.sms, &rplan)) {
+        rplan.p.x = xc;
+        rplan.p.w = w;
+        rplan.p.y = yc;
+        rc = launch_v1r(rplan, st);
+        if (rc) return rc;
+        char buf[64];
+        std::snprintf(buf, sizeof(buf), "%s.gemv.v1r.m%d.p%d%s", fmt_name, mc, rplan.P, M > 8 ? ".chunked" : "");
+        label = buf;
+        continue;
+      }
+      V1Plan vplan;
+      const bool want_v1 = force ? std::strcmp(force, "v1s") == 0 : true;
+      if (want_v1 && layout == WQ_LAYOUT_B200_V1 && aligned16(xc) &&
+          plan_v1(mc, N, K, block_size, di.sms, &vplan)) {
+        vplan.p.x = xc;
+        vplan.p.w = w;
+        vplan.p.y = yc;
+        rc = launch_v1(vplan, st);
+        if (rc) return rc;
+        char buf[64];
+        std::snprintf(buf, sizeof(buf), "%s.gemv.v1s.m%d.c%d%s", fmt_name, mc, vplan.p.C, M > 8 ? ".chunked" : "");
+        label = buf;
+        continue;
+      }
+    }
     const bool want_tc = force ? std::strcmp(force, "tc") == 0 : true;
     const bool want_cc = force ? std::strcmp(force, "cc") == 0 : true;
     TCPlan tplan;
