@@ -507,7 +507,8 @@ int v1_configure() {
 }
 
 // Geometry for cluster size C over n_clusters clusters; false if it does not fit.
-bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clusters, V1Plan* plan, int stage_kb) {
+bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clusters, V1Plan* plan, int stage_kb,
+                  int cps) {
   const char* w_env = std::getenv("WQ_V1_W");  // consumer warps (tuning)
   if (w_env) W = std::max(4, std::min(kV1MaxWarps - 2, std::atoi(w_env)));
   const int tpb = K / 128;
@@ -540,8 +541,6 @@ bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clust
   const long long part_bytes = C > 1 ? 4ll * bpc * 16 * M : 0;
   if (x_bytes > kV1XBudget || part_bytes > kV1PartBudget) return false;
   const long long fixed = round16(x_bytes) + 256 + round16(xs_bytes) + round16(red_bytes) + round16(part_bytes);
-  const char* cps_env = std::getenv("WQ_V1_CTAS");
-  const int cps = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : 1;
   const long long room = kSmemPerSm / cps - 1024 - fixed - (2ll * 16 * 8 + 8 + 16);
   const char* ns_env = std::getenv("WQ_V1_NS");
   const int NS = static_cast<int>(
@@ -575,35 +574,31 @@ bool plan_v1(int M, int N, int K, int block_size, int sms, V1Plan* out) {
   if (v1_configure() != WQ_OK) return false;
   const char* c_env = std::getenv("WQ_V1_C");
   const int c_force = c_env ? std::atoi(c_env) : 0;
-  const int W = 16;
+  const char* cps_env = std::getenv("WQ_V1_CTAS");
+  const int cps_force = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : 0;
   const int n_bands = (N + 15) / 16;
-  long long best_cost = -1;
-  // Cluster splits along K measured slower than whole bands per CTA on B200
-  // (smaller copies per band, an extra cluster reduction): only on request.
-  for (int C : {1, 2, 4}) {
-    if (c_force ? C != c_force : C != 1) continue;
-    const char* cps_env = std::getenv("WQ_V1_CTAS");
-    const int cps = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : 1;
-    int ncl = C == 1 ? cps * sms : v1_max_clusters(C, kSmemPerSm, (W + 2) * 32, sms);
-    if (ncl <= 0) continue;
+  if (c_force > 1) {
+    // cluster split along K (measured slower than whole bands per CTA on B200:
+    // smaller copies per band and an extra cluster reduction), on request only
+    const int W = 16;
+    int ncl = v1_max_clusters(c_force, kSmemPerSm, (W + 2) * 32, sms);
+    if (ncl <= 0) return false;
     ncl = std::min(ncl, n_bands);
-    V1Plan pl;
-    // shrink the stages until the ring holds three of them (large activations)
-    bool fits = false;
-    for (int kb : {52, 36, 24, 18}) {
-      if (plan_v1_geom(M, N, K, block_size, C, W, ncl, &pl, kb)) {
-        fits = true;
-        break;
-      }
-    }
-    if (!fits) continue;
-    const long long cost = static_cast<long long>((n_bands + ncl - 1) / ncl) * pl.p.tpc;
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      *out = pl;
-    }
+    for (int kb : {52, 36, 24, 18})
+      if (plan_v1_geom(M, N, K, block_size, c_force, W, ncl, out, kb, 1)) return true;
+    return false;
   }
-  return best_cost >= 0;
+  // Two CTAs per SM (12 consumer warps each) when 36 KB stages still fit: the
+  // next call's CTAs then start beside the current ones and fill their rings
+  // while these finish.  Otherwise one CTA per SM with 16 consumer warps and the
+  // largest stages that leave three in the ring.
+  if (cps_force != 1 &&
+      plan_v1_geom(M, N, K, block_size, 1, 12, std::min(n_bands, 2 * sms), out, 36, 2))
+    return true;
+  if (cps_force == 2) return false;
+  for (int kb : {52, 36, 24, 18})
+    if (plan_v1_geom(M, N, K, block_size, 1, 16, std::min(n_bands, sms), out, kb, 1)) return true;
+  return false;
 }
 
 // WQ_PDL=0 turns programmatic dependent launch off (A/B runs).
