@@ -256,6 +256,28 @@ def test_gemm_tcgen05_batched(M, fmt):
     check(y, W, x, f"tcgen05 {fmt} M={M}")
 
 
+@gpu
+@pytest.mark.parametrize("S", [1, 2, 4, 8])
+@pytest.mark.parametrize("M", [16, 33, 128])
+@pytest.mark.parametrize("fmt", ["int4", "q4k"])
+def test_gemm_tcgen05_cluster_split_k(S, M, fmt, monkeypatch):
+    """The tcgen05 batched path with K split over a cluster of S CTAs whose fp32
+    accumulators are added through distributed shared memory (ragged N tiles,
+    batch tiles of 16..128 columns).  Two calls in a row agree bit for bit."""
+    monkeypatch.setenv("WQ_TC5_S", str(S))
+    if fmt == "int4":
+        c = Int4Case(M, 300, 4096, 128, True, workload=31)
+        run = c.run
+    else:
+        c = Q4KCase(M, 300, 2048, workload=31)
+        run = lambda: c.run(False)  # noqa: E731
+    y = run()
+    label = wq.last_kernel()
+    assert ".gemm.tc5." in label and label.endswith(f".s{S}"), label
+    check(y, c.W(), c.x, f"tcgen05 {fmt} M={M} S={S}")
+    assert np.array_equal(y, run())
+
+
 # ----------------------------------------------------------- closed forms on the device
 
 @gpu

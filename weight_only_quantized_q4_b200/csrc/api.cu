@@ -5,6 +5,8 @@
 // arguments or enqueues kernels on the caller's stream.  There is no CPU
 // fallback and no silent kernel fallback: wq_last_kernel() names the kernel
 // each call launched.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -750,9 +752,41 @@ int launch_simple(const SimpleParams& sp, int M, int sms, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 // tcgen05 batched path (M >= 9): planner and launcher
 // ---------------------------------------------------------------------------
+// cuTensorMapEncodeTiled from the driver, looked up once (no link-time
+// dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+int encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, unsigned long long inner,
+              unsigned long long outer, unsigned long long row_bytes, unsigned box_inner, unsigned box_outer,
+              CUtensorMapSwizzle sw) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(static_cast<int>(r)) + ")");
+  return WQ_OK;
+}
+
 template <Fmt F>
 int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros, void* y, int M, int N,
-               int K, int nb, int zb, int block_size, cudaStream_t st, std::string* label) {
+               int K, int nb, int zb, int block_size, int sms, cudaStream_t st, std::string* label) {
   TC5Params p{};
   p.x = x;
   p.w = w;
@@ -767,10 +801,48 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   p.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
   p.BN = std::min(256, (M + 15) / 16 * 16);
   int cols = 32;
-  while (cols < p.BN) cols *= 2;
+  while (cols < 2 * p.BN) cols *= 2;  // two accumulator tiles (even / odd stages)
   p.tmem_cols = cols;
-  const int bsz = (p.BN * 128 + 1023) / 1024 * 1024;
-  const int smem = 1024 + 32768 + 2 * bsz + 64;
+  // shared memory: 4 A slots (16 KB), NX activation slots, NR raw slots, barriers
+  const int x_slot = (p.BN * 128 + 1023) / 1024 * 1024;
+  // raw slots of 256 k: int4 128 B per row, q4_K one 144-byte super-block per row
+  // (256-byte int4 rows measured no faster on B200)
+  p.spr = 4;
+  p.raw_pitch = F == Fmt::Int4 ? 128 : 144;
+  p.raw_bytes = 128 * p.raw_pitch;
+  p.NR = 3;
+  const int budget = kSmemPerSm - 1024 - 1024;
+  p.NX = std::max(2, std::min(8, (budget - kTc5NA * 16384 - p.NR * p.raw_bytes) / x_slot));
+  p.off_x = kTc5NA * 16384;
+  p.off_raw = p.off_x + p.NX * x_slot;
+  p.off_bar = (p.off_raw + p.NR * p.raw_bytes + 127) / 128 * 128;
+  const int smem = 1024 + p.off_bar + (2 * p.NR + 2 * p.NX + 2 * kTc5NA + 1) * 8 + 16;
+  if (smem > kSmemPerSm + 4096) return fail(WQ_ERR_UNSUPPORTED, "gemm_tc5: shared memory plan too large");
+  // Split K over a cluster of S CTAs (one CTA per SM) until the CTAs fill the
+  // SMs; every CTA keeps a whole number of 256-k raw slots.
+  const int n_tiles = (N + 127) / 128, m_tiles = (M + p.BN - 1) / p.BN;
+  const int nst = K / 64;
+  int S = 1;
+  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nst % (2 * p.spr * S) == 0) S *= 2;
+  if (const char* s_env = std::getenv("WQ_TC5_S")) {  // tests and tuning
+    const int sf = std::atoi(s_env);
+    if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
+      if (nst % (p.spr * sf)) return fail(WQ_ERR_ARG, "WQ_TC5_S does not divide K into whole raw slots");
+      S = sf;
+    }
+  }
+  if (S > 1 && 512 * p.BN > p.off_bar) return fail(WQ_ERR_UNSUPPORTED, "gemm_tc5: cluster partials do not fit");
+  p.S = S;
+  p.nks = nst / S;
+  int rc;
+  if constexpr (F == Fmt::Int4)
+    rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (K / 256) * 144ull, N, (K / 256) * 144ull, 144, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  rc = encode_2d(&p.tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, 2ull * K, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
   static std::mutex mu;
   static bool configured[2][64] = {};
   const int fi = F == Fmt::Int4 ? 0 : 1;
@@ -785,12 +857,24 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
       configured[fi][dev] = true;
     }
   }
-  dim3 grid((N + 127) / 128, (M + p.BN - 1) / p.BN);
-  gemm_tc5_kernel<F><<<grid, 128, smem, st>>>(p);
-  int rc = launch_check("gemm_tc5 launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles * S, m_tiles, 1);
+  cfg.blockDim = dim3(kTc5Warps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemm_tc5_kernel<F>, p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_tc5 launch: ") + cudaGetErrorString(e));
+  rc = launch_check("gemm_tc5 launch");
   if (rc) return rc;
   char buf[64];
-  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.bn%d", F == Fmt::Int4 ? "int4" : "q4k", p.BN);
+  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.bn%d.s%d", F == Fmt::Int4 ? "int4" : "q4k", p.BN, S);
   *label = buf;
   return WQ_OK;
 }
@@ -808,12 +892,12 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
   {
     // batches of 9 and more: one tcgen05 dequant-then-MMA launch (int4 canonical, q4_K)
     const char* force = forced_variant();
-    const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 128 == 0 && block_size >= 64) ||
+    const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0 && block_size >= 64) ||
                         (F == Fmt::Q4K && K % 256 == 0);
     const bool want = force ? std::strcmp(force, "tc5") == 0 : M >= 9;
     if (tc5_ok && want && aligned16(x)) {
       if constexpr (F == Fmt::Int4 || F == Fmt::Q4K) {
-        rc = launch_tc5<F>(x, w, scales, zeros, y, M, N, K, nb, zb, block_size, st, &label);
+        rc = launch_tc5<F>(x, w, scales, zeros, y, M, N, K, nb, zb, block_size, di.sms, st, &label);
         if (rc) return rc;
         set_last_kernel(label);
         return WQ_OK;

@@ -1,24 +1,31 @@
 // gemm_tc5.cuh — batched dequant-then-MMA on the 5th-generation tensor cores
 // (tcgen05, sm_100a) for M >= 9 decode/prefill batches.
 //
-// y[m, n] = Σ_k W[n, k]·x[m, k].  A CTA owns 128 weight rows (the UMMA M side)
-// and BN batch rows (the UMMA N side, a multiple of 16, <= 256).  For every
-// 64-k stage:
-//   * the 128 threads dequantize their row's 64 weights to fp16 and store them
-//     into a 128-byte-swizzled K-major A tile (16 KB); int4 as
-//     RN16((q - z)·s) (q - z exact in fp16, one rounding of the exact
-//     product), q4_K as RN16(d·sc·q - dmin·m) from the exact fp32 value;
-//   * they copy the BN × 64 activation slice into a B tile of the same layout;
-//   * one thread issues four tcgen05.mma (K = 16 each) accumulating into an
-//     fp32 TMEM accumulator of 128 lanes × BN columns, and commits them to an
-//     mbarrier that frees the stage's A/B buffers (two buffers: dequantizing
-//     stage s+1 overlaps the MMAs of stage s).
-// The epilogue reads the accumulator with tcgen05.ld (warp w owns TMEM lanes
-// 32w..32w+31 = weight rows) and stores fp16 y.  Weights are rounded to fp16
-// once before the MMA (error <= 2^-11 relative per weight, within the
-// 2e-3·Σ|w·x| acceptance bound); the device dequant exports stay exact fp32.
-// Every mbarrier wait is bounded (wq_device.cuh).
+// y[m, n] = Σ_k W[n, k]·x[m, k].  A CTA owns 128 weight rows (the UMMA M side),
+// BN batch rows (the UMMA N side, a multiple of 16, <= 256) and one K slice;
+// the S CTAs of a thread-block cluster share the rows and split K, and add
+// their fp32 accumulators through distributed shared memory (fixed rank
+// order).  Warp-specialized pipeline over 64-k stages, with full / empty
+// mbarrier rings and no block-wide synchronisation in the main loop:
+//   * producer warp: 2-D TMA copies (tensor maps, no multicast) of the raw
+//     weight bytes, 128 rows × 256 k per copy (int4: 128 B per row; q4_K: one
+//     144-byte super-block per row), and of the BN × 64 activation slice,
+//     128-byte swizzled so it lands in the UMMA K-major layout;
+//   * eight dequant warps (two threads per weight row, 32 k each) turn the raw
+//     bytes into a 128-byte-swizzled fp16 A tile in natural k order: int4 as
+//     RN16((q - z)·s) (q - z exact via magic-number codes, one rounding of the
+//     exact product), q4_K as RN16(d·sc·q - dmin·m) from the exact fp32 value;
+//   * one MMA warp issues four tcgen05.mma (K = 16 each) into an fp32 TMEM
+//     accumulator of 128 lanes × BN columns and commits them to the mbarriers
+//     that free the A and activation slots.
+// The epilogue reads the accumulator with tcgen05.ld (warps w and w + 4 share
+// TMEM lanes 32(w mod 4).. and split the columns) and stores fp16 y.  Weights
+// are rounded to fp16 once before the MMA (error <= 2^-11 relative per weight,
+// within the 2e-3·Σ|w·x| acceptance bound); the device dequant exports stay
+// exact fp32.  Every mbarrier wait is bounded (wq_device.cuh).
 #pragma once
+
+#include <cuda.h>
 
 #include "gemv_cc.cuh"
 #include "wq_device.cuh"
@@ -26,6 +33,8 @@
 namespace wq {
 
 struct TC5Params {
+  CUtensorMap tmap_w;  // raw weight bytes: [N][K/2] (int4) or [N][K/256·144] (q4_K), box 128 rows
+  CUtensorMap tmap_x;  // activations [M][K] fp16, box BN rows × 64, 128-byte swizzle
   const void* x;       // [M, K] fp16
   const uint8_t* w;    // int4 codes [N][K/2] or q4_K blocks [N][K/256][144]
   const uint8_t* scales;
@@ -34,7 +43,14 @@ struct TC5Params {
   int M, N, K;
   int nb, zb, block_shift;
   int BN;              // batch tile (UMMA N), multiple of 16
-  int tmem_cols;       // power of two >= max(32, BN)
+  int tmem_cols;       // power of two >= max(32, 2·BN): two accumulator tiles
+  int S;               // CTAs of a cluster (K slices)
+  int nks;             // 64-k stages per CTA (K / S / 64, a multiple of 4)
+  int NR, NX;          // raw-weight slots, activation slots (64 k each)
+  int spr;             // 64-k stages per raw slot (a power of two)
+  int raw_pitch;       // bytes per weight row in a raw slot
+  int raw_bytes;       // bytes of one raw slot (128 rows)
+  int off_x, off_raw, off_bar;  // shared-memory offsets (A slots start at 0)
 };
 
 __device__ __forceinline__ uint64_t umma_smem_desc_sw128(uint32_t saddr) {
@@ -101,101 +117,135 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
-// Raw data of one 64-k stage of one weight row, fetched ahead into registers.
-struct RawStage {
-  uint4 c0, c1, c2;  // int4: codes in c0, c1; q4_K: header in c0, codes in c1, c2
-  uint32_t sz;       // int4: fp16 scale bits | zero-point << 16
-};
-
+// Dequantize half h (32 k) of one stage of one weight row into 16 fp16x2
+// words in natural k order.  raw: the stage's 32 code bytes of the row in
+// shared memory; hdr (q4_K): the super-block's 16-byte header; sz (int4): fp16
+// scale bits | zero-point << 16.
 template <Fmt F>
-__device__ __forceinline__ void fetch_stage(const TC5Params& p, int row, int s, RawStage& r) {
-  const int k0 = s * 64;
-  if (row >= p.N) {
-    r.c0 = r.c1 = r.c2 = make_uint4(0u, 0u, 0u, 0u);
-    r.sz = 8u << 16;
-    return;
-  }
+__device__ __forceinline__ void dequant_stage(int s, int h, const uint8_t* raw, const uint8_t* hdr, uint32_t sz,
+                                              uint32_t (&o)[16]) {
   if constexpr (F == Fmt::Int4) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.w + static_cast<long long>(row) * (p.K / 2) + k0 / 2);
-    r.c0 = __ldcs(src);
-    r.c1 = __ldcs(src + 1);
-    const int b = k0 >> p.block_shift;  // blocks of >= 64 k: one scale / zero-point per stage
-    uint32_t z = 8u;
-    if (p.zeros) z = (p.zeros[static_cast<long long>(row) * p.zb + (b >> 1)] >> ((b & 1) * 4)) & 15u;
-    r.sz = reinterpret_cast<const uint16_t*>(p.scales)[static_cast<long long>(row) * p.nb + b] | (z << 16);
-  } else {
-    const int sb = k0 >> 8, pp = (k0 & 255) >> 6;
-    const uint8_t* blk = p.w + (static_cast<long long>(row) * (p.K / 256) + sb) * 144;
-    r.c0 = __ldcs(reinterpret_cast<const uint4*>(blk));
-    r.c1 = __ldcs(reinterpret_cast<const uint4*>(blk + 16 + 32 * pp));
-    r.c2 = __ldcs(reinterpret_cast<const uint4*>(blk + 32 + 32 * pp));
-  }
-}
-
-// Dequantize one stage of one row into 32 fp16x2 words (8 chunks of 8).
-// int4 chunk c holds codes of k = 8c + {0,4,1,5,2,6,3,7} (the activation tile
-// is permuted the same way); q4_K chunks are in natural k order.
-template <Fmt F>
-__device__ __forceinline__ void dequant_stage(const TC5Params& p, int s, const RawStage& r, uint32_t (&h)[32]) {
-  if constexpr (F == Fmt::Int4) {
-    const uint32_t sbits = r.sz & 0xFFFFu, z = r.sz >> 16;
+    const uint4 c = *reinterpret_cast<const uint4*>(raw + 16 * h);
+    const uint32_t sbits = sz & 0xFFFFu, z = sz >> 16;
     const uint32_t s2 = sbits | (sbits << 16);
-    const uint32_t zl = (0x6400u | z) * 0x00010001u, zh = (0x5400u | (z << 4)) * 0x00010001u;
-    const uint32_t words[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
+    // (1024 + z, 64 + z): subtracted from (1024 + q_even, 64 + q_odd) gives (q - z) exactly
+    const uint32_t zz = (0x6400u | z) | ((0x5400u | (z << 4)) << 16);
+    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int wd = 0; wd < 8; ++wd) {
-      const uint32_t v = words[wd], v8 = v >> 8;
-      uint32_t q[4];
-      q[0] = hsub2_f(lop3_or(v, 0x000F000Fu, 0x64006400u), zl);   // (n0, n4) - z, exact
-      q[1] = hsub2_f(lop3_or(v, 0x00F000F0u, 0x54005400u), zh);   // (n1, n5) - z
-      q[2] = hsub2_f(lop3_or(v8, 0x000F000Fu, 0x64006400u), zl);  // (n2, n6) - z
-      q[3] = hsub2_f(lop3_or(v8, 0x00F000F0u, 0x54005400u), zh);  // (n3, n7) - z
+    for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) h[wd * 4 + e] = hmul2_f(q[e], s2);  // RN16((q - z)·s): one rounding
+      for (int bt = 0; bt < 4; ++bt) {
+        // byte bt (codes k = 2bt, 2bt+1) into both halves, then the low nibble
+        // in the low half and the high nibble in the high half
+        const uint32_t t = __byte_perm(words[wd], 0u, 0x1010u + 0x0101u * static_cast<uint32_t>(bt));
+        o[wd * 4 + bt] = hmul2_f(hsub2_f(lop3_or(t, 0x00F0000Fu, 0x54006400u), zz), s2);
+      }
     }
   } else {
+    const uint4 c1 = *reinterpret_cast<const uint4*>(raw), c2 = *reinterpret_cast<const uint4*>(raw + 16);
+    const uint4 hd = *reinterpret_cast<const uint4*>(hdr);
     const int pp = ((s * 64) & 255) >> 6;
     uint32_t sc2, mn2;
-    q4k_scale_min_pair(r.c0.y, r.c0.z, r.c0.w, static_cast<uint32_t>(pp & 1), static_cast<uint32_t>(pp >> 1), sc2, mn2);
-    const float d = h16_to_f32(r.c0.x), dm = h16_to_f32(r.c0.x >> 16);
-    const float A0 = __fmul_rn(d, static_cast<float>(sc2 & 0xFFu)), A1 = __fmul_rn(d, static_cast<float>(sc2 >> 8));
-    const float B0 = -__fmul_rn(dm, static_cast<float>(mn2 & 0xFFu)), B1 = -__fmul_rn(dm, static_cast<float>(mn2 >> 8));
-    const uint32_t words[8] = {r.c1.x, r.c1.y, r.c1.z, r.c1.w, r.c2.x, r.c2.y, r.c2.z, r.c2.w};
+    q4k_scale_min_pair(hd.y, hd.z, hd.w, static_cast<uint32_t>(pp & 1), static_cast<uint32_t>(pp >> 1), sc2, mn2);
+    const float d = h16_to_f32(hd.x), dm = h16_to_f32(hd.x >> 16);
+    // half 0: chunk 2pp (low nibbles), half 1: chunk 2pp+1 (high nibbles)
+    const uint32_t scv = h ? (sc2 >> 8) : (sc2 & 0xFFu), mnv = h ? (mn2 >> 8) : (mn2 & 0xFFu);
+    const float A = __fmul_rn(d, static_cast<float>(scv)), B = -__fmul_rn(dm, static_cast<float>(mnv));
+    const uint32_t words[8] = {c1.x, c1.y, c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
+    const int sh = 4 * h;
 #pragma unroll
     for (int wd = 0; wd < 8; ++wd) {
-      const uint32_t v = words[wd];
-      float lo[4], hi[4];
+      const uint32_t v = words[wd] >> sh;
+      float f[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        lo[e] = fmaf(A0, __uint_as_float(0x4B000000u | ((v >> (8 * e)) & 15u)) - 8388608.0f, B0);
-        hi[e] = fmaf(A1, __uint_as_float(0x4B000000u | ((v >> (8 * e + 4)) & 15u)) - 8388608.0f, B1);
-      }
-      h[wd * 2 + 0] = pack_f16x2(lo[0], lo[1]);
-      h[wd * 2 + 1] = pack_f16x2(lo[2], lo[3]);
-      h[16 + wd * 2 + 0] = pack_f16x2(hi[0], hi[1]);
-      h[16 + wd * 2 + 1] = pack_f16x2(hi[2], hi[3]);
+      for (int e = 0; e < 4; ++e) f[e] = fmaf(A, __uint_as_float(0x4B000000u | ((v >> (8 * e)) & 15u)) - 8388608.0f, B);
+      o[wd * 2 + 0] = pack_f16x2(f[0], f[1]);
+      o[wd * 2 + 1] = pack_f16x2(f[2], f[3]);
     }
   }
 }
 
-constexpr int kTc5Prefetch = 4;  // stages of raw weights in flight per thread
+// int4 scale and zero-point of stage s of weight row `row` (packed fp16 | z << 16)
+__device__ __forceinline__ uint32_t fetch_sz(const TC5Params& p, int row, int s) {
+  if (row >= p.N) return 8u << 16;
+  const int b = (s * 64) >> p.block_shift;  // blocks of >= 64 k: one scale / zero-point per stage
+  uint32_t z = 8u;
+  if (p.zeros) z = (__ldg(p.zeros + static_cast<long long>(row) * p.zb + (b >> 1)) >> ((b & 1) * 4)) & 15u;
+  return __ldg(reinterpret_cast<const unsigned short*>(p.scales) + static_cast<long long>(row) * p.nb + b) | (z << 16);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most n of this thread's commit groups are pending (n = 0..7)
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
+}
+
+__device__ __forceinline__ uint32_t tc5_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void tc5_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float tc5_dsmem_ld(const float* local, uint32_t rank) {
+  uint32_t a;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+
+constexpr int kTc5SzAhead = 8;  // int4 scale / zero-point words fetched ahead in registers
+constexpr int kTc5NA = 4;       // A slots (16 KB each)
+constexpr int kTc5Warps = 10;   // 8 dequant / epilogue warps, producer, MMA issuer
+
+__device__ __forceinline__ void tc5_arrive(uint64_t* bar) {
+  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
 
 template <Fmt F>
-__global__ void __launch_bounds__(128, 2) gemm_tc5_kernel(const TC5Params p) {
+__global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __grid_constant__ TC5Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* A[2] = {smem, smem + 16384};
-  const int bsz = ((p.BN * 128) + 1023) & ~1023;
-  uint8_t* B[2] = {smem + 32768, smem + 32768 + bsz};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 32768 + 2 * bsz);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  uint64_t* raw_empty = raw_full + p.NR;
+  uint64_t* x_full = raw_empty + p.NR;
+  uint64_t* x_empty = x_full + p.NX;
+  uint64_t* a_full = x_empty + p.NX;
+  uint64_t* a_empty = a_full + kTc5NA;
+  uint64_t* done = a_empty + kTc5NA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int n0 = blockIdx.x * 128;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = p.S > 1 ? tc5_cluster_rank() : 0u;
+  const int n0 = (blockIdx.x / p.S) * 128;
   const int m0 = blockIdx.y * p.BN;
-  const int row = n0 + tid;  // weight row this thread dequantizes (TMEM lane tid)
+  const int s_begin = static_cast<int>(rank) * p.nks;  // first global 64-k stage of this CTA
+  const int nks = p.nks;
+  const int x_bytes = p.BN * 128;
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -203,9 +253,20 @@ __global__ void __launch_bounds__(128, 2) gemm_tc5_kernel(const TC5Params p) {
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+  if (tid == 32) {
+    for (int i = 0; i < p.NR; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 8);  // one arrival per dequant warp
+    }
+    for (int i = 0; i < p.NX; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], 1);  // tcgen05.commit
+    }
+    for (int i = 0; i < kTc5NA; ++i) {
+      mbar_init(&a_full[i], 8);
+      mbar_init(&a_empty[i], 1);
+    }
+    mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -213,79 +274,175 @@ __global__ void __launch_bounds__(128, 2) gemm_tc5_kernel(const TC5Params p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t idesc = umma_idesc_f16(p.BN);
-  const int nks = p.K / 64;
-  const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x);
 
-  RawStage raw[kTc5Prefetch];
-#pragma unroll
-  for (int i = 0; i < kTc5Prefetch; ++i)
-    if (i < nks) fetch_stage<F>(p, row, i, raw[i]);
-
-  for (int s0 = 0; s0 < nks; s0 += kTc5Prefetch) {
-#pragma unroll
-    for (int i = 0; i < kTc5Prefetch; ++i) {
-      const int s = s0 + i;
-      if (s >= nks) break;
-      const int slot = s & 1;
-      if (s >= 2 && !*abort_flag) {
-        if (!mbar_wait_bounded(&bars[slot], static_cast<uint32_t>(((s - 2) >> 1) & 1))) *abort_flag = 1;
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int rs = 0, ru = 0, xs = 0, xu = 0;  // slot index and use count of each ring
+      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+        const int gs = s_begin + ls;
+        if ((ls & (p.spr - 1)) == 0) {
+          if (ru > 0 && !mbar_wait_bounded(&raw_empty[rs], static_cast<uint32_t>((ru - 1) & 1))) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&raw_full[rs], static_cast<uint32_t>(p.raw_bytes));
+          const int c0 = F == Fmt::Int4 ? gs * 32 : (gs >> 2) * 144;  // byte column of the slot's first k
+          tma_load_2d(smem + p.off_raw + rs * p.raw_bytes, &p.tmap_w, c0, n0, &raw_full[rs]);
+          if (++rs == p.NR) {
+            rs = 0;
+            ++ru;
+          }
+        }
+        if (xu > 0 && !mbar_wait_bounded(&x_empty[xs], static_cast<uint32_t>((xu - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&x_full[xs], static_cast<uint32_t>(x_bytes));
+        tma_load_2d(smem + p.off_x + xs * ((x_bytes + 1023) & ~1023), &p.tmap_x, gs * 64, m0, &x_full[xs]);
+        if (++xs == p.NX) {
+          xs = 0;
+          ++xu;
+        }
       }
-      __syncthreads();
-      if (*abort_flag) break;
-      const int k0 = s * 64;
-      uint32_t h[32];
-      dequant_stage<F>(p, s, raw[i], h);
-      if (s + kTc5Prefetch < nks) fetch_stage<F>(p, row, s + kTc5Prefetch, raw[i]);
-      uint8_t* a = A[slot];
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(a + sw128(tid, c)) = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
-      // ---- B: activation rows m0 .. m0+BN-1, k0 .. k0+63 (zero past M)
-      uint8_t* bt = B[slot];
-      for (int c = tid; c < p.BN * 8; c += 128) {
-        const int n = c >> 3, kc = c & 7;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (m0 + n < p.M) v = *reinterpret_cast<const uint4*>(xg + static_cast<long long>(m0 + n) * p.K + k0 + 8 * kc);
-        if constexpr (F == Fmt::Int4)  // same k order as the A chunks: x0 x4 x1 x5 x2 x6 x3 x7
-          v = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632), __byte_perm(v.y, v.w, 0x5410),
-                         __byte_perm(v.y, v.w, 0x7632));
-        *reinterpret_cast<uint4*>(bt + sw128(n, kc)) = v;
-      }
-      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(p.BN);
+      int xs = 0, xu = 0;
+      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+        const int a = ls & (kTc5NA - 1), au = ls / kTc5NA;
+        if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>(au & 1)) ||
+            !mbar_wait_bounded(&x_full[xs], static_cast<uint32_t>(xu & 1))) {
+          *abort_flag = 1;
+          break;
+        }
         tc_fence_after();
-        const uint64_t ad = umma_smem_desc_sw128(smem_u32(a));
-        const uint64_t bd = umma_smem_desc_sw128(smem_u32(bt));
+        const uint64_t ad = umma_smem_desc_sw128(smem_u32(smem + a * 16384));
+        const uint64_t bd = umma_smem_desc_sw128(smem_u32(smem + p.off_x + xs * ((x_bytes + 1023) & ~1023)));
+        // even and odd stages accumulate into two TMEM tiles (columns [0, BN) and
+        // [BN, 2BN)), so consecutive stages' MMAs do not wait for each other
+        const uint32_t dacc = tmem + static_cast<uint32_t>((ls & 1) * p.BN);
 #pragma unroll
         for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
-          umma_f16(tmem, ad + 2ull * j, bd + 2ull * j, idesc, (s > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&bars[slot]);
+          umma_f16(dacc, ad + 2ull * j, bd + 2ull * j, idesc, (ls > 1 || j > 0) ? 1u : 0u);
+        umma_commit(&a_empty[a]);
+        umma_commit(&x_empty[xs]);
+        if (++xs == p.NX) {
+          xs = 0;
+          ++xu;
+        }
       }
+      umma_commit(done);  // arrives when every MMA issued above has completed
     }
-    if (*abort_flag) break;
-  }
-  // ---- wait for the last stage's MMAs, then read the accumulator
-  const int last = nks - 1;
-  bool ok = !*abort_flag;
-  if (ok && !mbar_wait_bounded(&bars[last & 1], static_cast<uint32_t>((last >> 1) & 1))) ok = false;
-  if (ok && nks >= 2 && !mbar_wait_bounded(&bars[(last - 1) & 1], static_cast<uint32_t>(((last - 1) >> 1) & 1)))
-    ok = false;
-  tc_fence_after();
-  if (ok) {
-    __half* y = reinterpret_cast<__half*>(p.y);
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    for (int c0 = 0; c0 < p.BN; c0 += 16) {
-      uint32_t r[16];
-      tmem_ld16(lane_base + c0, r);
+  } else {
+    // ------------------------------------------------------------ dequant warps
+    const int rl = tid & 127, h = tid >> 7;  // weight row (TMEM lane) and which 32 k of a stage
+    const int row = n0 + rl;
+    uint32_t szr[kTc5SzAhead];
+    if constexpr (F == Fmt::Int4) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int m = m0 + c0 + j;
-        if (m < p.M && row < p.N) y[static_cast<long long>(m) * p.N + row] = __float2half_rn(__uint_as_float(r[j]));
+      for (int i = 0; i < kTc5SzAhead; ++i) szr[i] = i < nks ? fetch_sz(p, row, s_begin + i) : 0u;
+    }
+    int rs = 0, ru = 0;
+    for (int s0 = 0; s0 < nks; s0 += kTc5SzAhead) {
+#pragma unroll
+      for (int i = 0; i < kTc5SzAhead; ++i) {
+        const int ls = s0 + i;
+        if (ls >= nks || *abort_flag) break;
+        if ((ls & (p.spr - 1)) == 0 && !mbar_wait_bounded(&raw_full[rs], static_cast<uint32_t>(ru & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        const int a = ls & (kTc5NA - 1), au = ls / kTc5NA;
+        if (au > 0 && !mbar_wait_bounded(&a_empty[a], static_cast<uint32_t>((au - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        uint32_t sz = 0u;
+        if constexpr (F == Fmt::Int4) {
+          sz = szr[i];
+          if (ls + kTc5SzAhead < nks) szr[i] = fetch_sz(p, row, s_begin + ls + kTc5SzAhead);
+        }
+        const uint8_t* rrow = smem + p.off_raw + rs * p.raw_bytes + rl * p.raw_pitch;
+        const uint8_t* codes = F == Fmt::Int4 ? rrow + 32 * (ls & (p.spr - 1)) : rrow + 16 + 32 * (ls & 3);
+        uint32_t o[16];
+        dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, o);
+        uint8_t* at = smem + a * 16384;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(at + sw128(rl, 4 * h + c)) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) tc5_arrive(&a_full[a]);
+        if ((ls & (p.spr - 1)) == p.spr - 1) {  // every stage of the raw slot is dequantized
+          if (lane == 0) tc5_arrive(&raw_empty[rs]);
+          if (++rs == p.NR) {
+            rs = 0;
+            ++ru;
+          }
+        }
       }
     }
+  }
+
+  // ---- epilogue: every thread waits for the last MMAs, the dequant warps read TMEM
+  bool ok = !*abort_flag && mbar_wait_bounded(done, 0u);
+  tc_fence_after();
+  const int lq = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quarter, column half
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+  const int trow = lq * 32 + lane;                // tile row this thread reads back
+  const bool split_cols = p.BN % 32 == 0;        // both column halves are whole 16-column groups
+  const int cols_per = split_cols ? p.BN / 2 : p.BN;
+  const int c_begin = split_cols ? ch * cols_per : 0;
+  const bool reads = warp < 8 && (split_cols || ch == 0);
+  __half* y = reinterpret_cast<__half*>(p.y);
+  // the two accumulator tiles of a 16-column group, added (fixed order)
+  auto acc16 = [&](int c0, float (&v)[16]) {
+    uint32_t r0[16], r1[16];
+    tmem_ld16(lane_base + c0, r0);
+    tmem_ld16(lane_base + p.BN + c0, r1);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
+  };
+  if (p.S == 1) {
+    if (ok && reads) {
+      for (int c0 = c_begin; c0 < c_begin + cols_per; c0 += 16) {
+        float v[16];
+        acc16(c0, v);
+        const int yrow = n0 + trow;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + c0 + j;
+          if (m < p.M && yrow < p.N) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(v[j]);
+        }
+      }
+    }
+  } else {
+    // K split over the cluster: park the fp32 tile [128][BN] in this CTA's shared
+    // memory (the rings are drained), then each rank adds 128/S rows over all ranks
+    float* acc = reinterpret_cast<float*>(smem);
+    __syncthreads();
+    if (reads) {
+      for (int c0 = c_begin; c0 < c_begin + cols_per; c0 += 16) {
+        float v[16];
+        if (ok) acc16(c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[trow * p.BN + c0 + j] = ok ? v[j] : 0.f;
+      }
+    }
+    tc5_cluster_sync();
+    const int rows_per = 128 / p.S;
+    const int items = rows_per * p.BN;
+    for (int i = tid; i < items; i += kTc5Warps * 32) {
+      const int rr = static_cast<int>(rank) * rows_per + i / p.BN, c = i % p.BN;
+      float sum = 0.f;
+      for (int q = 0; q < p.S; ++q) sum += tc5_dsmem_ld(acc + rr * p.BN + c, static_cast<uint32_t>(q));
+      const int m = m0 + c, yrow = n0 + rr;
+      if (m < p.M && yrow < p.N && !*abort_flag) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(sum);
+    }
+    tc5_cluster_sync();
   }
   tc_fence_before();
   __syncthreads();
