@@ -261,6 +261,23 @@ def _traffic(workload: str):
     return None
 
 
+def max_over_ranks(vals, dist, device):
+    """Each timing as the maximum over ranks (the slowest rank sets the job time)."""
+    if dist is None:
+        return [float(v) for v in vals]
+    import torch
+
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_gbs(world: int, bytes_per_call: int, calls: int, ms: float) -> float:
+    """Whole-job GB/s: every rank streams its own weights (replicas), so the job
+    moves world × bytes × calls in the max-over-ranks time."""
+    return world * bytes_per_call * calls / (ms * 1e-3) / 1e9
+
+
 def run_ours(args, w, wname, rank, world, dist):
     import torch
 
@@ -355,15 +372,12 @@ def run_ours(args, w, wname, rank, world, dist):
     ms_e2e = t0.elapsed_time(t1)
     steps_e2e = reps_e * Ge
 
-    if dist is not None:
-        t = torch.tensor([ms, ms_e2e], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], dist, "cuda")
 
     bytes_call = d.bytes
     ms_step = ms / steps
-    value = world * bytes_call * steps / (ms * 1e-3) / 1e9
-    e2e_value = world * bytes_call * steps_e2e / (ms_e2e * 1e-3) / 1e9
+    value = job_gbs(world, bytes_call, steps, ms)
+    e2e_value = job_gbs(world, bytes_call, steps_e2e, ms_e2e)
     peak, peak_kind = _peaks()
     # one launch of the kernel per step: its average duration over the timed region
     achieved = bytes_call / (ms_step * 1e-3) / 1e9
