@@ -68,6 +68,12 @@ int ilog2_int(int v) {
   return r;
 }
 
+// WQ_PDL=0 turns programmatic dependent launch off (A/B runs).
+bool pdl_enabled() {
+  const char* v = std::getenv("WQ_PDL");
+  return !(v && std::atoi(v) == 0);
+}
+
 int launch_check(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
@@ -449,7 +455,18 @@ int launch_tc(Fmt f, int layout, const TCPlan& plan, cudaStream_t st) {
       configured[slot][dev] = true;
     }
   }
-  fn<<<plan.grid, plan.threads, plan.smem, st>>>(plan.p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.grid, 1, 1);
+  cfg.blockDim = dim3(plan.threads, 1, 1);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, plan.p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemv_tc launch: ") + cudaGetErrorString(e));
   return launch_check("gemv_tc launch");
 }
 
@@ -603,11 +620,6 @@ bool plan_v1(int M, int N, int K, int block_size, int sms, V1Plan* out) {
   return false;
 }
 
-// WQ_PDL=0 turns programmatic dependent launch off (A/B runs).
-bool pdl_enabled() {
-  const char* v = std::getenv("WQ_PDL");
-  return !(v && std::atoi(v) == 0);
-}
 
 // ---------------------------------------------------------------------------
 // B200_V1 int4 GEMV, register-streaming kernel: planner and launcher

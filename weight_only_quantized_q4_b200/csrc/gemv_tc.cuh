@@ -128,6 +128,9 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
     fence_barrier_init();
   }
   __syncthreads();
+  // The next kernel in the stream may start streaming its weights now; this one
+  // waits for the previous kernel only where it reads x (producer) or writes y.
+  grid_launch_dependents();
 
   // ------------------------------------------------------------ producer warp
   // All 32 lanes issue copies: lane 0 arms the stage's barrier, then lane j
@@ -151,6 +154,7 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
       const uint32_t xb = p.x_res ? (S == 0 ? p.M * 2u * p.K : 0u) : p.M * 2u * kc;
       mbar_arrive_expect_tx(&full[slot], sbytes + xb);
       bulk_g2s_stream(st, src + static_cast<long long>(S) * sbytes, sbytes, &full[slot], policy);
+      grid_wait_prior();  // x may be the previous kernel's output (returns at once after the first time)
       if (p.x_res) {
         if (S == 0) bulk_g2s(smem + p.off_xres, p.x, p.M * 2u * p.K, &full[slot]);
       } else {
@@ -231,6 +235,7 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
           bulk_g2s_stream(st + j * p.pitch, p.w + static_cast<long long>(r0 + j) * p.row_bytes + kofs, seg,
                           &full[slot], policy);
       }
+      grid_wait_prior();  // x may be the previous kernel's output (returns at once after the first time)
       if (p.x_res) {
         // activations for the whole kernel ride on the first stage's barrier
         if (S == 0 && lane == 0) bulk_g2s(smem + p.off_xres, p.x, p.M * 2u * p.K, &full[slot]);
@@ -260,6 +265,7 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
   }
 
   // ------------------------------------------------------------ consumer warps
+  grid_wait_prior();  // y may still be read or written by the previous kernel
   const int g = lane >> 2;  // fragment row (and batch column of B)
   const int t = lane & 3;   // fragment k-pair / output column pair
   const int nthr = W * 32;

@@ -79,11 +79,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// Programmatic dependent launch: let the next kernel in the stream start its
-// independent prologue now / wait until the previous kernel has completed and
-// its writes are visible (a no-op when launched without the attribute).
-__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void grid_wait_prior() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // One 128-k tile of a 16-row band (rows g, g + 8 of the lane) against batch
 // row g (or a zero buffer for lanes past M):
 //   y += s_r·(2^-24·Σ q·x − z_r·(2^-24·Σ x))   for columns 2t, 2t + 1.
@@ -168,7 +163,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
   __syncthreads();
   // The next kernel in the stream may start its own weight stream now; this
   // one only waits for the previous kernel where it reads x or writes y.
-  v1d::grid_launch_dependents();
+  grid_launch_dependents();
 
   // ---------------------------------------------------------------- producer
   if (warp == W) {
@@ -184,7 +179,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
       // they are copied next, ahead of the rest of the weight stream (a load
       // queued behind a deep weight stream waits for all of it).
       auto copy_x = [&]() {
-        v1d::grid_wait_prior();
+        grid_wait_prior();
         mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.M) * 2u * Kc);
         for (int m = 0; m < p.M; ++m)
           bulk_g2s(smem + p.off_x + m * 2 * Kc,
@@ -232,7 +227,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
 
   // ---------------------------------------------------------------- reducer
   if (warp == W + 1) {
-    v1d::grid_wait_prior();  // y may still be read or written by the previous kernel
+    grid_wait_prior();  // y may still be read or written by the previous kernel
     for (int bl = 0; bl < n_bl; ++bl) {
       const int s = bl & 1;
       v1d::bar_sync(v1d::kBarFull0 + s, nthr_all);
@@ -443,7 +438,7 @@ __global__ void __launch_bounds__(kV1RMaxWarps * 32, 1) gemv_v1r_kernel(const V1
   const int n_bl = b_end - b_begin;
   const int n_tiles = n_bl * p.tpb;  // the CTA's tiles are one contiguous range of the stream
   const uint8_t* base = p.w + static_cast<long long>(b_begin) * p.tpb * p.tb;
-  v1d::grid_launch_dependents();
+  grid_launch_dependents();
 
   const int nthr_all = (W + 1) * 32;
   float* red = reinterpret_cast<float*>(smem + p.off_red);
@@ -451,7 +446,7 @@ __global__ void __launch_bounds__(kV1RMaxWarps * 32, 1) gemv_v1r_kernel(const V1
 
   if (warp == W) {
     // ---------------------------------------------------------------- reducer
-    v1d::grid_wait_prior();  // y may still be read or written by the previous kernel
+    grid_wait_prior();  // y may still be read or written by the previous kernel
     for (int bl = 0; bl < n_bl; ++bl) {
       const int s = bl & 1;
       v1d::bar_sync(v1d::kBarFull0 + s, nthr_all);
@@ -482,7 +477,7 @@ __global__ void __launch_bounds__(kV1RMaxWarps * 32, 1) gemv_v1r_kernel(const V1
   float* xs = reinterpret_cast<float*>(smem + p.off_xs);
   uint8_t* xsm = smem + p.off_x;
   uint8_t* zbuf = smem + p.off_zero;
-  v1d::grid_wait_prior();  // x may be the previous kernel's output
+  grid_wait_prior();  // x may be the previous kernel's output
   {
     // x -> shared memory, and Σx (×2^-24) per (tile, batch column): four
     // threads per tile and column, 32 k each
