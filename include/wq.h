@@ -18,7 +18,19 @@
  *    then holds a one-line message (per calling thread).
  *  - wq_last_kernel() names the kernel variant the last successful launch on
  *    the calling thread used (a liveness label such as
- *    "int4.gemv.cc.m1.b128"), so a test can assert which path ran.
+ *    "int4.gemv.v1s.m1.c1"), so a test can assert which path ran.
+ *  - The decode GEMV kernels are launched with programmatic dependent launch:
+ *    a call may start streaming its (read-only) weights while the previous
+ *    kernel in the stream is still running, and waits for that kernel to
+ *    complete before it reads x or writes y.  Stream order is preserved for
+ *    the caller; a following kernel that itself uses programmatic dependent
+ *    launch must wait (griddepcontrol.wait) before reading y, as usual.
+ *  - The first call on a device configures kernel attributes and looks up the
+ *    driver's tensor-map encoder; make it before capturing a CUDA graph.
+ *  - Environment variables read at each call, for tests and tuning only:
+ *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r) pins a kernel
+ *    family, WQ_PDL=0 disables programmatic dependent launch, and WQ_V1_*,
+ *    WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch geometry.
  *
  * Weight formats (canonical byte layouts, layout version WQ_LAYOUT_CANONICAL):
  *  - int4 MatMulNBits-style blocks (onnx-genai PR #1000, "What it does": int4
