@@ -341,19 +341,50 @@ def run_ours(args, w, wname, rank, world, dist):
     per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(n_ev)]
     avg_launch_ms = float(np.mean(per_launch))
 
-    # e2e: pinned host x in, device GEMV, pinned host y out, every step, through the API
-    xh = torch.empty_like(d.x, device="cpu").pin_memory()
-    xh.copy_(d.x.cpu())
-    yh = torch.empty_like(d.y, device="cpu").pin_memory()
-    xd, yd = torch.empty_like(d.x), torch.empty_like(d.y)
+    # e2e: every step copies its x in from pinned host memory, runs the GEMV
+    # through the API and copies its y out to pinned host memory.  Steps are
+    # pipelined as a serving loop would: the host-to-device copy of step i+1
+    # and the device-to-host copy of step i-1 run on two copy streams while the
+    # GEMV of step i runs, with NB device buffers per tensor and events guarding
+    # every reuse (x slot j is rewritten only after the GEMV that read it, y
+    # slot j only after the copy that drained it).
+    NB = 3
+    xh = [torch.empty_like(d.x, device="cpu").pin_memory() for _ in range(NB)]
+    for h in xh:
+        h.copy_(d.x.cpu())
+    yh = [torch.empty_like(d.y, device="cpu").pin_memory() for _ in range(NB)]
+    xd = [torch.empty_like(d.x) for _ in range(NB)]
+    yd = [torch.empty_like(d.y) for _ in range(NB)]
     Ge = min(G, 256)
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_x = [torch.cuda.Event() for _ in range(Ge)]
+    ev_k = [torch.cuda.Event() for _ in range(Ge)]
+    ev_y = [torch.cuda.Event() for _ in range(Ge)]
     ge = torch.cuda.CUDAGraph()
     with torch.cuda.graph(ge, stream=stream):
         cs = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(cs)
+        h2d_s.wait_event(fork)
+        d2h_s.wait_event(fork)
         for i in range(Ge):
-            xd.copy_(xh, non_blocking=True)
-            d.call(i, x=xd, y=yd, stream=cs)
-            yh.copy_(yd, non_blocking=True)
+            j = i % NB
+            with torch.cuda.stream(h2d_s):
+                if i >= NB:
+                    h2d_s.wait_event(ev_k[i - NB])  # the GEMV that read x slot j is done
+                xd[j].copy_(xh[j], non_blocking=True)
+                ev_x[i].record(h2d_s)
+            cs.wait_event(ev_x[i])
+            if i >= NB:
+                cs.wait_event(ev_y[i - NB])  # y slot j has been copied out
+            d.call(i, x=xd[j], y=yd[j], stream=cs)
+            ev_k[i].record(cs)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_k[i])
+                yh[j].copy_(yd[j], non_blocking=True)
+                ev_y[i].record(d2h_s)
+        cs.wait_event(ev_x[Ge - 1])
+        cs.wait_event(ev_y[Ge - 1])
     for _ in range(2):
         ge.replay()
     torch.cuda.synchronize()
@@ -371,6 +402,11 @@ def run_ours(args, w, wname, rank, world, dist):
     barrier()
     ms_e2e = t0.elapsed_time(t1)
     steps_e2e = reps_e * Ge
+    # the last step's result (same x, an identical weight copy) must have reached
+    # host memory bit for bit: the kernels are deterministic, so a difference
+    # would mean a missing dependency in the pipelined copies
+    if not torch.equal(yh[(Ge - 1) % NB].view(torch.int16), d.y.cpu().view(torch.int16)):
+        raise RuntimeError("e2e: host copy of y differs from the device result")
 
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], dist, "cuda")
 
@@ -406,7 +442,9 @@ def run_ours(args, w, wname, rank, world, dist):
                 "h2d_bytes_per_step": int(d.x.numel() * d.x.element_size()),
                 "d2h_bytes_per_step": int(d.y.numel() * d.y.element_size()),
                 "us_per_call": round(ms_e2e / steps_e2e * 1e3, 3),
-                "how": "per step: pinned x -> device, GEMV through the C ABI, y -> pinned host; graph-captured"},
+                "how": "per step: pinned x -> device, GEMV through the C ABI, y -> pinned host; steps pipelined over "
+                       "two copy streams with 3 device buffers per tensor (copies of neighbouring steps overlap the "
+                       "GEMV); graph-captured"},
         "gpu_launches": steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": _traffic(wname),
