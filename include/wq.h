@@ -73,7 +73,7 @@ extern "C" {
 #define WQ_ERR_CUDA (-4)        /* a CUDA runtime call or launch failed; see wq_last_error() */
 #define WQ_ERR_DEVICE (-5)      /* the current device is not sm_100 */
 #define WQ_ERR_TIMEOUT (-6)     /* a bounded device-side wait expired (see wq_device_status) */
-#define WQ_ERR_UNSUPPORTED (-7) /* valid arguments this build has no kernel for */
+#define WQ_ERR_UNSUPPORTED (-7) /* valid arguments this library version has no kernel for */
 
 /* Weight layout versions. */
 #define WQ_LAYOUT_CANONICAL 0
@@ -181,7 +181,7 @@ int wq_build_q4k_dsc_device(const void* w_q4k, void* out, int N, int K, void* st
  * ------------------------------------------------------------------------- */
 const char* wq_last_error(void);   /* message of the last failure on this thread */
 const char* wq_last_kernel(void);  /* liveness label of the last launch on this thread */
-int wq_layout_version(void);       /* newest layout version this build reads */
+int wq_layout_version(void);       /* newest layout version this library reads */
 const char* wq_build_info(void);   /* "sm_100a ..." build description */
 
 /* Synchronizes the current device, then reads and clears the device-side
