@@ -29,8 +29,10 @@
  *    driver's tensor-map encoder; make it before capturing a CUDA graph.
  *  - Environment variables read at each call, for tests and tuning only:
  *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r) pins a kernel
- *    family, WQ_PDL=0 disables programmatic dependent launch, and WQ_V1_*,
- *    WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch geometry.
+ *    family (a call that family cannot run returns WQ_ERR_UNSUPPORTED; there
+ *    is no silent substitute), WQ_PDL=0 disables programmatic dependent
+ *    launch, and WQ_V1_*, WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch
+ *    geometry.
  *
  * Weight formats (canonical byte layouts, layout version WQ_LAYOUT_CANONICAL):
  *  - int4 MatMulNBits-style blocks (onnx-genai PR #1000, "What it does": int4
@@ -181,13 +183,23 @@ int wq_build_q4k_dsc_device(const void* w_q4k, void* out, int N, int K, void* st
  * ------------------------------------------------------------------------- */
 const char* wq_last_error(void);   /* message of the last failure on this thread */
 const char* wq_last_kernel(void);  /* liveness label of the last launch on this thread */
-int wq_layout_version(void);       /* newest layout version this library reads */
+int wq_layout_version(void);       /* newest layout version this library reads (WQ_LAYOUT_B200_V1) */
 const char* wq_build_info(void);   /* "sm_100a ..." build description */
 
 /* Synchronizes the current device, then reads and clears the device-side
  * error word that bounded waits set when they give up.  Returns WQ_OK or
  * WQ_ERR_TIMEOUT (or WQ_ERR_CUDA if the synchronization itself fails). */
 int wq_device_status(void);
+
+/* Test hook for the failure path of bounded device waits (no counterpart on
+ * the pages; it exists so the timeout status can be tested without faulting a
+ * GPU).  Enqueues one tiny kernel on `stream` whose single thread waits on an
+ * mbarrier that nothing arrives at, with no copy in flight, and gives up after
+ * limit_ns nanoseconds (1e3 .. 1e9), recording the timeout in the device
+ * error word exactly as a real wait that gives up does; the kernel then
+ * returns.  The next wq_device_status() reports WQ_ERR_TIMEOUT once.
+ * Errors: WQ_ERR_ARG (limit out of range), WQ_ERR_DEVICE, WQ_ERR_CUDA. */
+int wq_test_expire_wait(unsigned long long limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

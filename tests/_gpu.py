@@ -24,6 +24,40 @@ def bf16_bits_of(t: torch.Tensor) -> np.ndarray:
     return t.cpu().view(torch.int16).numpy().view(np.uint16)
 
 
+GUARD = 256       # canary bytes on each side of every output buffer
+CANARY = 0xA5
+
+
+class Guarded:
+    """A device output buffer with GUARD canary bytes on each side.
+
+    compute-sanitizer is not available on the GPU pool, so out-of-bounds
+    stores are caught this way instead: every kernel output in the tests
+    lives between two bands of known bytes, and check() asserts the bands
+    are untouched after the call.  `lead` extra bytes before the tensor
+    (part of the front band) give a tensor an odd 2-byte offset."""
+
+    def __init__(self, shape, dtype, lead: int = 0):
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.lead, self.n = GUARD + lead, n
+        self.buf = torch.full((self.lead + n + GUARD,), CANARY, dtype=torch.uint8, device=DEV)
+        self.ptr = self.buf.data_ptr() + self.lead
+        self.t = self.buf[self.lead:self.lead + n].view(dtype).view(shape) if lead % 16 == 0 else None
+
+    def check(self, what: str = "output") -> None:
+        b = self.buf.cpu().numpy()
+        head, tail = b[:self.lead], b[self.lead + self.n:]
+        if (head != CANARY).any() or (tail != CANARY).any():
+            hb = np.flatnonzero(head != CANARY)
+            tb = np.flatnonzero(tail != CANARY)
+            raise AssertionError(f"{what}: store outside the output buffer (bytes before: {hb[:8].tolist()}, "
+                                 f"bytes after: {tb[:8].tolist()})")
+
+
+def guarded_empty(shape, dtype):
+    return Guarded(shape, dtype)
+
+
 def check(y_dev: np.ndarray, W: np.ndarray, x: np.ndarray, what: str) -> None:
     """Accept iff |y − y_ref| ≤ 2e-3·Σ|w·x| + 1e-3 for every element."""
     y_ref = oracle.gemv(W, x)
@@ -46,18 +80,22 @@ class Int4Case:
         self.dw, self.ds = dev(self.w), dev(self.s)
         self.dz = dev(self.z) if self.z is not None else None
         if layout == wq.WQ_LAYOUT_B200_V1:
-            packed = torch.full((wq.wq_int4_packed_bytes(N, K, bs, layout),), 0x5A, dtype=torch.uint8, device=DEV)
-            wq.wq_repack_int4(self.dw, self.ds, self.dz, packed, N, K, bs, layout)
+            g = Guarded((wq.wq_int4_packed_bytes(N, K, bs, layout),), torch.uint8)
+            g.buf[g.lead:g.lead + g.n] = 0x5A
+            wq.wq_repack_int4(self.dw, self.ds, self.dz, g.t, N, K, bs, layout)
             torch.cuda.synchronize()
-            self.dw = packed
+            g.check("B200_V1 repack output")
+            self._packed_guard = g
+            self.dw = g.t
         self.dx = dev(self.x)
 
     def run(self, stream=None) -> np.ndarray:
-        y = torch.empty((self.M, self.N), dtype=torch.float16, device=DEV)
-        wq.gemv_int4_blockwise(self.dx, self.dw, self.ds, self.dz, y, self.M, self.N, self.K, self.bs,
+        g = Guarded((self.M, self.N), torch.float16)
+        wq.gemv_int4_blockwise(self.dx, self.dw, self.ds, self.dz, g.t, self.M, self.N, self.K, self.bs,
                                layout=self.layout, stream=stream)
         torch.cuda.synchronize()
-        return f16_of(y).astype(np.float64)
+        g.check(f"int4 y M={self.M} N={self.N} K={self.K}")
+        return f16_of(g.t).astype(np.float64)
 
     def W(self, rows=None):
         r = slice(None) if rows is None else rows
@@ -78,20 +116,23 @@ class Q4KCase:
 
     def plane_dev(self):
         if self._plane is None:
-            P = torch.empty((self.K // 32, self.N, 2), dtype=torch.float32, device=DEV)
-            wq.wq_build_q4k_dsc_device(self.draw, P, self.N, self.K)
+            g = Guarded((self.K // 32, self.N, 2), torch.float32)
+            wq.wq_build_q4k_dsc_device(self.draw, g.t, self.N, self.K)
             torch.cuda.synchronize()
-            self._plane = P
+            g.check("W_dsc plane")
+            self._plane_guard = g
+            self._plane = g.t
         return self._plane
 
     def run(self, dsc: bool, stream=None) -> np.ndarray:
-        y = torch.empty((self.M, self.N), dtype=torch.float16, device=DEV)
+        g = Guarded((self.M, self.N), torch.float16)
         if dsc:
-            wq.gemv_q4k_dsc(self.dx, self.draw, self.plane_dev(), y, self.M, self.N, self.K, stream=stream)
+            wq.gemv_q4k_dsc(self.dx, self.draw, self.plane_dev(), g.t, self.M, self.N, self.K, stream=stream)
         else:
-            wq.gemv_q4k(self.dx, self.draw, y, self.M, self.N, self.K, stream=stream)
+            wq.gemv_q4k(self.dx, self.draw, g.t, self.M, self.N, self.K, stream=stream)
         torch.cuda.synchronize()
-        return f16_of(y).astype(np.float64)
+        g.check(f"q4k y dsc={dsc} M={self.M} N={self.N} K={self.K}")
+        return f16_of(g.t).astype(np.float64)
 
     def W(self, rows=None):
         if rows is None:
@@ -112,12 +153,13 @@ class BF16Case:
         self.dxbuf = dev(xbuf.view(np.int16)).view(torch.bfloat16)
 
     def run(self, stream=None) -> np.ndarray:
-        ybuf = torch.zeros(self.M * self.N + 8, dtype=torch.bfloat16, device=DEV)
-        yp = ybuf.data_ptr() + 2 * self.offset
-        wq.gemv_bf16(self.dxbuf.data_ptr() + 2 * self.offset, self.dwbuf.data_ptr() + 2 * self.offset, yp,
+        g = Guarded((self.M * self.N,), torch.bfloat16, lead=2 * self.offset)
+        wq.gemv_bf16(self.dxbuf.data_ptr() + 2 * self.offset, self.dwbuf.data_ptr() + 2 * self.offset, g.ptr,
                      self.M, self.N, self.K, stream=stream)
         torch.cuda.synchronize()
-        bits = bf16_bits_of(ybuf)[self.offset:self.offset + self.M * self.N].reshape(self.M, self.N)
+        g.check(f"bf16 y M={self.M} N={self.N} K={self.K} offset={self.offset}")
+        raw = g.buf[g.lead:g.lead + g.n].cpu().numpy()
+        bits = raw.view(np.uint16).reshape(self.M, self.N)
         return oracle.q4.bf16_bits_to_f64(bits)
 
     def W(self, rows=None):
@@ -133,7 +175,9 @@ VARIANTS = ("tc", "cc", "simple", "tc5", "v1s", "v1r", None)
 
 def each_variant(run, W, x, what):
     """Run `run()` under every forced GEMV variant (and the default); check each
-    against the oracle; return the liveness labels seen."""
+    against the oracle; return the liveness labels seen.  A forced family that
+    cannot run the call must say so (WQ_ERR_UNSUPPORTED, label "unsupported");
+    one that runs must be the family that was asked for."""
     import os
 
     labels = {}
@@ -144,8 +188,16 @@ def each_variant(run, W, x, what):
                 os.environ.pop("WQ_FORCE_KERNEL", None)
             else:
                 os.environ["WQ_FORCE_KERNEL"] = v
-            y = run()
+            try:
+                y = run()
+            except wq.WQError as e:
+                if v is None or e.code != wq.WQ_ERR_UNSUPPORTED:
+                    raise
+                labels[v] = "unsupported"
+                continue
             labels[v or "default"] = wq.last_kernel()
+            if v is not None:
+                assert f".{v}." in labels[v], (what, v, labels[v])
             check(y, W, x, f"{what} [{v or 'default'} -> {labels[v or 'default']}]")
     finally:
         if old is None:

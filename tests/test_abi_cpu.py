@@ -72,6 +72,8 @@ def test_q4k_and_bf16_argument_errors():
     assert L.gemv_bf16(A16, A16, A16, 1, 0, 7, None) == _lib.WQ_ERR_ARG
     assert L.dequant_q4k(A16, None, A16, 4, 100, 0, None) == _lib.WQ_ERR_ARG
     assert L.wq_build_q4k_dsc(None, 4, 256, None) == _lib.WQ_ERR_ARG
+    assert L.wq_test_expire_wait(10, None) == _lib.WQ_ERR_ARG
+    assert L.wq_test_expire_wait(2 * 10**9, None) == _lib.WQ_ERR_ARG
 
 
 def test_v1_layout_argument_errors():
@@ -101,7 +103,7 @@ def test_size_queries():
     assert wq.wq_q4k_bytes(4096, 4096) == 4096 * 16 * 144
     assert wq.wq_q4k_dsc_bytes(4096, 11008) == 4096 * 11008 // 4
     assert wq.wq_q4k_dsc_bytes(4, 100) == 0
-    assert wq.wq_layout_version() == 0
+    assert wq.wq_layout_version() == wq.WQ_LAYOUT_B200_V1 == 1
 
 
 @pytest.mark.parametrize("N,K", [(1, 256), (5, 768), (64, 4096)])

@@ -6,6 +6,8 @@ The kernels live in libwq.so (C ABI in include/wq.h); this package is a thin
 ctypes binding with the same entry-point names.
 """
 from .api import (  # noqa: F401
+    WQ_ERR_TIMEOUT,
+    WQ_ERR_UNSUPPORTED,
     WQ_LAYOUT_B200_V1,
     WQ_LAYOUT_CANONICAL,
     WQError,
@@ -27,4 +29,5 @@ from .api import (  # noqa: F401
     wq_layout_version,
     wq_q4k_bytes,
     wq_q4k_dsc_bytes,
+    wq_test_expire_wait,
 )

@@ -48,6 +48,7 @@ SIGNATURES = {
     "wq_layout_version": (_i, []),
     "wq_build_info": (_cp, []),
     "wq_device_status": (_i, []),
+    "wq_test_expire_wait": (_i, [ctypes.c_ulonglong, _vp]),
 }
 
 _lib = None

@@ -11,7 +11,8 @@ import ctypes
 
 import numpy as np
 
-from ._lib import WQ_LAYOUT_B200_V1, WQ_LAYOUT_CANONICAL, WQError, _check, last_error, last_kernel, lib  # noqa: F401
+from ._lib import (WQ_ERR_TIMEOUT, WQ_ERR_UNSUPPORTED, WQ_LAYOUT_B200_V1, WQ_LAYOUT_CANONICAL, WQError,  # noqa: F401
+                   _check, last_error, last_kernel, lib)
 
 
 def _ptr(t):
@@ -105,3 +106,7 @@ def wq_layout_version() -> int:
 
 def wq_device_status() -> None:
     _check(lib().wq_device_status(), "wq_device_status")
+
+
+def wq_test_expire_wait(limit_ns: int, stream=None) -> None:
+    _check(lib().wq_test_expire_wait(int(limit_ns), _stream(stream)), "wq_test_expire_wait")

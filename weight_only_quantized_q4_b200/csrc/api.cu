@@ -839,7 +839,9 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   if (const char* s_env = std::getenv("WQ_TC5_S")) {  // tests and tuning
     const int sf = std::atoi(s_env);
     if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
-      if (nst % (p.spr * sf)) return fail(WQ_ERR_ARG, "WQ_TC5_S does not divide K into whole raw slots");
+      // the same rule as the automatic choice: every CTA gets an even number of
+      // raw slots, so its even / odd accumulator tiles see the same stage count
+      if (nst % (2 * p.spr * sf)) return fail(WQ_ERR_ARG, "WQ_TC5_S does not split K into an even number of raw slots per CTA");
       S = sf;
     }
   }
@@ -985,6 +987,9 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
       if (rc) return rc;
       label = cc_label(fmt_name, mc, plan.KS, M > 8 ? ".chunked" : "");
     } else {
+      if (force && std::strcmp(force, "simple") != 0)
+        return fail(WQ_ERR_UNSUPPORTED, std::string("WQ_FORCE_KERNEL=") + force +
+                                            ": that kernel family cannot run this call (format, layout, shape or alignment)");
       SimpleParams sp{};
       sp.x = xc;
       sp.w = w;
@@ -1197,8 +1202,24 @@ int wq_build_q4k_dsc_device(const void* w_q4k, void* out, int N, int K, void* st
 
 const char* wq_last_error(void) { return t_last_error.c_str(); }
 const char* wq_last_kernel(void) { return t_last_kernel.c_str(); }
-int wq_layout_version(void) { return WQ_LAYOUT_CANONICAL; }
-const char* wq_build_info(void) { return "libwq sm_100a; CUDA-core streaming GEMV (M<=8), fallback GEMV, exports"; }
+int wq_layout_version(void) { return WQ_LAYOUT_B200_V1; }
+const char* wq_build_info(void) {
+  return "libwq sm_100a: decode GEMV M<=8 (B200_V1 int4 bulk-copy ring + warp MMA; warp-MMA GEMV for canonical "
+         "int4, q4_K raw / W_dsc plane and bf16; CUDA-core and scalar GEMVs), tcgen05 dequant-then-MMA for M>=9 "
+         "(int4 canonical, q4_K), device dequant exports, B200_V1 repack, W_dsc plane builders";
+}
+
+int wq_test_expire_wait(unsigned long long limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull)
+    return fail(WQ_ERR_ARG, "wq_test_expire_wait: limit_ns must be in [1e3, 1e9]");
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  expire_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  if ((rc = launch_check("expire_wait launch"))) return rc;
+  set_last_kernel("test.expire_wait");
+  return WQ_OK;
+}
 
 int wq_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();

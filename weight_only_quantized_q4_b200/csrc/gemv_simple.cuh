@@ -342,4 +342,19 @@ __global__ void build_q4k_dsc_kernel(const uint8_t* w, float2* plane, int N, int
   }
 }
 
+// Test hook for the failure path of bounded waits: one thread waits on an
+// mbarrier that nothing arrives at (no copy in flight), gives up after
+// limit_ns and records the timeout in the device error word, as a real wait
+// that gives up does; the kernel then returns normally.
+__global__ void expire_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded_ns(&bar, 0u, limit_ns);
+  __syncthreads();
+}
+
 }  // namespace wq

@@ -81,18 +81,22 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs.
+// Wait for phase `parity` of `bar` to complete, for at most `limit_ns`.
 // Returns false (and records kDevErrTimeout) when the limit is reached.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded_ns(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       atomicOr(&g_device_error, kDevErrTimeout);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_bounded_ns(bar, parity, kWaitLimitNs);
 }
 
 // 1-D bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
