@@ -12,7 +12,10 @@ another (the canonical-layout, q4_K, bf16 and batched workloads).
 Metric: achieved HBM GB/s (weight + scale + zero-point bytes ÷ device time)
 and µs per call.  Timing: CUDA graphs of back-to-back calls, each call on the
 next of R weight copies whose total exceeds 3× the L2, CUDA events on the
-launching stream, barrier + synchronize on both sides, max over ranks.
+launching stream, barrier + synchronize on both sides, max over ranks; five
+repetitions of at least 50 ms and 200 calls each (more when --steps asks for
+more), reported as the median with its spread.  Decode workloads also get the
+same measurement at M = 1, 2, 4 and 8 on their shape (``per_m``).
 
 ``--impl reference`` times the CPU oracle (test infrastructure) on the host
 cores, on a bounded sample of the same workload.
@@ -212,21 +215,32 @@ class DeviceWorkload:
             self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
 
-    def call(self, i, x=None, y=None, stream=None):
+    def batch_buffers(self, M):
+        """Activations and output of batch M for the same weights (seeded like the workload's x)."""
+        torch, w = self.torch, self.w
+        dev = self.x.device
+        if w["fmt"] == "bf16":
+            x = torch.from_numpy(synth.activations_bf16_bits(M, self.K, workload=w["workload"]).view(np.int16))
+            return x.to(dev).view(torch.bfloat16), torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
+        x = torch.from_numpy(synth.activations_f16(M, self.K, workload=w["workload"])).to(dev)
+        return x, torch.empty((M, self.N), dtype=torch.float16, device=dev)
+
+    def call(self, i, x=None, y=None, stream=None, M=None):
         c = self.copies[i % self.R]
         x = self.x if x is None else x
         y = self.y if y is None else y
+        M = self.M if M is None else M
         w, wq = self.w, self.wq
         if w["fmt"] == "int4":
-            wq.gemv_int4_blockwise(x, c[0], c[1], c[2], y, self.M, self.N, self.K, w["bs"],
+            wq.gemv_int4_blockwise(x, c[0], c[1], c[2], y, M, self.N, self.K, w["bs"],
                                    layout=w.get("layout", 0), stream=stream)
         elif w["fmt"] == "q4k":
             if w["dsc"]:
-                wq.gemv_q4k_dsc(x, c[0], c[1], y, self.M, self.N, self.K, stream=stream)
+                wq.gemv_q4k_dsc(x, c[0], c[1], y, M, self.N, self.K, stream=stream)
             else:
-                wq.gemv_q4k(x, c[0], y, self.M, self.N, self.K, stream=stream)
+                wq.gemv_q4k(x, c[0], y, M, self.N, self.K, stream=stream)
         else:
-            wq.gemv_bf16(x, c[0], y, self.M, self.N, self.K, stream=stream)
+            wq.gemv_bf16(x, c[0], y, M, self.N, self.K, stream=stream)
 
 
 def _peaks():
@@ -278,6 +292,54 @@ def job_gbs(world: int, bytes_per_call: int, calls: int, ms: float) -> float:
     return world * bytes_per_call * calls / (ms * 1e-3) / 1e9
 
 
+def _timed_reps(torch, replay, calls_per_replay, stream, steps_req, reps, min_ms, warmup, barrier):
+    """Replay a captured graph of back-to-back calls: `warmup` untimed replays,
+    then `reps` timed repetitions, each of enough replays for at least
+    `min_ms` milliseconds and 200 calls (and, over all repetitions, at least
+    `steps_req` calls), bracketed by a barrier + synchronize on both sides and
+    CUDA events on the launching stream.  Returns (replays per repetition,
+    [ms per repetition])."""
+    for _ in range(max(warmup, 3)):
+        replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_one = max(e0.elapsed_time(e1), 1e-3)
+    per_rep = max(1, -(-200 // calls_per_replay), int(np.ceil(min_ms / t_one)),
+                  -(-steps_req // (calls_per_replay * reps)))
+    times = []
+    for _ in range(reps):
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(per_rep):
+            replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        times.append(e0.elapsed_time(e1))
+    return per_rep, times
+
+
+def _rep_summary(times_ms, calls_per_rep):
+    us = sorted(t * 1e3 / calls_per_rep for t in times_ms)
+    med = float(statistics.median(us))
+    return {"us_per_call_median": round(med, 3), "us_per_call_min": round(us[0], 3),
+            "us_per_call_max": round(us[-1], 3), "spread_pct": round(100.0 * (us[-1] - us[0]) / med, 2),
+            "reps": len(us), "calls_per_rep": calls_per_rep}
+
+
+def _capture(torch, d, stream, G, x=None, y=None):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(G):
+            d.call(i, x=x, y=y, stream=torch.cuda.current_stream())
+    return g
+
+
 def run_ours(args, w, wname, rank, world, dist):
     import torch
 
@@ -289,17 +351,19 @@ def run_ours(args, w, wname, rank, world, dist):
     d = DeviceWorkload(w, host, torch, wq, l2, copies=args.copies)
     stream = torch.cuda.Stream()
 
-    # configure every kernel once outside capture, then capture a graph of G calls
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # configure every kernel once outside capture, then capture a graph of G
+    # back-to-back calls (a whole number of passes over the R weight copies)
     with torch.cuda.stream(stream):
         d.call(0, stream=stream)
     torch.cuda.synchronize()
     label = wq.last_kernel()
-    G = max(d.R, min(args.graph_calls, args.steps))
+    G = max(d.R, args.graph_calls)
     G = -(-G // d.R) * d.R
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for i in range(G):
-            d.call(i, stream=torch.cuda.current_stream())
+    g = _capture(torch, d, stream, G)
     # per-launch durations: events between consecutive calls in a second graph
     n_ev = min(G, 256)
     evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev + 1)]
@@ -311,35 +375,40 @@ def run_ours(args, w, wname, rank, world, dist):
             d.call(i, stream=cs)
         evs[n_ev].record(cs)
 
-    reps = max(1, -(-args.steps // G))
-    steps = reps * G
-    for _ in range(max(args.warmup, 3)):
-        g.replay()
-    torch.cuda.synchronize()
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    peak, peak_kind = _peaks()
+    reps = max(4, args.reps)
+    per_m = []
     with ClockSampler(torch.cuda.current_device()) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        e0.record(stream)
         with torch.cuda.stream(stream):
-            for _ in range(reps):
-                g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        # per-launch timing pass (same clocks window)
-        with torch.cuda.stream(stream):
+            per_rep, times = _timed_reps(torch, g.replay, G, stream, args.steps, reps, args.min_ms, args.warmup,
+                                         barrier)
+            # per-launch timing pass (same clocks window)
             for _ in range(3):
                 g_ev.replay()
-        torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+            torch.cuda.synchronize()
+            # the same measurement for M = 1, 2, 4, 8 on this shape (decode GEMV workloads)
+            if w["M"] <= 8 and not args.no_per_m:
+                for Mb in (1, 2, 4, 8):
+                    xb, yb = d.batch_buffers(Mb)
+                    d.call(0, x=xb, y=yb, M=Mb, stream=stream)
+                    torch.cuda.synchronize()
+                    gb = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gb, stream=stream):
+                        for i in range(G):
+                            d.call(i, x=xb, y=yb, M=Mb, stream=torch.cuda.current_stream())
+                    pr, tb = _timed_reps(torch, gb.replay, G, stream, 0, reps, args.min_ms, 3, barrier)
+                    tb = max_over_ranks(tb, dist, "cuda")
+                    sm_ = _rep_summary(tb, pr * G)
+                    gbs = d.bytes / (sm_["us_per_call_median"] * 1e-6) / 1e9
+                    per_m.append({"M": Mb, "us_per_call": sm_["us_per_call_median"], "gbs": round(gbs, 1),
+                                  "frac": round(gbs / peak, 4), "spread_pct": sm_["spread_pct"],
+                                  "calls_timed": pr * G * reps, "kernel": wq.last_kernel()})
+                    del gb
+    times = max_over_ranks(times, dist, "cuda")
     per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(n_ev)]
     avg_launch_ms = float(np.mean(per_launch))
+    calls_per_rep = per_rep * G
+    rs = _rep_summary(times, calls_per_rep)
 
     # e2e: every step copies its x in from pinned host memory, runs the GEMV
     # through the API and copies its y out to pinned host memory.  Steps are
@@ -385,37 +454,22 @@ def run_ours(args, w, wname, rank, world, dist):
                 ev_y[i].record(d2h_s)
         cs.wait_event(ev_x[Ge - 1])
         cs.wait_event(ev_y[Ge - 1])
-    for _ in range(2):
-        ge.replay()
-    torch.cuda.synchronize()
-    reps_e = max(1, -(-min(args.steps, 20000) // Ge))
-    barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
     with torch.cuda.stream(stream):
-        for _ in range(reps_e):
-            ge.replay()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e = t0.elapsed_time(t1)
-    steps_e2e = reps_e * Ge
+        pe, te = _timed_reps(torch, ge.replay, Ge, stream, 0, reps, args.min_ms, 2, barrier)
     # the last step's result (same x, an identical weight copy) must have reached
     # host memory bit for bit: the kernels are deterministic, so a difference
     # would mean a missing dependency in the pipelined copies
     if not torch.equal(yh[(Ge - 1) % NB].view(torch.int16), d.y.cpu().view(torch.int16)):
         raise RuntimeError("e2e: host copy of y differs from the device result")
-
-    ms, ms_e2e = max_over_ranks([ms, ms_e2e], dist, "cuda")
+    te = max_over_ranks(te, dist, "cuda")
+    es = _rep_summary(te, pe * Ge)
 
     bytes_call = d.bytes
-    ms_step = ms / steps
-    value = job_gbs(world, bytes_call, steps, ms)
-    e2e_value = job_gbs(world, bytes_call, steps_e2e, ms_e2e)
-    peak, peak_kind = _peaks()
-    # one launch of the kernel per step: its average duration over the timed region
+    ms_step = rs["us_per_call_median"] * 1e-3
+    steps = calls_per_rep * reps
+    value = job_gbs(world, bytes_call, 1, ms_step)
+    e2e_value = job_gbs(world, bytes_call, 1, es["us_per_call_median"] * 1e-3)
+    # one launch of the kernel per step: its median duration over the timed region
     achieved = bytes_call / (ms_step * 1e-3) / 1e9
     out = {
         "metric": METRIC,
@@ -423,9 +477,10 @@ def run_ours(args, w, wname, rank, world, dist):
         "unit": "GB/s",
         "n_gpus": world,
         "steps": steps,
+        "steps_requested": args.steps,
         "warmup": max(args.warmup, 3),
         "ms_per_step": ms_step,
-        "us_per_call": round(ms_step * 1e3, 3),
+        "us_per_call": rs["us_per_call_median"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -436,25 +491,30 @@ def run_ours(args, w, wname, rank, world, dist):
                    "weight_bytes_per_call": bytes_call, "weight_copies_rotated": d.R,
                    "l2": f"inputs larger than L2: {d.R} rotating weight copies, {d.R * bytes_call / 1e6:.0f} MB "
                          f">= 3x L2 ({l2 / 1e6:.0f} MB)",
-                   "timing": f"CUDA graph of {G} back-to-back calls replayed {reps}x, CUDA events on the stream",
+                   "timing": f"{reps} repetitions of {calls_per_rep} back-to-back calls (CUDA graph of {G} calls "
+                             f"replayed {per_rep}x, >= {args.min_ms:g} ms and >= 200 calls per repetition), CUDA "
+                             f"events on the launching stream; value and us_per_call from the median repetition",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "kernel": label},
+        "timing": rs,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": int(d.x.numel() * d.x.element_size()),
                 "d2h_bytes_per_step": int(d.y.numel() * d.y.element_size()),
-                "us_per_call": round(ms_e2e / steps_e2e * 1e3, 3),
+                "us_per_call": es["us_per_call_median"], "spread_pct": es["spread_pct"],
                 "how": "per step: pinned x -> device, GEMV through the C ABI, y -> pinned host; steps pipelined over "
                        "two copy streams with 3 device buffers per tensor (copies of neighbouring steps overlap the "
-                       "GEMV); graph-captured"},
+                       "GEMV); graph-captured; median of the repetitions"},
         "gpu_launches": steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": _traffic(wname),
-                     "peak_kind": f"{peak_kind} copy bandwidth", "avg_launch_us": round(ms_step * 1e3, 3),
+                     "peak_kind": f"{peak_kind} copy bandwidth", "avg_launch_us": rs["us_per_call_median"],
                      "isolated_launch_us": round(avg_launch_ms * 1e3, 3),
-                     "how": "achieved = algorithmic bytes per launch / average launch duration over the timed "
-                            "region (one launch per step, CUDA events on the launching stream); "
+                     "how": "achieved = algorithmic bytes per launch / median launch duration over the timed "
+                            "repetitions (one launch per step, CUDA events on the launching stream); "
                             "isolated_launch_us = events around single launches (no overlap with the next call)"},
         "clocks": clk.summary(),
     }
+    if per_m:
+        out["per_m"] = per_m
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, host, budget_s=args.cpu_budget)
     return out
@@ -536,13 +596,17 @@ def run_reference(args, w, wname):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--sweep", action="store_true", help="one JSON line per workload of the sweep list")
     ap.add_argument("--sweep-batched", action="store_true", help="one JSON line per batched (M >= 16) workload")
-    ap.add_argument("--graph-calls", type=int, default=1000)
+    ap.add_argument("--graph-calls", type=int, default=200, help="calls captured in one graph (rounded up to "
+                    "whole passes over the weight copies)")
+    ap.add_argument("--reps", type=int, default=5, help="timed repetitions (at least 4)")
+    ap.add_argument("--min-ms", type=float, default=50.0, help="minimum duration of one timed repetition")
+    ap.add_argument("--no-per-m", action="store_true", help="skip the M = 1, 2, 4, 8 record")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=0,

@@ -99,6 +99,23 @@ extern "C" {
 #define WQ_INT4_V1_TILE_BYTES(bs) \
   ((1024 + ((bs) >= 128 ? 1 : 128 / (bs)) * 40 + 15) / 16 * 16)
 #define WQ_LAYOUT_B200_V1 1
+/* B200_V1 (q4_K): the same band idea for q4_K super-blocks.  Rows are grouped
+ * in bands of 16 (the last band padded with zero codes and zero d, dmin and
+ * scales); a band is K/256 consecutive tiles of WQ_Q4K_V1_TILE_BYTES bytes,
+ * tile s holding super-block s of the band's 16 rows (exactly the 16 × 144
+ * canonical bytes, reordered; minfer doc 62 "r59 — q4_K W_dsc plane", §3.2
+ * for the canonical fields):
+ *   bytes [0, 2048): codes in warp-MMA fragment order: offset h·512 + lane·16
+ *     + 4·(2·(gi & 1) + r8) holds the 32-bit code word of band row
+ *     (lane / 4) + 8·r8 for k = 256s + 32·gi + 8·(lane % 4) + e, e = 0..7
+ *     (gi = 2h + (0|1) = the 32-element chunk, h = 0..3), code e in nibble
+ *     position (e >> 1) | ((e & 1) << 2);
+ *   bytes [2048, 2112): the rows' (d, dmin) fp16 pairs, 4 bytes per row;
+ *   bytes [2112, 2304): 24-bit little-endian entries, entry (pair p, row r) at
+ *     2112 + 3·(16p + r) = sc_{2p} | sc_{2p+1} << 6 | m_{2p} << 12 |
+ *     m_{2p+1} << 18 (the 6-bit scales and mins of chunks 2p, 2p+1, §2.1).
+ * Built on the device by wq_repack_q4k. */
+#define WQ_Q4K_V1_TILE_BYTES 2304
 
 /* ---------------------------------------------------------------------------
  * GEMV / GEMM entry points.  All device pointers; y is written, never read.
@@ -140,7 +157,9 @@ int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const v
                            float* w_out, int N, int K, int block_size, int layout, void* stream);
 /* (layout selects how w_packed is read: canonical or B200_V1.) */
 
-/* w_dsc NULL: coefficients decoded from the packed fields; else taken from the plane. */
+/* w_dsc NULL: coefficients decoded from the packed fields; else taken from the
+ * plane.  layout WQ_LAYOUT_B200_V1 reads a wq_repack_q4k stream (w_dsc must
+ * then be NULL). */
 int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K, int layout,
                 void* stream);
 
@@ -169,6 +188,17 @@ size_t wq_int4_packed_bytes(int N, int K, int block_size, int layout);
 /* Bytes of a q4_K tensor and of its W_dsc plane; 0 for invalid arguments. */
 size_t wq_q4k_bytes(int N, int K);
 size_t wq_q4k_dsc_bytes(int N, int K);
+
+/* Bytes of the B200_V1 q4_K stream of an N × K tensor (layout must be
+ * WQ_LAYOUT_B200_V1), 0 if invalid. */
+size_t wq_q4k_packed_bytes(int N, int K, int layout);
+
+/* Rewrite canonical q4_K super-blocks (N·(K/256)·144 bytes, device) into the
+ * B200_V1 q4_K stream at w_out (wq_q4k_packed_bytes(N, K, to_layout) bytes,
+ * device, must not overlap the source).  Errors: WQ_ERR_ARG (K % 256 != 0),
+ * WQ_ERR_LAYOUT (to_layout is not WQ_LAYOUT_B200_V1), WQ_ERR_ALIGN,
+ * WQ_ERR_CUDA. */
+int wq_repack_q4k(const void* w_q4k, void* w_out, int N, int K, int to_layout, void* stream);
 
 /* Build the W_dsc plane on the host (minfer doc 62, §2.2-§2.3): one IEEE fp32
  * multiply per coefficient and an exact negation, no contraction.

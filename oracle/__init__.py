@@ -36,5 +36,9 @@ from .q4 import (  # noqa: F401
     q4k_fields,
     q4k_plane,
     q4k_scales_mins,
+    SILU_MAX_SLOPE,
+    silu,
+    swiglu_gemv,
+    swiglu_tolerance,
     violations,
 )

@@ -222,3 +222,42 @@ def violations(y, y_ref, B, rel: float = 2e-3, abs_: float = 1e-3) -> np.ndarray
 def accept(y, y_ref, B, rel: float = 2e-3, abs_: float = 1e-3) -> bool:
     """True iff every element satisfies |y − y_ref| ≤ rel·B + abs_ (NaN fails)."""
     return not bool(np.any(violations(y, y_ref, B, rel, abs_)))
+
+
+# --------------------------------------------------------------------------
+# fused gate / up projection with the SiLU·mul epilogue (the "swiglu" launch
+# that minfer doc 62 "r59 — q4_K W_dsc plane", §3.3 riders, prewarms; the page
+# names the fused launch but not its formula: the reading taken is the usual
+# SwiGLU feed-forward half, silu(x·Wgᵀ) ⊙ (x·Wuᵀ), with silu(a) = a·σ(a))
+# --------------------------------------------------------------------------
+
+SILU_MAX_SLOPE = 1.0999  # an upper bound of |d silu / da| over the reals (1.09984 near a = 2.4)
+
+
+def silu(a) -> np.ndarray:
+    """silu(a) = a·σ(a) = a / (1 + e^(−a)) in float64."""
+    a = np.asarray(a, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return a / (1.0 + np.exp(-a))
+
+
+def swiglu_gemv(Wg, Wu, x) -> np.ndarray:
+    """y[m, n] = silu(Σ_k Wg[n,k]·x[m,k]) · Σ_k Wu[n,k]·x[m,k] in float64."""
+    return silu(gemv(Wg, x)) * gemv(Wu, x)
+
+
+def swiglu_tolerance(a, b, Ba, Bb, rel: float = 2e-3, abs_: float = 1e-3) -> np.ndarray:
+    """Acceptance bound for y = silu(a)·b when each projection is computed to
+    the GEMV bound |Δa| ≤ ea = rel·Ba + abs_, |Δb| ≤ eb = rel·Bb + abs_ (Ba,
+    Bb the Σ|w·x| of each), and y is rounded once to fp16 at the end:
+
+      |Δy| ≤ S·ea·(|b| + eb) + |silu(a)|·eb + 2^-10·(|silu(a)·b| + S·ea·(|b| + eb) + |silu(a)|·eb) + abs_,
+
+    S the largest slope of silu (mean value theorem on silu(a + Δa)), 2^-10 a
+    generous bound on the relative rounding of the fp16 result and of the
+    fp32 evaluation of silu."""
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    ea = rel * np.asarray(Ba, dtype=np.float64) + abs_
+    eb = rel * np.asarray(Bb, dtype=np.float64) + abs_
+    prop = SILU_MAX_SLOPE * ea * (np.abs(b) + eb) + np.abs(silu(a)) * eb
+    return prop + 2.0 ** -10 * (np.abs(silu(a) * b) + prop) + abs_

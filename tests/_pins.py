@@ -339,6 +339,63 @@ def pin_exact_in_f32(o):
     assert not o.exact_in_f32(np.array([1.0 + 2.0 ** -30]))
 
 
+# ---------------------------------------------------------------- SwiGLU pins
+
+def pin_silu_closed_forms(o):
+    """silu(a) = a·σ(a) where the logistic function has closed forms:
+    σ(0) = 1/2, σ(ln 3) = 3/4, σ(−ln 3) = 1/4, σ(1) = e/(e + 1); and its limits."""
+    ln3 = math.log(3.0)
+    assert float(o.silu(0.0)) == 0.0
+    assert abs(float(o.silu(ln3)) - 0.75 * ln3) <= 1e-15
+    assert abs(float(o.silu(-ln3)) + 0.25 * ln3) <= 1e-15
+    assert abs(float(o.silu(1.0)) - math.e / (math.e + 1.0)) <= 1e-15
+    assert float(o.silu(40.0)) == 40.0
+    assert abs(float(o.silu(-40.0))) <= 1e-15 and float(o.silu(-1e4)) == 0.0
+
+
+def pin_silu_reflection_and_slope(o):
+    """silu(a) − silu(−a) = a (σ(a) + σ(−a) = 1), and the slope bound the
+    tolerance uses is attained: the steepest finite-difference slope on a
+    fine grid lies just below it."""
+    a = np.random.default_rng(71).uniform(-30.0, 30.0, 2000)
+    assert np.allclose(o.silu(a) - o.silu(-a), a, rtol=1e-12, atol=1e-12)
+    g = np.linspace(-12.0, 12.0, 240001)
+    h = 1e-6
+    slope = np.abs((o.silu(g + h) - o.silu(g - h)) / (2 * h))
+    assert slope.max() <= o.SILU_MAX_SLOPE and slope.max() >= o.SILU_MAX_SLOPE - 1e-3
+
+
+def pin_swiglu_hand(o):
+    """Hand example: gate row (0.5, 0.5) and x = (1, 1) give a = 1, up row
+    (2, 0) gives b = 2, so y = 2·silu(1) = 2e/(e + 1); a gate row of zeros
+    gives y = 0 whatever b is; a = −30 gives |y| ≤ 30·e^-30·|b|."""
+    Wg = np.array([[0.5, 0.5], [0.0, 0.0]])
+    Wu = np.array([[2.0, 0.0], [1.0, 3.0]])
+    y = o.swiglu_gemv(Wg, Wu, np.array([[1.0, 1.0]]))
+    assert abs(y[0, 0] - 2.0 * math.e / (math.e + 1.0)) <= 1e-15 and y[0, 1] == 0.0
+    y2 = o.swiglu_gemv(Wg, Wu, np.array([[-60.0, 0.0]]))
+    assert abs(y2[0, 0]) <= 30.0 * math.exp(-30.0) * 120.0 * 1.0001 and y2[0, 1] == 0.0
+
+
+def pin_swiglu_tolerance_covers_worst_case(o):
+    """The acceptance bound of the fused projection covers every combination
+    of a and b each off by its full GEMV bound, plus fp16 rounding of y."""
+    rng = np.random.default_rng(72)
+    a = rng.uniform(-8, 8, 4000)
+    b = rng.uniform(-8, 8, 4000) * rng.choice([1.0, 1e-3], 4000)
+    Ba = np.abs(a) * rng.uniform(1, 50, 4000)
+    Bb = np.abs(b) * rng.uniform(1, 50, 4000)
+    tol = o.swiglu_tolerance(a, b, Ba, Bb)
+    ea, eb = 2e-3 * Ba + 1e-3, 2e-3 * Bb + 1e-3
+    y = a / (1 + np.exp(-a)) * b  # the unperturbed value, for the property only
+    for sa in (-1, 1):
+        for sb in (-1, 1):
+            a2, b2 = a + sa * ea, b + sb * eb
+            yp = a2 / (1 + np.exp(-a2)) * b2
+            for r in (1 - 2.0 ** -11, 1 + 2.0 ** -11):
+                assert np.all(np.abs(yp * r - y) <= tol)
+
+
 ALL_PINS = [
     pin_scale_min_golden,
     pin_scale_min_bijection,
@@ -356,4 +413,8 @@ ALL_PINS = [
     pin_gemv_fsum,
     pin_accept_threshold,
     pin_exact_in_f32,
+    pin_silu_closed_forms,
+    pin_silu_reflection_and_slope,
+    pin_swiglu_hand,
+    pin_swiglu_tolerance_covers_worst_case,
 ]

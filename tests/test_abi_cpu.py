@@ -72,6 +72,10 @@ def test_q4k_and_bf16_argument_errors():
     assert L.gemv_bf16(A16, A16, A16, 1, 0, 7, None) == _lib.WQ_ERR_ARG
     assert L.dequant_q4k(A16, None, A16, 4, 100, 0, None) == _lib.WQ_ERR_ARG
     assert L.wq_build_q4k_dsc(None, 4, 256, None) == _lib.WQ_ERR_ARG
+    assert L.wq_repack_q4k(A16, A16, 16, 300, 1, None) == _lib.WQ_ERR_ARG
+    assert L.wq_repack_q4k(A16, A16, 16, 256, 0, None) == _lib.WQ_ERR_LAYOUT
+    assert L.wq_repack_q4k(A16 + 4, A16, 16, 256, 1, None) == _lib.WQ_ERR_ALIGN
+    assert L.dequant_q4k(A16, A16, A16, 4, 256, 1, None) == _lib.WQ_ERR_LAYOUT
     assert L.wq_test_expire_wait(10, None) == _lib.WQ_ERR_ARG
     assert L.wq_test_expire_wait(2 * 10**9, None) == _lib.WQ_ERR_ARG
 
@@ -103,6 +107,9 @@ def test_size_queries():
     assert wq.wq_q4k_bytes(4096, 4096) == 4096 * 16 * 144
     assert wq.wq_q4k_dsc_bytes(4096, 11008) == 4096 * 11008 // 4
     assert wq.wq_q4k_dsc_bytes(4, 100) == 0
+    assert wq.wq_q4k_packed_bytes(21, 512) == 2 * 2 * 2304
+    assert wq.wq_q4k_packed_bytes(21, 512, 0) == 0
+    assert wq.wq_q4k_packed_bytes(4096, 11008) == 256 * 43 * 2304 == wq.wq_q4k_bytes(4096, 11008)
     assert wq.wq_layout_version() == wq.WQ_LAYOUT_B200_V1 == 1
 
 

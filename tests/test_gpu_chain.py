@@ -96,3 +96,55 @@ def test_chained_calls_match_isolated_calls(first, second, graph):
     wq.wq_device_status()
     for i, (y2, w) in enumerate(zip(outs, want)):
         assert np.array_equal(y2.cpu().view(torch.int16).numpy(), w.view(torch.int16).numpy()), (first, second, i)
+
+
+@gpu
+@pytest.mark.parametrize("case", ["int4_v1_repack", "int4_canonical_torch_kernel", "q4k_torch_kernel"])
+def test_weights_written_by_the_kernel_right_before(case):
+    """The kernel right before a GEMV on the same stream writes that GEMV's
+    weights (the load-time repack, or a torch elementwise kernel), with no
+    synchronization in between: the GEMV must read the new weights.  Weights
+    alternate between two seeded sets, so stale data would show."""
+    import oracle
+
+    torch.cuda.set_device(DEV)
+    N, K = 2048, 4096
+    s = torch.cuda.Stream()
+    x = synth.activations_f16(1, K, workload=61)
+    dx = torch.from_numpy(x).to(DEV)
+    sets, refs = [], []
+    for wl in (62, 63):
+        if case.startswith("int4"):
+            t = synth.int4_weights(N, K, 128, scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=wl)
+            sets.append([torch.from_numpy(t[k]).to(DEV) for k in ("w_packed", "scales", "zeros")])
+            W = oracle.dequant_int4(t["w_packed"], t["scales"], t["zeros"], N, K, 128)
+        else:
+            raw = synth.q4k_weights(N, K, workload=wl)
+            sets.append([torch.from_numpy(raw).to(DEV)])
+            W = oracle.dequant_q4k(raw, N, K)
+        refs.append((oracle.gemv(W, x), oracle.bound(W, x)))
+    if case == "int4_v1_repack":
+        live = torch.empty((wq.wq_int4_packed_bytes(N, K, 128, wq.WQ_LAYOUT_B200_V1),), dtype=torch.uint8, device=DEV)
+    else:
+        live = [torch.empty_like(t) for t in sets[0]]
+    torch.cuda.synchronize()
+    outs = [torch.empty((1, N), dtype=torch.float16, device=DEV) for _ in range(8)]
+    with torch.cuda.stream(s):
+        for i, y in enumerate(outs):
+            src = sets[i % 2]
+            if case == "int4_v1_repack":
+                wq.wq_repack_int4(src[0], src[1], src[2], live, N, K, 128, wq.WQ_LAYOUT_B200_V1, stream=s)
+                wq.gemv_int4_blockwise(dx, live, None, None, y, 1, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1, stream=s)
+            elif case == "int4_canonical_torch_kernel":
+                for dst, t in zip(live, src):
+                    torch.bitwise_or(t, 0, out=dst)  # an elementwise kernel writes the weights
+                wq.gemv_int4_blockwise(dx, live[0], live[1], live[2], y, 1, N, K, 128, stream=s)
+            else:
+                torch.bitwise_or(src[0], 0, out=live[0])
+                wq.gemv_q4k(dx, live[0], y, 1, N, K, stream=s)
+    torch.cuda.synchronize()
+    wq.wq_device_status()
+    for i, y in enumerate(outs):
+        y_ref, B = refs[i % 2]
+        bad = oracle.violations(y.cpu().numpy().astype(np.float64), y_ref, B)
+        assert not bad.any(), (case, i, int(bad.sum()))

@@ -135,6 +135,74 @@ def test_repack_v1_layout_matches_header(bs):
     assert np.all(q[N:] == 0) and np.all(sc[N:] == 0) and np.all(zp[N:] == 8)
 
 
+def decode_q4k_v1(buf, N, K):
+    """Read a B200_V1 q4_K stream back into (q, d, dmin, sc, m) per the layout
+    the header documents (plain numpy, independent of the device code)."""
+    nb, tpb = (N + 15) // 16, K // 256
+    q = np.zeros((nb * 16, K), dtype=np.int64)
+    d = np.zeros((nb * 16, tpb), dtype=np.float64)
+    dm = np.zeros((nb * 16, tpb), dtype=np.float64)
+    sc = np.zeros((nb * 16, tpb, 8), dtype=np.int64)
+    mn = np.zeros((nb * 16, tpb, 8), dtype=np.int64)
+    for band in range(nb):
+        for s_ in range(tpb):
+            tile = buf[(band * tpb + s_) * 2304:(band * tpb + s_ + 1) * 2304]
+            words = tile[:2048].view(np.uint32)
+            for h in range(4):
+                for lane in range(32):
+                    g, t = lane // 4, lane % 4
+                    for j in range(4):
+                        gi, r8 = 2 * h + j // 2, j % 2
+                        word = int(words[(h * 512 + lane * 16 + 4 * j) // 4])
+                        row = band * 16 + g + 8 * r8
+                        for e in range(8):
+                            pos = (e >> 1) | ((e & 1) << 2)
+                            q[row, 256 * s_ + 32 * gi + 8 * t + e] = (word >> (4 * pos)) & 15
+            dd = tile[2048:2112].view(np.float16).astype(np.float64).reshape(16, 2)
+            for r in range(16):
+                row = band * 16 + r
+                d[row, s_], dm[row, s_] = dd[r, 0], dd[r, 1]
+                for p in range(4):
+                    o = 2112 + 3 * (16 * p + r)
+                    ent = int(tile[o]) | (int(tile[o + 1]) << 8) | (int(tile[o + 2]) << 16)
+                    sc[row, s_, 2 * p], sc[row, s_, 2 * p + 1] = ent & 63, (ent >> 6) & 63
+                    mn[row, s_, 2 * p], mn[row, s_, 2 * p + 1] = (ent >> 12) & 63, (ent >> 18) & 63
+    return q, d, dm, sc, mn
+
+
+@gpu
+@pytest.mark.parametrize("N,K", [(21, 256), (16, 512), (5, 768)])
+def test_repack_q4k_v1_layout_matches_header(N, K):
+    """The q4_K band stream, decoded by a plain reading of the documented
+    layout, gives the oracle's weights; pad rows are all zero."""
+    raw = synth.q4k_weights(N, K, workload=17)
+    gp = Guarded((wq.wq_q4k_packed_bytes(N, K),), torch.uint8)
+    wq.wq_repack_q4k(dev(raw), gp.t, N, K)
+    torch.cuda.synchronize()
+    gp.check("q4_K B200_V1 repack output")
+    q, d, dm, sc, mn = decode_q4k_v1(gp.t.cpu().numpy(), N, K)
+    chunk = (np.arange(K) % 256) // 32
+    sbk = np.arange(K) // 256
+    W = d[:, sbk] * sc[:, sbk, chunk] * q - dm[:, sbk] * mn[:, sbk, chunk]
+    assert np.array_equal(W[:N], oracle.dequant_q4k(raw, N, K))
+    assert np.all(q[N:] == 0) and np.all(d[N:] == 0) and np.all(sc[N:] == 0) and np.all(mn[N:] == 0)
+
+
+@gpu
+@pytest.mark.parametrize("N,K", [(3, 256), (17, 768), (40, 4096)])
+def test_dequant_q4k_v1_layout_bit_exact(N, K):
+    raw = synth.q4k_weights(N, K, workload=18)
+    packed = torch.empty((wq.wq_q4k_packed_bytes(N, K),), dtype=torch.uint8, device=DEV)
+    wq.wq_repack_q4k(dev(raw), packed, N, K)
+    go = Guarded((N, K), torch.float32)
+    wq.dequant_q4k(packed, None, go.t, N, K, layout=wq.WQ_LAYOUT_B200_V1)
+    torch.cuda.synchronize()
+    go.check("q4_K B200_V1 dequant export")
+    assert wq.last_kernel() == "q4k.dequant.v1"
+    ref = oracle.dequant_q4k(raw, N, K).astype(np.float32)
+    assert np.array_equal(go.t.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
 # ----------------------------------------------------------- GEMV, whole outputs
 
 @gpu

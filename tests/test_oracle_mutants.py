@@ -102,6 +102,27 @@ def _dequant_int4_block_off_by_one(w_packed, scales, zeros, N, K, block_size):
     return (q - z[:, blk]).astype(np.float64) * s[:, blk]
 
 
+def _silu_without_a(a):
+    a = np.asarray(a, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(-a))
+
+
+def _silu_reflected(a):
+    a = np.asarray(a, dtype=np.float64)
+    return a / (1.0 + np.exp(a))
+
+
+def _swiglu_gate_up_swapped(Wg, Wu, x):
+    return oq.silu(oq.gemv(Wu, x)) * oq.gemv(Wg, x)
+
+
+def _swiglu_tolerance_no_up_term(a, b, Ba, Bb, rel=2e-3, abs_=1e-3):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    ea = rel * np.asarray(Ba, dtype=np.float64) + abs_
+    prop = oq.SILU_MAX_SLOPE * ea * np.abs(b)
+    return prop + 2.0 ** -10 * (np.abs(oq.silu(a) * b) + prop) + abs_
+
+
 MUTANTS = {
     "int4 nibbles high-first": ("int4_codes", _int4_codes_high_first),
     "int4 default zero-point 0": ("int4_zero_points", _zero_points_default_zero),
@@ -117,6 +138,10 @@ MUTANTS = {
     "bound without abs": ("bound", _bound_no_abs),
     "acceptance twice as loose": ("accept", _accept_loose),
     "bf16 offset ignored": ("dequant_bf16", _dequant_bf16_ignores_offset),
+    "silu without the a factor": ("silu", _silu_without_a),
+    "silu reflected": ("silu", _silu_reflected),
+    "swiglu gate and up swapped": ("swiglu_gemv", _swiglu_gate_up_swapped),
+    "swiglu tolerance without the up error": ("swiglu_tolerance", _swiglu_tolerance_no_up_term),
 }
 
 

@@ -29,5 +29,7 @@ from .api import (  # noqa: F401
     wq_layout_version,
     wq_q4k_bytes,
     wq_q4k_dsc_bytes,
+    wq_q4k_packed_bytes,
+    wq_repack_q4k,
     wq_test_expire_wait,
 )

@@ -41,6 +41,8 @@ SIGNATURES = {
     "wq_int4_packed_bytes": (_sz, [_i, _i, _i, _i]),
     "wq_q4k_bytes": (_sz, [_i, _i]),
     "wq_q4k_dsc_bytes": (_sz, [_i, _i]),
+    "wq_q4k_packed_bytes": (_sz, [_i, _i, _i]),
+    "wq_repack_q4k": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "wq_build_q4k_dsc": (_i, [_vp, _i, _i, _vp]),
     "wq_build_q4k_dsc_device": (_i, [_vp, _vp, _i, _i, _vp]),
     "wq_last_error": (_cp, []),

@@ -87,6 +87,14 @@ def wq_q4k_dsc_bytes(N, K) -> int:
     return int(lib().wq_q4k_dsc_bytes(N, K))
 
 
+def wq_q4k_packed_bytes(N, K, layout=WQ_LAYOUT_B200_V1) -> int:
+    return int(lib().wq_q4k_packed_bytes(N, K, layout))
+
+
+def wq_repack_q4k(w_q4k, w_out, N, K, to_layout=WQ_LAYOUT_B200_V1, stream=None):
+    _check(lib().wq_repack_q4k(_ptr(w_q4k), _ptr(w_out), N, K, to_layout, _stream(stream)), "wq_repack_q4k")
+
+
 def wq_build_q4k_dsc(w_q4k_host: np.ndarray, N: int, K: int) -> np.ndarray:
     """Host plane builder: returns float32 [K/32, N, 2] built by libwq's C++ packer."""
     src = np.ascontiguousarray(w_q4k_host, dtype=np.uint8)

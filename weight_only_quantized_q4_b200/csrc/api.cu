@@ -546,8 +546,14 @@ bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clust
   const char* sk_env = std::getenv("WQ_V1_STAGE_KB");
   const int stage_budget = (sk_env ? std::max(1, std::atoi(sk_env)) : stage_kb) * 1024;
   p.tps = W * std::max(1, stage_budget / (W * p.tb));
-  const char* pre_env = std::getenv("WQ_V1_PRE");  // stages requested before the x copy (tuning)
-  p.pre = pre_env ? std::max(0, std::atoi(pre_env)) : 2;
+  // Before waiting for the previous kernel: an L2 prefetch of the head of the
+  // CTA's stream (safe whatever that kernel wrote; WQ_V1_PFKB, KB), or ring
+  // stages copied to shared memory (WQ_V1_PRE, stages; only correct when the
+  // kernel right before the GEMV does not write its weights).
+  const char* pre_env = std::getenv("WQ_V1_PRE");
+  p.pre = pre_env ? std::max(0, std::atoi(pre_env)) : 0;
+  const char* pf_env = std::getenv("WQ_V1_PFKB");
+  p.pf_bytes = p.pre > 0 ? 0 : (pf_env ? std::max(0, std::atoi(pf_env)) : 96) * 1024;
   const char* h_env = std::getenv("WQ_V1_HINT");
   p.hint = h_env ? (std::atoi(h_env) != 0) : 1;
   p.stage_bytes = p.tps * p.tb;
@@ -594,8 +600,20 @@ bool plan_v1(int M, int N, int K, int block_size, int sms, V1Plan* out) {
   const char* c_env = std::getenv("WQ_V1_C");
   const int c_force = c_env ? std::atoi(c_env) : 0;
   const char* cps_env = std::getenv("WQ_V1_CTAS");
-  const int cps_force = cps_env ? std::max(1, std::min(2, std::atoi(cps_env))) : 0;
+  const int cps_force = cps_env ? std::max(1, std::min(4, std::atoi(cps_env))) : 0;
   const int n_bands = (N + 15) / 16;
+  // Explicit geometry (tuning): WQ_V1_BPC bands per cluster, WQ_V1_CTAS CTAs
+  // per SM (1..4), WQ_V1_C CTAs per cluster along K, WQ_V1_W consumer warps,
+  // WQ_V1_STAGE_KB stage size.
+  if (const char* bpc_env = std::getenv("WQ_V1_BPC")) {
+    const int bpc = std::max(1, std::atoi(bpc_env));
+    const int C = c_force > 1 ? c_force : 1;
+    const int cps = cps_force > 0 ? cps_force : 1;
+    const int ncl = (n_bands + bpc - 1) / bpc;
+    for (int kb : {52, 36, 24, 18, 12, 8, 4})
+      if (plan_v1_geom(M, N, K, block_size, C, 8, ncl, out, kb, cps)) return true;
+    return false;
+  }
   if (c_force > 1) {
     // cluster split along K (measured slower than whole bands per CTA on B200:
     // smaller copies per band and an extra cluster reduction), on request only
@@ -1140,13 +1158,25 @@ int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const v
 int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K, int layout, void* stream) {
   int rc = check_dims(1, N, K);
   if (rc) return rc;
-  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
+  if (layout != WQ_LAYOUT_CANONICAL && layout != WQ_LAYOUT_B200_V1)
+    return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
+  if (layout == WQ_LAYOUT_B200_V1 && w_dsc)
+    return fail(WQ_ERR_LAYOUT, "dequant_q4k: the B200_V1 q4_K stream carries its coefficients; w_dsc must be NULL");
   if (K % 256) return fail(WQ_ERR_ARG, "dequant_q4k: K must be a multiple of 256");
   if (!w_q4k || !w_out) return fail(WQ_ERR_ARG, "dequant_q4k: null pointer");
   if (!aligned16(w_q4k) || (w_dsc && !aligned16(w_dsc)) || !aligned16(w_out))
     return fail(WQ_ERR_ALIGN, "dequant_q4k: device pointers must be 16-byte aligned");
   DeviceInfo di;
   if ((rc = device_info(&di))) return rc;
+  if (layout == WQ_LAYOUT_B200_V1) {
+    const long long vwords = static_cast<long long>(N) * (K / 8);
+    const int vgrid = static_cast<int>(std::min<long long>((vwords + 255) / 256, di.sms * 32ll));
+    dequant_q4k_v1_kernel<<<vgrid, 256, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<const uint8_t*>(w_q4k),
+                                                                                w_out, N, K);
+    if ((rc = launch_check("dequant_q4k_v1 launch"))) return rc;
+    set_last_kernel("q4k.dequant.v1");
+    return WQ_OK;
+  }
   const long long words = static_cast<long long>(N) * (K / 256) * 32;
   const int grid = static_cast<int>(std::min<long long>((words + 255) / 256, di.sms * 32ll));
   dequant_q4k_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -1180,6 +1210,28 @@ int wq_repack_int4(const void* w_canonical, const void* scales_f16, const void* 
       K, block_size);
   if ((rc = launch_check("repack_int4 meta launch"))) return rc;
   set_last_kernel("int4.repack.v1");
+  return WQ_OK;
+}
+
+int wq_repack_q4k(const void* w_q4k, void* w_out, int N, int K, int to_layout, void* stream) {
+  if (N <= 0 || K <= 0 || K % 256) return fail(WQ_ERR_ARG, "wq_repack_q4k: need N > 0 and K % 256 == 0");
+  if (!w_q4k || !w_out) return fail(WQ_ERR_ARG, "wq_repack_q4k: null pointer");
+  if (to_layout != WQ_LAYOUT_B200_V1) return fail(WQ_ERR_LAYOUT, "wq_repack_q4k: target layout must be B200_V1");
+  if (!aligned16(w_q4k) || !aligned16(w_out))
+    return fail(WQ_ERR_ALIGN, "wq_repack_q4k: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const long long tiles = static_cast<long long>((N + 15) / 16) * (K / 256);
+  const int g1 = static_cast<int>(std::min<long long>((tiles * 128 + 255) / 256, di.sms * 32ll));
+  repack_q4k_v1_codes_kernel<<<g1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_q4k), static_cast<uint8_t*>(w_out), N, K);
+  if ((rc = launch_check("repack_q4k codes launch"))) return rc;
+  const int g2 = static_cast<int>(std::min<long long>((tiles * 16 + 255) / 256, di.sms * 32ll));
+  repack_q4k_v1_meta_kernel<<<g2, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_q4k), static_cast<uint8_t*>(w_out), N, K);
+  if ((rc = launch_check("repack_q4k meta launch"))) return rc;
+  set_last_kernel("q4k.repack.v1");
   return WQ_OK;
 }
 

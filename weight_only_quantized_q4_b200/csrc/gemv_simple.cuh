@@ -48,6 +48,35 @@ __host__ __device__ __forceinline__ long long int4_v1_zero_offset(long long row,
          ((row & 15) >> 1);
 }
 
+// B200_V1 q4_K stream geometry (see include/wq.h): bands of 16 rows, K/256
+// tiles per band, one super-block of the band's rows per tile, 2304 bytes:
+// 2048 code bytes in warp-MMA fragment order (the int4 B200_V1 code order over
+// eight 32-k groups, group = chunk), 16 (d, dmin) fp16 pairs, then 64 24-bit
+// scale entries: entry (pair p, row r) at 2112 + 3·(16p + r) holds
+// sc_{2p} | sc_{2p+1} << 6 | m_{2p} << 12 | m_{2p+1} << 18.
+constexpr int kQ4KV1TileBytes = 2304;
+__host__ __device__ __forceinline__ long long q4k_v1_tile_offset(long long row, int k, int K) {
+  return ((row >> 4) * (K / 256) + (k >> 8)) * static_cast<long long>(kQ4KV1TileBytes);
+}
+__host__ __device__ __forceinline__ long long q4k_v1_word_offset(long long row, int k8, int K) {
+  const int r = static_cast<int>(row & 15);
+  const int g = r & 7, r8 = r >> 3;
+  const int kk = k8 & 255;
+  const int gi = kk >> 5, t = (kk & 31) >> 3;
+  return q4k_v1_tile_offset(row, k8, K) + (gi >> 1) * 512 + (4 * g + t) * 16 + 4 * (2 * (gi & 1) + r8);
+}
+__host__ __device__ __forceinline__ long long q4k_v1_dd_offset(long long row, int k, int K) {
+  return q4k_v1_tile_offset(row, k, K) + 2048 + 4 * (row & 15);
+}
+__host__ __device__ __forceinline__ long long q4k_v1_entry_offset(long long row, int k, int K) {
+  const int c = (k & 255) >> 5;
+  return q4k_v1_tile_offset(row, k, K) + 2112 + 3 * (16 * (c >> 1) + (row & 15));
+}
+// The 24-bit entry of (pair, row) from three bytes.
+__device__ __forceinline__ uint32_t q4k_v1_entry(const uint8_t* e) {
+  return static_cast<uint32_t>(e[0]) | (static_cast<uint32_t>(e[1]) << 8) | (static_cast<uint32_t>(e[2]) << 16);
+}
+
 struct SimpleParams {
   const void* x;
   const uint8_t* w;
@@ -87,6 +116,18 @@ __device__ __forceinline__ float weight_scalar(const SimpleParams& p, int row, i
     }
     return static_cast<float>(static_cast<int>(q) - static_cast<int>(z)) * h16_to_f32(sb);
   } else if constexpr (F == Fmt::Q4K || F == Fmt::Q4KDsc) {
+    if (F == Fmt::Q4K && p.layout == 1) {
+      const int pos = int4_v1_nibble_pos(k & 7);
+      const uint32_t byte = p.w[q4k_v1_word_offset(row, k & ~7, p.K) + (pos >> 1)];
+      const uint32_t q = (pos & 1) ? (byte >> 4) : (byte & 15u);
+      const uint32_t dd = *reinterpret_cast<const uint32_t*>(p.w + q4k_v1_dd_offset(row, k, p.K));
+      const uint32_t ent = q4k_v1_entry(p.w + q4k_v1_entry_offset(row, k, p.K));
+      const int hi = ((k & 255) >> 5) & 1;
+      const uint32_t sc = (ent >> (6 * hi)) & 63u, mn = (ent >> (12 + 6 * hi)) & 63u;
+      const float A = __fmul_rn(h16_to_f32(dd), static_cast<float>(sc));
+      const float B = -__fmul_rn(h16_to_f32(dd >> 16), static_cast<float>(mn));
+      return fmaf(A, static_cast<float>(q), B);
+    }
     const uint8_t* blk = p.w + (static_cast<long long>(row) * (p.K / 256) + (k >> 8)) * 144;
     const int e = k & 255;
     const int c = e >> 5;
@@ -322,6 +363,104 @@ __global__ void repack_int4_v1_meta_kernel(const uint8_t* scales, const uint8_t*
     tp[1024 + 32 * bpt + bt * 8 + rp] = static_cast<uint8_t>(zbyte);
     if (bt == 0 && rp == 0)
       for (int o = 1024 + 40 * bpt; o < tb; ++o) tp[o] = 0;
+  }
+}
+
+// q4_K B200_V1 export: thread per 32-bit code word (8 codes of one chunk of
+// one row), coefficients from the tile's (d, dmin) pair and 24-bit entry.
+__global__ void dequant_q4k_v1_kernel(const uint8_t* w, float* out, int N, int K) {
+  const long long words_per_row = K / 8;
+  const long long total = static_cast<long long>(N) * words_per_row;
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = t / words_per_row;
+    const int k0 = 8 * static_cast<int>(t - row * words_per_row);
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(w + q4k_v1_word_offset(row, k0, K));
+    const uint32_t dd = *reinterpret_cast<const uint32_t*>(w + q4k_v1_dd_offset(row, k0, K));
+    const uint32_t ent = q4k_v1_entry(w + q4k_v1_entry_offset(row, k0, K));
+    const int hi = ((k0 & 255) >> 5) & 1;
+    const float A = __fmul_rn(h16_to_f32(dd), static_cast<float>((ent >> (6 * hi)) & 63u));
+    const float B = -__fmul_rn(h16_to_f32(dd >> 16), static_cast<float>((ent >> (12 + 6 * hi)) & 63u));
+    // pairs by nibble position (p0,p4) (p1,p5) (p2,p6) (p3,p7); position p holds code e = 2·(p & 3) + (p >> 2)
+    const uint32_t pr[4] = {lo4(v), hi4(v), lo4(v >> 8), hi4(v >> 8)};
+    float* o = out + row * K + k0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool high = (i & 1) != 0;
+      const int p0 = (i >> 1) * 2 + (high ? 1 : 0);
+      const int e0 = 2 * (p0 & 3) + (p0 >> 2), e1 = 2 * ((p0 + 4) & 3) + ((p0 + 4) >> 2);
+      o[e0] = fmaf(A, code_of(pr[i], 0, high), B);
+      o[e1] = fmaf(A, code_of(pr[i], 1, high), B);
+    }
+  }
+}
+
+// Canonical q4_K -> B200_V1, codes: thread per 16-byte code chunk of a tile
+// (128 per tile; rows past N get zero codes).
+__global__ void repack_q4k_v1_codes_kernel(const uint8_t* w, uint8_t* out, int N, int K) {
+  const long long n_bands = (N + 15) / 16;
+  const int tpb = K / 256;
+  const long long chunks = n_bands * tpb * 128;
+  for (long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
+       c += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long tile = c >> 7;  // band * tpb + sb
+    const int q = static_cast<int>(c & 127);
+    const long long band = tile / tpb;
+    const int sb = static_cast<int>(tile - band * tpb);
+    const int h = q >> 5, lane = q & 31;
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gi = 2 * h + (j >> 1), r8 = j & 1;  // gi = chunk of the super-block
+      const long long row = 16 * band + g + 8 * r8;
+      uint32_t o = 0;
+      if (row < N) {
+        const uint8_t* qs = w + (row * tpb + sb) * 144 + 16 + 32 * (gi >> 1) + 8 * t;
+        const int sh = 4 * (gi & 1);  // even chunk: low nibbles of its run, odd: high
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o |= ((static_cast<uint32_t>(qs[e]) >> sh) & 15u) << (4 * int4_v1_nibble_pos(e));
+      }
+      v[j] = o;
+    }
+    *reinterpret_cast<uint4*>(out + tile * kQ4KV1TileBytes + q * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+// Canonical q4_K -> B200_V1, coefficients: thread per (tile, row): the row's
+// (d, dmin) word and its four 24-bit (scale, min) pair entries (zeros for pad rows).
+__global__ void repack_q4k_v1_meta_kernel(const uint8_t* w, uint8_t* out, int N, int K) {
+  const long long n_bands = (N + 15) / 16;
+  const int tpb = K / 256;
+  const long long items = n_bands * tpb * 16;
+  for (long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
+       it += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(it & 15);
+    const long long tile = it >> 4;
+    const long long band = tile / tpb;
+    const int sb = static_cast<int>(tile - band * tpb);
+    const long long row = 16 * band + r;
+    uint8_t* tp = out + tile * kQ4KV1TileBytes;
+    uint32_t dd = 0, e[4] = {0u, 0u, 0u, 0u};
+    if (row < N) {
+      const uint32_t* hw = reinterpret_cast<const uint32_t*>(w + (row * tpb + sb) * 144);
+      dd = hw[0];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        uint32_t s0, m0, s1, m1;
+        q4k_scale_min(hw[1], hw[2], hw[3], 2 * p, s0, m0);
+        q4k_scale_min(hw[1], hw[2], hw[3], 2 * p + 1, s1, m1);
+        e[p] = s0 | (s1 << 6) | (m0 << 12) | (m1 << 18);
+      }
+    }
+    *reinterpret_cast<uint32_t*>(tp + 2048 + 4 * r) = dd;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      uint8_t* ep = tp + 2112 + 3 * (16 * p + r);
+      ep[0] = static_cast<uint8_t>(e[p]);
+      ep[1] = static_cast<uint8_t>(e[p] >> 8);
+      ep[2] = static_cast<uint8_t>(e[p] >> 16);
+    }
   }
 }
 

@@ -49,7 +49,8 @@ struct V1Params {
   int C;             // CTAs per cluster (along K)
   int W;             // consumer warps
   int hint;          // 1: weight copies carry the L2 evict-first policy
-  int pre;           // stages requested before waiting for the previous kernel
+  int pre;           // stages copied to shared memory before waiting for the previous kernel
+  int pf_bytes;      // bytes of the CTA's stream prefetched into L2 before that wait (pre == 0)
   int Mp;            // M rounded up to even (stride of a partial row)
   int off_x;         // activations [M][tpc·128] fp16
   int off_zero;      // 256 zero bytes
@@ -174,10 +175,24 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
       int slot = 0, bl = 0, ti = 0;  // next tile: band bl (local), k-tile ti (local)
       uint32_t phase = 0;
       const int pre = min(p.pre, n_stages);
-      // The weights are read-only: the first `pre` stages are requested before
-      // the previous kernel has finished.  The activations may be its output;
-      // they are copied next, ahead of the rest of the weight stream (a load
-      // queued behind a deep weight stream waits for all of it).
+      // Before the wait for the previous kernel, the head of this CTA's weight
+      // stream is either prefetched into L2 (pf_bytes; L2 is the point of
+      // coherence, so a prefetch can never return data older than a write of
+      // the previous kernel) or, when the caller has declared that no kernel
+      // right before a GEMV writes its weights, copied straight into the ring
+      // (`pre` stages).  The activations may be the previous kernel's output;
+      // they are copied right after the wait, ahead of the rest of the weight
+      // stream (a load queued behind a deep weight stream waits for all of it).
+      if (p.pf_bytes > 0) {
+        long long left = p.pf_bytes;
+        for (int b = 0; b < n_bl && left > 0; ++b) {
+          const uint8_t* run = base + b * band_bytes;
+          const long long rb = min(left, static_cast<long long>(p.tpc) * p.tb);
+          for (long long o = 0; o < rb; o += 32768)
+            prefetch_l2(run + o, static_cast<uint32_t>(min(rb - o, 32768ll)));
+          left -= rb;
+        }
+      }
       auto copy_x = [&]() {
         grid_wait_prior();
         mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.M) * 2u * Kc);
@@ -358,9 +373,12 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
     // partials of every band are in `part` of each CTA of the cluster: add them
     // in rank order, the CTAs splitting the outputs between them
     v1d::cluster_sync();
+    // The producer warp (warp W) has exited: number the W consumer warps and
+    // the reducer warp (W + 1) contiguously so every item has a thread.
     const int nthr_red = (W + 1) * 32;
+    const int rt = warp == W + 1 ? W * 32 + lane : tid;
     const int items = n_bl * 16 * p.M;
-    for (int i = static_cast<int>(rank) * nthr_red + tid; i < items; i += p.C * nthr_red) {
+    for (int i = static_cast<int>(rank) * nthr_red + rt; i < items; i += p.C * nthr_red) {
       const int n = i % p.M, br = i / p.M, row = br & 15, b = br >> 4;
       const int r = (b_begin + b) * 16 + row;
       float sum = 0.f;

@@ -76,6 +76,11 @@ extern "C" size_t wq_int4_packed_bytes(int N, int K, int block_size, int layout)
   return static_cast<size_t>((N + 15) / 16) * (K / 128) * WQ_INT4_V1_TILE_BYTES(block_size);
 }
 
+extern "C" size_t wq_q4k_packed_bytes(int N, int K, int layout) {
+  if (N <= 0 || K <= 0 || K % 256 || layout != WQ_LAYOUT_B200_V1) return 0;
+  return static_cast<size_t>((N + 15) / 16) * (K / 256) * WQ_Q4K_V1_TILE_BYTES;
+}
+
 extern "C" size_t wq_int4_bytes(int N, int K, int block_size, int layout) {
   if (N <= 0 || K <= 0) return 0;
   if (block_size < 16 || block_size > 256 || (block_size & (block_size - 1)) || K % block_size) return 0;
