@@ -20,11 +20,16 @@
  *    the calling thread used (a liveness label such as
  *    "int4.gemv.v1s.m1.c1"), so a test can assert which path ran.
  *  - The decode GEMV kernels are launched with programmatic dependent launch:
- *    a call may start streaming its (read-only) weights while the previous
- *    kernel in the stream is still running, and waits for that kernel to
- *    complete before it reads x or writes y.  Stream order is preserved for
- *    the caller; a following kernel that itself uses programmatic dependent
- *    launch must wait (griddepcontrol.wait) before reading y, as usual.
+ *    a call may start while the previous kernel in the stream is still
+ *    running.  Until that kernel has completed, a call only prefetches the
+ *    head of its weight stream into L2 (L2 is the point of coherence, so this
+ *    can never return data older than a write of that kernel); it copies
+ *    weights into shared memory or registers, reads x and writes y only
+ *    after waiting for the previous kernel to complete.  The previous kernel
+ *    may therefore write this call's weights (a repack, an upload kernel)
+ *    with no synchronization in between.  A following kernel that itself
+ *    uses programmatic dependent launch must wait (griddepcontrol.wait)
+ *    before reading y, as usual.
  *  - The first call on a device configures kernel attributes and looks up the
  *    driver's tensor-map encoder; make it before capturing a CUDA graph.
  *  - Environment variables read at each call, for tests and tuning only:

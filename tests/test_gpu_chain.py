@@ -98,6 +98,13 @@ def test_chained_calls_match_isolated_calls(first, second, graph):
         assert np.array_equal(y2.cpu().view(torch.int16).numpy(), w.view(torch.int16).numpy()), (first, second, i)
 
 
+def _kernel_copy(dst, src):
+    """dst = src through an elementwise torch kernel (not a memcpy), so the
+    write comes from a kernel the GEMV may overlap with."""
+    it = torch.int16 if src.element_size() == 2 else torch.uint8
+    torch.bitwise_or(src.view(it), 0, out=dst.view(it))
+
+
 @gpu
 @pytest.mark.parametrize("case", ["int4_v1_repack", "int4_canonical_torch_kernel", "q4k_torch_kernel"])
 def test_weights_written_by_the_kernel_right_before(case):
@@ -137,10 +144,10 @@ def test_weights_written_by_the_kernel_right_before(case):
                 wq.gemv_int4_blockwise(dx, live, None, None, y, 1, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1, stream=s)
             elif case == "int4_canonical_torch_kernel":
                 for dst, t in zip(live, src):
-                    torch.bitwise_or(t, 0, out=dst)  # an elementwise kernel writes the weights
+                    _kernel_copy(dst, t)
                 wq.gemv_int4_blockwise(dx, live[0], live[1], live[2], y, 1, N, K, 128, stream=s)
             else:
-                torch.bitwise_or(src[0], 0, out=live[0])
+                _kernel_copy(live[0], src[0])
                 wq.gemv_q4k(dx, live[0], y, 1, N, K, stream=s)
     torch.cuda.synchronize()
     wq.wq_device_status()

@@ -142,6 +142,12 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
     const uint64_t policy = policy_evict_first();
     const uint32_t sbytes = static_cast<uint32_t>(p.v1_tps * p.v1_tb);
     const uint8_t* src = p.w + static_cast<long long>(b_begin) * p.v1_tpb * p.v1_tb;
+    // Until the previous kernel has completed only L2 may be filled (it is the
+    // point of coherence, so a prefetch cannot return data older than a write
+    // of that kernel): prefetch the first ring's worth of this CTA's stream,
+    // then wait, then copy into shared memory.
+    for (int S = 0; S < min(total, p.NS); ++S) prefetch_l2(src + static_cast<long long>(S) * sbytes, sbytes);
+    grid_wait_prior();
     int ks = 0, slot = 0;
     uint32_t phase = 0;
     for (int S = 0; S < total; ++S) {
@@ -154,7 +160,6 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
       const uint32_t xb = p.x_res ? (S == 0 ? p.M * 2u * p.K : 0u) : p.M * 2u * kc;
       mbar_arrive_expect_tx(&full[slot], sbytes + xb);
       bulk_g2s_stream(st, src + static_cast<long long>(S) * sbytes, sbytes, &full[slot], policy);
-      grid_wait_prior();  // x may be the previous kernel's output (returns at once after the first time)
       if (p.x_res) {
         if (S == 0) bulk_g2s(smem + p.off_xres, p.x, p.M * 2u * p.K, &full[slot]);
       } else {
@@ -173,6 +178,27 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
   }
   if (warp == W) {
     const uint64_t policy = policy_evict_first();
+    {
+      // L2 prefetch of the rows of this CTA's first band (first ring's worth of
+      // stages), the only weight traffic issued before the previous kernel
+      // has completed (see the B200_V1 producer above)
+      const int r0 = b_begin * p.rpb, nr = min(p.rpb, p.N - r0);
+      const int ns = min(p.n_kst, p.NS);
+      long long seg = 0;
+      if constexpr (F == Fmt::Int4) seg = static_cast<long long>(min(p.K, ns * p.Kc)) / 2;
+      else if constexpr (F == Fmt::BF16) seg = 2ll * min(p.K, ns * p.Kc);
+      else seg = static_cast<long long>(min(p.K, ns * p.Kc) / 256) * 144;
+      if (b_begin < b_end)
+        for (int j = lane; j < nr; j += 32) {
+          const uint8_t* rowp = p.w + static_cast<long long>(r0 + j) * p.row_bytes;
+          // whole 16-byte units inside the segment only (never past the tensor)
+          const uint64_t a = (reinterpret_cast<uint64_t>(rowp) + 15) & ~15ull;
+          const uint64_t e = (reinterpret_cast<uint64_t>(rowp) + seg) & ~15ull;
+          for (uint64_t o = a; o < e; o += 32768)
+            prefetch_l2(reinterpret_cast<const void*>(o), static_cast<uint32_t>(e - o < 32768ull ? e - o : 32768ull));
+        }
+    }
+    grid_wait_prior();
     int band = b_begin, ks = 0, slot = 0;  // stage bookkeeping kept incremental (no divisions)
     uint32_t phase = 0;
     for (int S = 0; S < total; ++S) {
@@ -235,7 +261,6 @@ __global__ void __launch_bounds__(544, 1) gemv_tc_kernel(const TCParams p) {
           bulk_g2s_stream(st + j * p.pitch, p.w + static_cast<long long>(r0 + j) * p.row_bytes + kofs, seg,
                           &full[slot], policy);
       }
-      grid_wait_prior();  // x may be the previous kernel's output (returns at once after the first time)
       if (p.x_res) {
         // activations for the whole kernel ride on the first stage's barrier
         if (S == 0 && lane == 0) bulk_g2s(smem + p.off_xres, p.x, p.M * 2u * p.K, &full[slot]);

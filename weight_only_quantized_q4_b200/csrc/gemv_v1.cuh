@@ -487,7 +487,12 @@ __global__ void __launch_bounds__(kV1RMaxWarps * 32, 1) gemv_v1r_kernel(const V1
   const int nthr = W * 32;
   const int cnt = warp < n_tiles ? (n_tiles - warp + W - 1) / W : 0;  // this warp's tiles: warp + W·i
   TileRegs q[P];
-  // weights do not depend on the previous kernel: request the first P tiles now
+  // Before the previous kernel has completed only L2 is warmed (a register
+  // load could return weights older than a write of that kernel): lane 0
+  // prefetches this warp's first P tiles, the loads follow the wait.
+  if (lane == 0)
+    for (int j = 0; j < P && j < cnt; ++j) prefetch_l2(base + static_cast<long long>(warp + W * j) * p.tb, p.tb);
+  grid_wait_prior();  // x, and possibly the weights, may be the previous kernel's output
 #pragma unroll
   for (int j = 0; j < P; ++j)
     if (j < cnt) tile_ldg(base + static_cast<long long>(warp + W * j) * p.tb, lane, g, q[j]);
@@ -495,7 +500,6 @@ __global__ void __launch_bounds__(kV1RMaxWarps * 32, 1) gemv_v1r_kernel(const V1
   float* xs = reinterpret_cast<float*>(smem + p.off_xs);
   uint8_t* xsm = smem + p.off_x;
   uint8_t* zbuf = smem + p.off_zero;
-  grid_wait_prior();  // x may be the previous kernel's output
   {
     // x -> shared memory, and Σx (×2^-24) per (tile, batch column): four
     // threads per tile and column, 32 k each
