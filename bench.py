@@ -58,6 +58,7 @@ for _M in (1, 2, 4, 8):
     for _N, _K in ((4096, 4096), (11008, 4096), (4096, 11008)):
         WORKLOADS[f"q4k_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=False, workload=4)
         WORKLOADS[f"q4k_dsc_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=True, workload=4)
+        WORKLOADS[f"q4k_v1_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=False, workload=4, layout=1)
 for _M in (1, 3, 8):
     for _N, _K in ((1536, 1536), (256, 1536), (1536, 6912), (151936, 1536)):
         WORKLOADS[f"bf16_m{_M}_{_N}x{_K}"] = dict(fmt="bf16", M=_M, N=_N, K=_K, workload=2)
@@ -76,7 +77,7 @@ DEFAULT_WORKLOAD = "int4_b128_zp_v1_m1_4096x14336"
 METRIC = "achieved HBM GB/s and \u00b5s/call per quantized GEMV at M=1..8 vs ~8 TB/s peak"
 SWEEP_BATCHED = [f"batched_{f}_m{m}_{n}x{k}" for f in ("int4_b128_zp", "q4k") for m in (16, 64, 128)
                  for n, k in ((4096, 4096), (14336, 4096), (32000, 4096))]
-SWEEP = ["int4_b128_zp_v1_m1_4096x14336", "int4_b128_zp_v1_m2_4096x14336", "int4_b128_zp_v1_m4_4096x14336", "int4_b128_zp_v1_m8_4096x14336",
+SWEEP = ["q4k_v1_m1_4096x11008", "q4k_v1_m4_4096x11008", "q4k_v1_m1_11008x4096", "int4_b128_zp_v1_m1_4096x14336", "int4_b128_zp_v1_m2_4096x14336", "int4_b128_zp_v1_m4_4096x14336", "int4_b128_zp_v1_m8_4096x14336",
          "int4_b128_zp_v1_m1_14336x4096", "int4_b128_zp_v1_m1_4096x4096",
          "int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
          "int4_b32_m1_256x1024", "q4k_m1_4096x11008", "q4k_dsc_m1_4096x11008", "q4k_m4_11008x4096",
@@ -198,6 +199,10 @@ class DeviceWorkload:
             self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
         elif w["fmt"] == "q4k":
             raw = torch.from_numpy(host["raw"]).to(dev)
+            if w.get("layout", 0) == 1:  # offline repack to the B200_V1 q4_K band stream
+                packed = torch.empty(wq.wq_q4k_packed_bytes(N, K, 1), dtype=torch.uint8, device=dev)
+                wq.wq_repack_q4k(raw, packed, N, K, 1)
+                raw = packed
             for _ in range(self.R):
                 c = [raw.clone()]
                 if w["dsc"]:
@@ -238,7 +243,7 @@ class DeviceWorkload:
             if w["dsc"]:
                 wq.gemv_q4k_dsc(x, c[0], c[1], y, M, self.N, self.K, stream=stream)
             else:
-                wq.gemv_q4k(x, c[0], y, M, self.N, self.K, stream=stream)
+                wq.gemv_q4k(x, c[0], y, M, self.N, self.K, layout=w.get("layout", 0), stream=stream)
         else:
             wq.gemv_bf16(x, c[0], y, M, self.N, self.K, stream=stream)
 

@@ -137,6 +137,21 @@ int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* sca
                         const void* zeros_u4, void* y_f16, int M, int N, int K,
                         int block_size, int layout, void* stream);
 
+/* Fused gate / up projection of a SwiGLU feed-forward block:
+ *   y[M,N] fp16 = silu(x·W_gateᵀ) ⊙ (x·W_upᵀ),  silu(a) = a·σ(a) = a / (1 + e^-a),
+ * both projections accumulated in fp32 from the same resident activations and
+ * combined in fp32 before the one rounding to fp16 (the fused "swiglu" launch
+ * of minfer doc 62 "r59 — q4_K W_dsc plane", §3.3; the page names the launch,
+ * the formula is the SwiGLU definition).  w_gate_up is the fused B200_V1
+ * stream of wq_repack_int4_gate_up: in every 16-row band, the tiles alternate
+ * gate tile s, up tile s (each a B200_V1 int4 tile).  block_size 128 or 256,
+ * K % 128 == 0, layout WQ_LAYOUT_B200_V1; up to 8 rows of x per launch whose
+ * activations fit in 120 KB (more rows run in chunks).  Errors: WQ_ERR_ARG,
+ * WQ_ERR_ALIGN, WQ_ERR_LAYOUT, WQ_ERR_UNSUPPORTED (K too large), WQ_ERR_DEVICE,
+ * WQ_ERR_CUDA. */
+int gemv_int4_swiglu(const void* x_f16, const void* w_gate_up, void* y_f16, int M, int N, int K,
+                     int block_size, int layout, void* stream);
+
 /* y[M,N] fp16 = x[M,K] fp16 · dequant(q4_K)ᵀ, scales decoded in-kernel from
  * the packed 6-bit fields.  K % 256 == 0.  w_q4k is N·(K/256)·144 bytes. */
 int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K,
@@ -189,6 +204,19 @@ int wq_repack_int4(const void* w_canonical, const void* scales_f16, const void* 
 
 /* Bytes of the buffer wq_repack_int4 writes (B200_V1), 0 if invalid. */
 size_t wq_int4_packed_bytes(int N, int K, int block_size, int layout);
+
+/* Rewrite two canonical int4 weights of the same shape (gate and up
+ * projections: codes, scales, zero-points or NULL each) into the fused
+ * B200_V1 gate-up stream at w_out (wq_int4_gate_up_packed_bytes bytes,
+ * device): tile slot 2i holds tile i of the gate stream, slot 2i + 1 tile i
+ * of the up stream.  block_size 128 or 256, K % 128 == 0.  Errors:
+ * WQ_ERR_ARG, WQ_ERR_LAYOUT, WQ_ERR_ALIGN, WQ_ERR_CUDA. */
+int wq_repack_int4_gate_up(const void* w_gate, const void* scales_gate, const void* zeros_gate,
+                           const void* w_up, const void* scales_up, const void* zeros_up, void* w_out,
+                           int N, int K, int block_size, int to_layout, void* stream);
+
+/* Bytes of the fused gate-up stream (twice the B200_V1 stream), 0 if invalid. */
+size_t wq_int4_gate_up_packed_bytes(int N, int K, int block_size, int layout);
 
 /* Bytes of a q4_K tensor and of its W_dsc plane; 0 for invalid arguments. */
 size_t wq_q4k_bytes(int N, int K);

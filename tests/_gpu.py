@@ -107,12 +107,20 @@ class Int4Case:
 # ----------------------------------------------------------------- q4_K
 
 class Q4KCase:
-    def __init__(self, M, N, K, workload=4):
-        self.M, self.N, self.K = M, N, K
+    def __init__(self, M, N, K, workload=4, layout=0):
+        self.M, self.N, self.K, self.layout = M, N, K, layout
         self.raw = synth.q4k_weights(N, K, workload=workload)
         self.x = synth.activations_f16(M, K, workload=workload)
         self.draw, self.dx = dev(self.raw), dev(self.x)
         self._plane = None
+        self.dw = self.draw
+        if layout == wq.WQ_LAYOUT_B200_V1:
+            g = Guarded((wq.wq_q4k_packed_bytes(N, K, layout),), torch.uint8)
+            wq.wq_repack_q4k(self.draw, g.t, N, K, layout)
+            torch.cuda.synchronize()
+            g.check("q4_K B200_V1 repack output")
+            self._packed_guard = g
+            self.dw = g.t
 
     def plane_dev(self):
         if self._plane is None:
@@ -129,7 +137,7 @@ class Q4KCase:
         if dsc:
             wq.gemv_q4k_dsc(self.dx, self.draw, self.plane_dev(), g.t, self.M, self.N, self.K, stream=stream)
         else:
-            wq.gemv_q4k(self.dx, self.draw, g.t, self.M, self.N, self.K, stream=stream)
+            wq.gemv_q4k(self.dx, self.dw, g.t, self.M, self.N, self.K, layout=self.layout, stream=stream)
         torch.cuda.synchronize()
         g.check(f"q4k y dsc={dsc} M={self.M} N={self.N} K={self.K}")
         return f16_of(g.t).astype(np.float64)
@@ -170,7 +178,7 @@ class BF16Case:
         return oracle.dequant_bf16(self.xb, self.M, self.K)
 
 
-VARIANTS = ("tc", "cc", "simple", "tc5", "v1s", "v1r", None)
+VARIANTS = ("tc", "cc", "simple", "tc5", "v1s", "v1r", "v1k", None)
 
 
 def each_variant(run, W, x, what):

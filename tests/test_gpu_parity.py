@@ -236,6 +236,33 @@ def test_gemv_int4_v1_cluster_split(C, M, N, K, bs, zeros, monkeypatch):
 
 
 @gpu
+@pytest.mark.parametrize("ctas", [1, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("N,K,bs,zeros", [(37, 2048, 128, True), (1000, 1536, 256, False), (300, 512, 128, True),
+                                          (4100, 1024, 128, True), (16, 4096, 256, True), (5, 128, 128, True),
+                                          (2368, 14336, 128, True)])
+def test_gemv_int4_v1_stream_k(ctas, M, N, K, bs, zeros, monkeypatch):
+    """The stream-K B200_V1 kernel: every CTA takes an equal run of tiles, so
+    bands are cut between CTAs (a band over up to 16 CTAs when N is small)
+    and finished by the fix-up through the split-band workspace.  The fix-up
+    adds the pieces in CTA order: two calls in a row agree bit for bit, and
+    so does a third call after other shapes have used the workspace."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1k")
+    monkeypatch.setenv("WQ_V1K_CTAS", str(ctas))
+    monkeypatch.setenv("WQ_V1K_W", "16" if ctas == 1 else "4")  # four CTAs per SM leave room for 4 warps' stages
+    c = Int4Case(M, N, K, bs, zeros, workload=25, layout=wq.WQ_LAYOUT_B200_V1)
+    y1 = c.run()
+    label = wq.last_kernel()
+    assert ".gemv.v1k." in label, label
+    check(y1, c.W(), c.x, f"v1k ctas={ctas} M={M} N={N} K={K} bs={bs} zp={zeros}")
+    assert np.array_equal(y1, c.run())
+    other = Int4Case(1, 77, 1024, 128, True, workload=26, layout=wq.WQ_LAYOUT_B200_V1)
+    other.run()
+    assert np.array_equal(y1, c.run())
+    wq.wq_device_status()
+
+
+@gpu
 @pytest.mark.parametrize("P", [2, 3, 4])
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("N,K,bs,zeros", [(37, 2048, 128, True), (1000, 1536, 256, False), (300, 512, 128, True),
@@ -258,7 +285,7 @@ def test_gemv_int4_v1_default_kernel_full_size():
     c = Int4Case(1, 4096, 14336, 128, True, workload=3, layout=wq.WQ_LAYOUT_B200_V1)
     rows = sample_rows(4096)
     y = c.run()
-    assert ".gemv.v1s." in wq.last_kernel(), wq.last_kernel()
+    assert ".gemv.v1k." in wq.last_kernel(), wq.last_kernel()
     W = oracle.dequant_int4(c.w[rows], c.s[rows], c.z[rows], len(rows), 14336, 128)
     check(y[:, rows], W, c.x, "B200_V1 4096x14336 sampled rows")
 
@@ -283,6 +310,21 @@ def test_gemv_q4k_small(M, N, K, dsc):
     c = Q4KCase(M, N, K, workload=22)
     labels = each_variant(lambda: c.run(dsc), c.W(), c.x, f"q4k dsc={dsc} M={M} N={N} K={K}")
     assert ".tc." in labels["tc"] and (".cc." in labels["cc"] or labels["cc"] == "unsupported"), labels
+
+
+@gpu
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 11])
+@pytest.mark.parametrize("N,K", [(3, 256), (129, 1024), (250, 2816), (64, 11008), (16, 4096)])
+def test_gemv_q4k_v1_layout(M, N, K):
+    """q4_K in the B200_V1 band stream: the stream-K kernel (MMA columns carrying
+    chunks at M < 8) and the scalar kernel, against the oracle; two calls in a
+    row agree bit for bit."""
+    c = Q4KCase(M, N, K, workload=27, layout=wq.WQ_LAYOUT_B200_V1)
+    labels = each_variant(lambda: c.run(False), c.W(), c.x, f"q4k v1 M={M} N={N} K={K}")
+    assert ".simple." in labels["simple"] and labels["tc"] == "unsupported" and labels["tc5"] == "unsupported", labels
+    if 2 * M * K <= 120 * 1024:
+        assert ".gemv.v1k." in labels["default"], labels
+        assert np.array_equal(c.run(False), c.run(False))
 
 
 @gpu
@@ -347,13 +389,24 @@ def test_gemm_tcgen05_cluster_split_k(S, M, fmt, monkeypatch):
         c = Int4Case(M, 300, 4096, 128, True, workload=31)
         run = c.run
     else:
-        c = Q4KCase(M, 300, 2048, workload=31)
+        c = Q4KCase(M, 300, 4096, workload=31)
         run = lambda: c.run(False)  # noqa: E731
     y = run()
     label = wq.last_kernel()
     assert ".gemm.tc5." in label and label.endswith(f".s{S}"), label
     check(y, c.W(), c.x, f"tcgen05 {fmt} M={M} S={S}")
     assert np.array_equal(y, run())
+
+
+@gpu
+def test_gemm_tcgen05_forced_split_follows_the_automatic_rule(monkeypatch):
+    """A forced cluster split must give every CTA an even number of 256-k raw
+    slots (the rule of the automatic choice); K = 2048 with S = 8 gives one."""
+    monkeypatch.setenv("WQ_TC5_S", "8")
+    c = Q4KCase(16, 300, 2048, workload=31)
+    with pytest.raises(wq.WQError) as e:
+        c.run(False)
+    assert e.value.code == wq.WQ_ERR_ARG
 
 
 # ----------------------------------------------------------- closed forms on the device
@@ -445,6 +498,16 @@ def test_full_int4_b128_sampled(M, N, K, layout):
 def test_full_int4_b32_config():
     c = Int4Case(1, 256, 1024, 32, False, workload=1, s_lo=0.005, s_hi=0.02)
     check(c.run(), c.W(), c.x, "int4 b32 256x1024")
+
+
+@gpu
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+@pytest.mark.parametrize("N,K", FULL_Q4K)
+def test_full_q4k_v1_sampled(M, N, K):
+    c = Q4KCase(M, N, K, workload=4, layout=wq.WQ_LAYOUT_B200_V1)
+    rows = sample_rows(N)
+    y = c.run(False)
+    check(y[:, rows], c.W(rows), c.x, f"q4k B200_V1 full {N}x{K} M={M} [{wq.last_kernel()}]")
 
 
 @gpu

@@ -6,6 +6,7 @@ The kernels live in libwq.so (C ABI in include/wq.h); this package is a thin
 ctypes binding with the same entry-point names.
 """
 from .api import (  # noqa: F401
+    WQ_ERR_ARG,
     WQ_ERR_TIMEOUT,
     WQ_ERR_UNSUPPORTED,
     WQ_LAYOUT_B200_V1,
@@ -15,6 +16,7 @@ from .api import (  # noqa: F401
     dequant_q4k,
     gemv_bf16,
     gemv_int4_blockwise,
+    gemv_int4_swiglu,
     gemv_q4k,
     gemv_q4k_dsc,
     last_error,
@@ -24,8 +26,10 @@ from .api import (  # noqa: F401
     wq_device_status,
     wq_int4_bytes,
     wq_int4_codes_bytes,
+    wq_int4_gate_up_packed_bytes,
     wq_int4_packed_bytes,
     wq_repack_int4,
+    wq_repack_int4_gate_up,
     wq_layout_version,
     wq_q4k_bytes,
     wq_q4k_dsc_bytes,

@@ -11,7 +11,7 @@ import ctypes
 
 import numpy as np
 
-from ._lib import (WQ_ERR_TIMEOUT, WQ_ERR_UNSUPPORTED, WQ_LAYOUT_B200_V1, WQ_LAYOUT_CANONICAL, WQError,  # noqa: F401
+from ._lib import (WQ_ERR_ARG, WQ_ERR_TIMEOUT, WQ_ERR_UNSUPPORTED, WQ_LAYOUT_B200_V1, WQ_LAYOUT_CANONICAL, WQError,  # noqa: F401
                    _check, last_error, last_kernel, lib)
 
 
@@ -50,6 +50,22 @@ def gemv_q4k_dsc(x, w_q4k, w_dsc, y, M, N, K, layout=WQ_LAYOUT_CANONICAL, stream
 
 def gemv_bf16(x, w, y, M, N, K, stream=None):
     _check(lib().gemv_bf16(_ptr(x), _ptr(w), _ptr(y), M, N, K, _stream(stream)), "gemv_bf16")
+
+
+def gemv_int4_swiglu(x, w_gate_up, y, M, N, K, block_size, layout=WQ_LAYOUT_B200_V1, stream=None):
+    _check(lib().gemv_int4_swiglu(_ptr(x), _ptr(w_gate_up), _ptr(y), M, N, K, block_size, layout, _stream(stream)),
+           "gemv_int4_swiglu")
+
+
+def wq_int4_gate_up_packed_bytes(N, K, block_size, layout=WQ_LAYOUT_B200_V1) -> int:
+    return int(lib().wq_int4_gate_up_packed_bytes(N, K, block_size, layout))
+
+
+def wq_repack_int4_gate_up(w_gate, scales_gate, zeros_gate, w_up, scales_up, zeros_up, w_out, N, K, block_size,
+                           to_layout=WQ_LAYOUT_B200_V1, stream=None):
+    _check(lib().wq_repack_int4_gate_up(_ptr(w_gate), _ptr(scales_gate), _ptr(zeros_gate), _ptr(w_up),
+                                        _ptr(scales_up), _ptr(zeros_up), _ptr(w_out), N, K, block_size, to_layout,
+                                        _stream(stream)), "wq_repack_int4_gate_up")
 
 
 def dequant_int4_blockwise(w_packed, scales, zeros, w_out, N, K, block_size, layout=WQ_LAYOUT_CANONICAL,

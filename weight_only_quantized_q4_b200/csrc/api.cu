@@ -13,14 +13,17 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/wq.h"
 #include "gemv_cc.cuh"
 #include "gemv_simple.cuh"
 #include "gemv_tc.cuh"
 #include "gemv_v1.cuh"
+#include "gemv_v1k.cuh"
 #include "gemm_tc5.cuh"
 #include "wq_host.h"
 
@@ -753,6 +756,184 @@ int launch_v1(const V1Plan& plan, cudaStream_t st) {
   return launch_check("gemv_v1 launch");
 }
 
+// ---------------------------------------------------------------------------
+// Split-band workspace: counters and partial sums of bands cut by CTA
+// boundaries (stream-K kernels).  One per (device, stream), allocated and
+// zeroed at the first such call on that stream; the kernels leave every
+// counter at zero when they finish.  Calls on one stream are ordered (the
+// kernels touch the workspace only after waiting for the previous kernel);
+// separate streams have separate workspaces.
+// ---------------------------------------------------------------------------
+constexpr long long kWsMaxBands = 65536;   // rows up to 1,048,576
+constexpr long long kWsMaxCtas = 1024;
+// partials: [CTA][first / last band][gate, up][16 rows][8 batch rows] fp32
+constexpr size_t kWsBytes = static_cast<size_t>(kWsMaxBands * 4 + kWsMaxCtas * 2 * 2 * 128 * 4);
+
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, void*> g_ws;
+
+int split_workspace(cudaStream_t st, int** counters, float** partials) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  auto it = g_ws.find({dev, st});
+  void* ptr = nullptr;
+  if (it != g_ws.end()) {
+    ptr = it->second;
+  } else {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone)
+      return fail(WQ_ERR_CUDA,
+                  "the first decode call on a stream sets up that stream's split-band workspace and cannot be "
+                  "captured: make one call on this stream before capturing a CUDA graph");
+    if ((e = cudaMalloc(&ptr, kWsBytes)) != cudaSuccess)
+      return fail(WQ_ERR_CUDA, std::string("workspace cudaMalloc: ") + cudaGetErrorString(e));
+    if ((e = cudaMemset(ptr, 0, kWsBytes)) != cudaSuccess)
+      return fail(WQ_ERR_CUDA, std::string("workspace cudaMemset: ") + cudaGetErrorString(e));
+    g_ws[{dev, st}] = ptr;
+  }
+  *counters = static_cast<int*>(ptr);
+  *partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ptr) + kWsMaxBands * 4);
+  return WQ_OK;
+}
+
+// Zero every split-band workspace of the current device (after a kernel gave
+// up, its counters may not have been reset).
+int reset_workspaces() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  for (auto& kv : g_ws)
+    if (kv.first.first == dev && cudaMemset(kv.second, 0, kWsBytes) != cudaSuccess)
+      return fail(WQ_ERR_CUDA, "workspace reset failed");
+  return WQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// B200_V1 int4 GEMV, stream-K: planner and launcher
+// ---------------------------------------------------------------------------
+struct V1KPlan {
+  V1KParams p;
+  int grid = 0, threads = 0, smem = 0;
+  Fmt fmt = Fmt::Int4;
+  int mp2 = 8;
+  bool dual = false;
+};
+
+using V1KKernel = void (*)(const V1KParams);
+
+V1KKernel v1k_kernel(Fmt f, int mp2, bool dual) {
+  if (f == Fmt::Int4) return dual ? &gemv_v1k_kernel<Fmt::Int4, 8, true> : &gemv_v1k_kernel<Fmt::Int4, 8>;
+  switch (mp2) {
+    case 1: return &gemv_v1k_kernel<Fmt::Q4K, 1>;
+    case 2: return &gemv_v1k_kernel<Fmt::Q4K, 2>;
+    case 4: return &gemv_v1k_kernel<Fmt::Q4K, 4>;
+    default: return &gemv_v1k_kernel<Fmt::Q4K, 8>;
+  }
+}
+
+constexpr int kV1KXBudget = 120 * 1024;  // resident activations per CTA
+
+bool plan_v1k(Fmt f, int M, int N, int K, int block_size, int sms, V1KPlan* out, bool dual = false) {
+  if (M < 1 || M > 8) return false;
+  if (dual && f != Fmt::Int4) return false;
+  if (f == Fmt::Int4 && (K % 128 || block_size < 128)) return false;
+  if (f == Fmt::Q4K && K % 256) return false;
+  if (f != Fmt::Int4 && f != Fmt::Q4K) return false;
+  const bool q4k = f == Fmt::Q4K;
+  const char* w_env = std::getenv("WQ_V1K_W");       // consumer warps (tuning)
+  const char* c_env = std::getenv("WQ_V1K_CTAS");    // CTAs per SM (tuning)
+  const char* st_env = std::getenv("WQ_V1K_STAGE");  // tiles per stage (tuning)
+  const char* ns_env = std::getenv("WQ_V1K_NS");     // ring depth cap (tuning)
+  const char* pf_env = std::getenv("WQ_V1K_PFKB");   // KB prefetched into L2 before the wait (tuning)
+  const char* r_env = std::getenv("WQ_V1K_RES");     // CTAs each SM must be able to hold (tuning)
+  V1KParams& p = out->p;
+  const int W = w_env ? std::max(1, std::min(kV1KMaxWarps - 2, std::atoi(w_env))) : 16;
+  const int cps = c_env ? std::max(1, std::min(4, std::atoi(c_env))) : 1;
+  // shared memory is sized so that `res` CTAs fit on an SM: with res > cps the
+  // next call's CTAs are resident while this call runs (and prefetch into L2)
+  const int res = std::max(cps, r_env ? std::max(1, std::min(4, std::atoi(r_env))) : cps);
+  const int stage_tiles = st_env ? std::max(1, std::atoi(st_env)) : 16;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_bands = (N + 15) / 16;
+  if (p.n_bands > kWsMaxBands) return false;
+  p.tpb = q4k ? K / 256 : K / 128;
+  p.T = static_cast<long long>(p.n_bands) * p.tpb;
+  p.tb = q4k ? kQ4KV1TileBytes : int4_v1_tile_bytes(block_size) * (dual ? 2 : 1);
+  out->fmt = f;
+  out->dual = dual;
+  const int nsum = dual ? 2 : 1;
+  int mp2 = 1;
+  while (mp2 < M) mp2 *= 2;
+  out->mp2 = mp2;
+  p.W = W;
+  p.tps = W * std::max(1, stage_tiles / W);  // a multiple of W: every warp's tile sequence runs on across stages
+  p.stage_bytes = p.tps * p.tb;
+  p.Mp = (M + 1) & ~1;
+  p.pf_bytes = (pf_env ? std::max(0, std::atoi(pf_env)) : 96) * 1024;
+  const long long x_bytes = 2ll * M * K;
+  if (x_bytes > kV1KXBudget) return false;
+  const long long xs_bytes = (q4k ? 256ll : 32ll) * p.tpb;  // Σx table: 8 floats per k-unit
+  const long long fixed = round16(x_bytes) + 256 + round16(xs_bytes) + round16(2ll * nsum * W * 16 * p.Mp * 4);
+  const long long room = kSmemPerSm / res - 1024 - fixed - (2ll * 16 * 8 + 8 + 16);
+  const int ns_cap = ns_env ? std::max(2, std::atoi(ns_env)) : 16;
+  const int NS = static_cast<int>(std::min<long long>(ns_cap, room / p.stage_bytes));
+  if (NS < 2) return false;
+  p.NS = NS;
+  long long off = static_cast<long long>(NS) * p.stage_bytes;
+  p.off_x = static_cast<int>(off);
+  off += round16(x_bytes);
+  p.off_zero = static_cast<int>(off);
+  off += 256;
+  p.off_xs = static_cast<int>(off);
+  off += round16(xs_bytes);
+  p.off_red = static_cast<int>(off);
+  off += round16(2ll * nsum * W * 16 * p.Mp * 4);
+  p.off_bar = static_cast<int>(off);
+  off += 2ll * NS * 8 + 8 + 16;
+  out->smem = static_cast<int>(off);
+  out->threads = (W + 2) * 32;
+  out->grid = static_cast<int>(std::min<long long>(std::min<long long>(sms * cps, p.T), kWsMaxCtas));
+  return true;
+}
+
+int launch_v1k(V1KPlan& plan, cudaStream_t st) {
+  static std::mutex mu;
+  static bool configured[6][64] = {};
+  const V1KKernel fn = v1k_kernel(plan.fmt, plan.mp2, plan.dual);
+  const int ki = plan.fmt == Fmt::Int4 ? (plan.dual ? 5 : 0)
+                                       : 1 + (plan.mp2 == 1 ? 0 : plan.mp2 == 2 ? 1 : plan.mp2 == 4 ? 2 : 3);
+  {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && !configured[ki][dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[ki][dev] = true;
+    }
+  }
+  int rc = split_workspace(st, &plan.p.counters, &plan.p.partials);
+  if (rc) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.grid, 1, 1);
+  cfg.blockDim = dim3(plan.threads, 1, 1);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, plan.p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemv_v1k launch: ") + cudaGetErrorString(e));
+  return launch_check("gemv_v1k launch");
+}
+
 // WQ_FORCE_KERNEL = "cc" | "tc" | "simple" pins the GEMV variant (A/B runs and
 // per-variant parity tests); unset means the default choice below.
 const char* forced_variant() {
@@ -925,7 +1106,7 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     // batches of 9 and more: one tcgen05 dequant-then-MMA launch (int4 canonical, q4_K)
     const char* force = forced_variant();
     const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0 && block_size >= 64) ||
-                        (F == Fmt::Q4K && K % 256 == 0);
+                        (F == Fmt::Q4K && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0);
     const bool want = force ? std::strcmp(force, "tc5") == 0 : M >= 9;
     if (tc5_ok && want && aligned16(x)) {
       if constexpr (F == Fmt::Int4 || F == Fmt::Q4K) {
@@ -941,6 +1122,25 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     const void* xc = static_cast<const uint8_t*>(x) + static_cast<long long>(m0) * K * x_elt;
     void* yc = static_cast<uint8_t*>(y) + static_cast<long long>(m0) * N * 2;
     const char* force = forced_variant();
+    if constexpr (F == Fmt::Q4K) {
+      if (layout == WQ_LAYOUT_B200_V1) {
+        // B200_V1 q4_K: the stream-K band kernel, or the scalar kernel (which
+        // reads every layout) when the activations do not fit or it is forced
+        V1KPlan kplan;
+        const bool want_v1k = force ? std::strcmp(force, "v1k") == 0 : true;
+        if (want_v1k && aligned16(xc) && plan_v1k(Fmt::Q4K, mc, N, K, 0, di.sms, &kplan)) {
+          kplan.p.x = xc;
+          kplan.p.w = w;
+          kplan.p.y = yc;
+          rc = launch_v1k(kplan, st);
+          if (rc) return rc;
+          char buf[64];
+          std::snprintf(buf, sizeof(buf), "%s.gemv.v1k.m%d.g%d%s", fmt_name, mc, kplan.grid, M > 8 ? ".chunked" : "");
+          label = buf;
+          continue;
+        }
+      }
+    }
     if constexpr (F == Fmt::Int4) {
       V1RPlan rplan;
       // (the register-streaming kernel measured slower than the bulk-copy ring
@@ -954,6 +1154,20 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
         if (rc) return rc;
         char buf[64];
         std::snprintf(buf, sizeof(buf), "%s.gemv.v1r.m%d.p%d%s", fmt_name, mc, rplan.P, M > 8 ? ".chunked" : "");
+        label = buf;
+        continue;
+      }
+      V1KPlan kplan;
+      const bool want_v1k = force ? std::strcmp(force, "v1k") == 0 : true;
+      if (want_v1k && layout == WQ_LAYOUT_B200_V1 && aligned16(xc) &&
+          plan_v1k(Fmt::Int4, mc, N, K, block_size, di.sms, &kplan)) {
+        kplan.p.x = xc;
+        kplan.p.w = w;
+        kplan.p.y = yc;
+        rc = launch_v1k(kplan, st);
+        if (rc) return rc;
+        char buf[64];
+        std::snprintf(buf, sizeof(buf), "%s.gemv.v1k.m%d.g%d%s", fmt_name, mc, kplan.grid, M > 8 ? ".chunked" : "");
         label = buf;
         continue;
       }
@@ -975,7 +1189,8 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     const bool want_tc = force ? std::strcmp(force, "tc") == 0 : true;
     const bool want_cc = force ? std::strcmp(force, "cc") == 0 : true;
     TCPlan tplan;
-    if (want_tc && fast_ok && aligned16(xc) &&
+    const bool tc_layout_ok = layout == WQ_LAYOUT_CANONICAL || F == Fmt::Int4;  // q4_K B200_V1: v1k / scalar only
+    if (want_tc && fast_ok && tc_layout_ok && aligned16(xc) &&
         plan_tc(F, mc, N, K, row_bytes, nb, zb, block_size, layout, di.sms, &tplan)) {
       tplan.p.x = xc;
       tplan.p.w = w;
@@ -1092,14 +1307,15 @@ int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* sca
 int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K, int layout, void* stream) {
   int rc = check_dims(M, N, K);
   if (rc) return rc;
-  if (layout != WQ_LAYOUT_CANONICAL) return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
+  if (layout != WQ_LAYOUT_CANONICAL && layout != WQ_LAYOUT_B200_V1)
+    return fail(WQ_ERR_LAYOUT, "unknown q4_K layout version");
   if (K % 256) return fail(WQ_ERR_ARG, "gemv_q4k: K must be a multiple of 256");
   if (!x_f16 || !w_q4k || !y_f16) return fail(WQ_ERR_ARG, "gemv_q4k: null pointer");
   if (!aligned16(x_f16) || !aligned16(w_q4k) || !aligned16(y_f16))
     return fail(WQ_ERR_ALIGN, "gemv_q4k: device pointers must be 16-byte aligned");
   return run_gemv<Fmt::Q4K>("q4k", x_f16, static_cast<const uint8_t*>(w_q4k), nullptr, nullptr, nullptr, y_f16, M,
                             N, K, static_cast<long long>(K / 256) * 144, 0, 0, 0, true,
-                            static_cast<cudaStream_t>(stream));
+                            static_cast<cudaStream_t>(stream), layout);
 }
 
 int gemv_q4k_dsc(const void* x_f16, const void* w_q4k, const void* w_dsc, void* y_f16, int M, int N, int K,
@@ -1213,6 +1429,75 @@ int wq_repack_int4(const void* w_canonical, const void* scales_f16, const void* 
   return WQ_OK;
 }
 
+int wq_repack_int4_gate_up(const void* w_gate, const void* scales_gate, const void* zeros_gate, const void* w_up,
+                           const void* scales_up, const void* zeros_up, void* w_out, int N, int K, int block_size,
+                           int to_layout, void* stream) {
+  if (N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "wq_repack_int4_gate_up: need N, K > 0");
+  if (!w_gate || !scales_gate || !w_up || !scales_up || !w_out)
+    return fail(WQ_ERR_ARG, "wq_repack_int4_gate_up: null pointer");
+  if (to_layout != WQ_LAYOUT_B200_V1)
+    return fail(WQ_ERR_LAYOUT, "wq_repack_int4_gate_up: target layout must be B200_V1");
+  if (block_size < 128 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size)
+    return fail(WQ_ERR_ARG, "wq_repack_int4_gate_up: needs block_size 128 or 256 and K % 128 == 0");
+  if (!aligned16(w_gate) || !aligned16(scales_gate) || (zeros_gate && !aligned16(zeros_gate)) || !aligned16(w_up) ||
+      !aligned16(scales_up) || (zeros_up && !aligned16(zeros_up)) || !aligned16(w_out))
+    return fail(WQ_ERR_ALIGN, "wq_repack_int4_gate_up: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const long long tiles = static_cast<long long>((N + 15) / 16) * (K / 128);
+  const int g1 = static_cast<int>(std::min<long long>((tiles * 64 + 255) / 256, di.sms * 32ll));
+  const int g2 = static_cast<int>(std::min<long long>((tiles * 8 + 255) / 256, di.sms * 32ll));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const void* ws[2] = {w_gate, w_up};
+  const void* ss[2] = {scales_gate, scales_up};
+  const void* zs[2] = {zeros_gate, zeros_up};
+  for (int h = 0; h < 2; ++h) {  // gate tiles at even tile slots, up tiles at odd ones
+    repack_int4_v1_codes_kernel<<<g1, 256, 0, st>>>(static_cast<const uint8_t*>(ws[h]), static_cast<uint8_t*>(w_out), N,
+                                                    K, block_size, 2, h);
+    if ((rc = launch_check("repack_int4_gate_up codes launch"))) return rc;
+    repack_int4_v1_meta_kernel<<<g2, 256, 0, st>>>(static_cast<const uint8_t*>(ss[h]), static_cast<const uint8_t*>(zs[h]),
+                                                   static_cast<uint8_t*>(w_out), N, K, block_size, 2, h);
+    if ((rc = launch_check("repack_int4_gate_up meta launch"))) return rc;
+  }
+  set_last_kernel("int4.repack.gate_up.v1");
+  return WQ_OK;
+}
+
+int gemv_int4_swiglu(const void* x_f16, const void* w_gate_up, void* y_f16, int M, int N, int K, int block_size,
+                     int layout, void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (layout != WQ_LAYOUT_B200_V1)
+    return fail(WQ_ERR_LAYOUT, "gemv_int4_swiglu: the fused gate-up stream exists in the B200_V1 layout only");
+  if (block_size < 128 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size)
+    return fail(WQ_ERR_ARG, "gemv_int4_swiglu: needs block_size 128 or 256 and K % 128 == 0");
+  if (!x_f16 || !w_gate_up || !y_f16) return fail(WQ_ERR_ARG, "gemv_int4_swiglu: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_gate_up) || !aligned16(y_f16))
+    return fail(WQ_ERR_ALIGN, "gemv_int4_swiglu: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  // rows of x per launch: at most 8, and few enough that they fit in shared memory
+  const int mc_max = std::max(1, std::min(8, kV1KXBudget / (2 * K)));
+  if (2 * K > kV1KXBudget) return fail(WQ_ERR_UNSUPPORTED, "gemv_int4_swiglu: K too large for resident activations");
+  std::string label;
+  for (int m0 = 0; m0 < M; m0 += mc_max) {
+    const int mc = std::min(mc_max, M - m0);
+    V1KPlan plan;
+    if (!plan_v1k(Fmt::Int4, mc, N, K, block_size, di.sms, &plan, true))
+      return fail(WQ_ERR_UNSUPPORTED, "gemv_int4_swiglu: no launch plan for this shape");
+    plan.p.x = static_cast<const uint8_t*>(x_f16) + static_cast<long long>(m0) * K * 2;
+    plan.p.w = static_cast<const uint8_t*>(w_gate_up);
+    plan.p.y = static_cast<uint8_t*>(y_f16) + static_cast<long long>(m0) * N * 2;
+    if ((rc = launch_v1k(plan, static_cast<cudaStream_t>(stream)))) return rc;
+    char buf[64];
+    std::snprintf(buf, sizeof(buf), "int4.swiglu.v1k.m%d.g%d%s", mc, plan.grid, M > mc_max ? ".chunked" : "");
+    label = buf;
+  }
+  set_last_kernel(label);
+  return WQ_OK;
+}
+
 int wq_repack_q4k(const void* w_q4k, void* w_out, int N, int K, int to_layout, void* stream) {
   if (N <= 0 || K <= 0 || K % 256) return fail(WQ_ERR_ARG, "wq_repack_q4k: need N > 0 and K % 256 == 0");
   if (!w_q4k || !w_out) return fail(WQ_ERR_ARG, "wq_repack_q4k: null pointer");
@@ -1281,7 +1566,10 @@ int wq_device_status(void) {
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("read device error word: ") + cudaGetErrorString(e));
   e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("clear device error word: ") + cudaGetErrorString(e));
-  if (v & kDevErrTimeout) return fail(WQ_ERR_TIMEOUT, "a bounded device-side wait expired");
+  if (v & kDevErrTimeout) {
+    reset_workspaces();  // a kernel that gave up may have left split-band counters set
+    return fail(WQ_ERR_TIMEOUT, "a bounded device-side wait expired");
+  }
   return WQ_OK;
 }
 

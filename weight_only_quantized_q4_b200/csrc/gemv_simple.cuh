@@ -295,8 +295,11 @@ __global__ void dequant_q4k_kernel(const uint8_t* w, const uint8_t* plane, float
 }
 
 // Canonical int4 -> B200_V1, codes: thread per 16-byte code chunk of a tile
-// (rows past N get zero codes).
-__global__ void repack_int4_v1_codes_kernel(const uint8_t* w, uint8_t* out, int N, int K, int bs) {
+// (rows past N get zero codes).  Tile i of the stream is written at tile slot
+// i·tile_mul + tile_add of `out` (1, 0 for a plain stream; 2, 0 / 2, 1 for the
+// gate / up halves of the fused gate-up stream).
+__global__ void repack_int4_v1_codes_kernel(const uint8_t* w, uint8_t* out, int N, int K, int bs, int tile_mul = 1,
+                                            int tile_add = 0) {
   const long long n_bands = (N + 15) / 16;
   const int tpb = K / 128;
   const int tb = int4_v1_tile_bytes(bs);
@@ -321,7 +324,7 @@ __global__ void repack_int4_v1_codes_kernel(const uint8_t* w, uint8_t* out, int 
       for (int e = 0; e < 8; ++e) o |= ((cw >> (4 * e)) & 15u) << (4 * int4_v1_nibble_pos(e));
       v[j] = o;
     }
-    *reinterpret_cast<uint4*>(out + tile * tb + q * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<uint4*>(out + (tile * tile_mul + tile_add) * tb + q * 16) = make_uint4(v[0], v[1], v[2], v[3]);
   }
 }
 
@@ -329,7 +332,7 @@ __global__ void repack_int4_v1_codes_kernel(const uint8_t* w, uint8_t* out, int 
 // the two rows' fp16 scales and their shared zero-point byte (pads: scale 0,
 // zero-point 8); the 16-byte tail padding of a tile is zeroed by slot 0.
 __global__ void repack_int4_v1_meta_kernel(const uint8_t* scales, const uint8_t* zeros, uint8_t* out, int N, int K,
-                                           int bs) {
+                                           int bs, int tile_mul = 1, int tile_add = 0) {
   const long long n_bands = (N + 15) / 16;
   const int tpb = K / 128;
   const int bpt = int4_v1_bpt(bs);
@@ -345,7 +348,7 @@ __global__ void repack_int4_v1_meta_kernel(const uint8_t* scales, const uint8_t*
     const long long band = tile / tpb;
     const int s = static_cast<int>(tile - band * tpb);
     const int blk = (128 * s + bt * (bs < 128 ? bs : 0)) / bs;
-    uint8_t* tp = out + tile * tb;
+    uint8_t* tp = out + (tile * tile_mul + tile_add) * tb;
     uint32_t zbyte = 0;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {

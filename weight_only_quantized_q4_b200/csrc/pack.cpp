@@ -76,6 +76,11 @@ extern "C" size_t wq_int4_packed_bytes(int N, int K, int block_size, int layout)
   return static_cast<size_t>((N + 15) / 16) * (K / 128) * WQ_INT4_V1_TILE_BYTES(block_size);
 }
 
+extern "C" size_t wq_int4_gate_up_packed_bytes(int N, int K, int block_size, int layout) {
+  if (block_size < 128) return 0;
+  return 2 * wq_int4_packed_bytes(N, K, block_size, layout);
+}
+
 extern "C" size_t wq_q4k_packed_bytes(int N, int K, int layout) {
   if (N <= 0 || K <= 0 || K % 256 || layout != WQ_LAYOUT_B200_V1) return 0;
   return static_cast<size_t>((N + 15) / 16) * (K / 256) * WQ_Q4K_V1_TILE_BYTES;
