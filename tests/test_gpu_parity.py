@@ -236,18 +236,22 @@ def test_gemv_int4_v1_cluster_split(C, M, N, K, bs, zeros, monkeypatch):
 
 
 @gpu
+@pytest.mark.parametrize("zq", [0, 1])
 @pytest.mark.parametrize("ctas", [1, 4])
 @pytest.mark.parametrize("M", [1, 2, 3, 4])
 @pytest.mark.parametrize("N,K,bs,zeros", [(37, 2048, 128, True), (1000, 1536, 256, False), (300, 512, 128, True),
                                           (4100, 1024, 128, True), (16, 4096, 256, True), (5, 128, 128, True),
                                           (2368, 14336, 128, True)])
-def test_gemv_int4_v1_stream_k(ctas, M, N, K, bs, zeros, monkeypatch):
+def test_gemv_int4_v1_stream_k(zq, ctas, M, N, K, bs, zeros, monkeypatch):
     """The stream-K B200_V1 kernel: every CTA takes an equal run of tiles, so
     bands are cut between CTAs (a band over up to 16 CTAs when N is small)
     and finished by the fix-up through the split-band workspace.  The fix-up
     adds the pieces in CTA order: two calls in a row agree bit for bit, and
     so does a third call after other shapes have used the workspace."""
+    if ctas == 4 and 2 * M * K > 24 * 1024:
+        pytest.skip("four CTAs per SM leave no room for these resident activations")
     monkeypatch.setenv("WQ_FORCE_KERNEL", "v1k")
+    monkeypatch.setenv("WQ_V1K_ZQ", str(zq))
     monkeypatch.setenv("WQ_V1K_CTAS", str(ctas))
     monkeypatch.setenv("WQ_V1K_W", "16" if ctas == 1 else "4")  # four CTAs per SM leave room for 4 warps' stages
     c = Int4Case(M, N, K, bs, zeros, workload=25, layout=wq.WQ_LAYOUT_B200_V1)
@@ -374,6 +378,20 @@ def test_gemm_tcgen05_batched(M, fmt):
         W, x = c.W(), c.x
     assert ".gemm.tc5." in wq.last_kernel(), wq.last_kernel()
     check(y, W, x, f"tcgen05 {fmt} M={M}")
+
+
+@gpu
+@pytest.mark.parametrize("M", [9, 16, 33, 128])
+@pytest.mark.parametrize("N,K", [(300, 1536), (1536, 6912), (77, 136)])
+def test_gemm_tcgen05_bf16(M, N, K):
+    """bf16 batches of 9 and more run the tcgen05 kernel with the weights
+    TMA-loaded straight into the MMA's A slots (K = 136: a partial last 64-k
+    stage, zero-filled by the tensor-map bounds)."""
+    c = BF16Case(M, N, K, workload=30)
+    y = c.run()
+    assert ".gemm.tc5." in wq.last_kernel() and wq.last_kernel().startswith("bf16"), wq.last_kernel()
+    check(y, c.W(), c.X(), f"tcgen05 bf16 M={M} N={N} K={K}")
+    assert np.array_equal(y, c.run())
 
 
 @gpu

@@ -823,8 +823,17 @@ struct V1KPlan {
 
 using V1KKernel = void (*)(const V1KParams);
 
+// WQ_V1K_ZQ=1 selects the int4 tile with the zero-point inside the MMA operand (tuning)
+bool v1k_zq() {
+  const char* v = std::getenv("WQ_V1K_ZQ");
+  return v && std::atoi(v) != 0;
+}
+
 V1KKernel v1k_kernel(Fmt f, int mp2, bool dual) {
-  if (f == Fmt::Int4) return dual ? &gemv_v1k_kernel<Fmt::Int4, 8, true> : &gemv_v1k_kernel<Fmt::Int4, 8>;
+  if (f == Fmt::Int4) {
+    if (v1k_zq()) return dual ? &gemv_v1k_kernel<Fmt::Int4, 8, true, true> : &gemv_v1k_kernel<Fmt::Int4, 8, false, true>;
+    return dual ? &gemv_v1k_kernel<Fmt::Int4, 8, true> : &gemv_v1k_kernel<Fmt::Int4, 8>;
+  }
   switch (mp2) {
     case 1: return &gemv_v1k_kernel<Fmt::Q4K, 1>;
     case 2: return &gemv_v1k_kernel<Fmt::Q4K, 2>;
@@ -877,9 +886,15 @@ bool plan_v1k(Fmt f, int M, int N, int K, int block_size, int sms, V1KPlan* out,
   const long long x_bytes = 2ll * M * K;
   if (x_bytes > kV1KXBudget) return false;
   const long long xs_bytes = (q4k ? 256ll : 32ll) * p.tpb;  // Σx table: 8 floats per k-unit
-  const long long fixed = round16(x_bytes) + 256 + round16(xs_bytes) + round16(2ll * nsum * W * 16 * p.Mp * 4);
+  const long long fixed =
+      round16(x_bytes) + 256 + round16(xs_bytes) + round16(1ll * kRedSlots * nsum * W * 16 * p.Mp * 4);
   const long long room = kSmemPerSm / res - 1024 - fixed - (2ll * 16 * 8 + 8 + 16);
   const int ns_cap = ns_env ? std::max(2, std::atoi(ns_env)) : 16;
+  // smaller stages (still a multiple of W tiles) until at least two fit
+  while (room / p.stage_bytes < 2 && p.tps > W) {
+    p.tps = W * std::max(1, p.tps / W / 2);
+    p.stage_bytes = p.tps * p.tb;
+  }
   const int NS = static_cast<int>(std::min<long long>(ns_cap, room / p.stage_bytes));
   if (NS < 2) return false;
   p.NS = NS;
@@ -891,7 +906,7 @@ bool plan_v1k(Fmt f, int M, int N, int K, int block_size, int sms, V1KPlan* out,
   p.off_xs = static_cast<int>(off);
   off += round16(xs_bytes);
   p.off_red = static_cast<int>(off);
-  off += round16(2ll * nsum * W * 16 * p.Mp * 4);
+  off += round16(1ll * kRedSlots * nsum * W * 16 * p.Mp * 4);
   p.off_bar = static_cast<int>(off);
   off += 2ll * NS * 8 + 8 + 16;
   out->smem = static_cast<int>(off);
@@ -902,10 +917,10 @@ bool plan_v1k(Fmt f, int M, int N, int K, int block_size, int sms, V1KPlan* out,
 
 int launch_v1k(V1KPlan& plan, cudaStream_t st) {
   static std::mutex mu;
-  static bool configured[6][64] = {};
+  static bool configured[8][64] = {};
   const V1KKernel fn = v1k_kernel(plan.fmt, plan.mp2, plan.dual);
-  const int ki = plan.fmt == Fmt::Int4 ? (plan.dual ? 5 : 0)
-                                       : 1 + (plan.mp2 == 1 ? 0 : plan.mp2 == 2 ? 1 : plan.mp2 == 4 ? 2 : 3);
+  const int ki = plan.fmt == Fmt::Int4 ? 4 + (plan.dual ? 2 : 0) + (v1k_zq() ? 1 : 0)
+                                       : (plan.mp2 == 1 ? 0 : plan.mp2 == 2 ? 1 : plan.mp2 == 4 ? 2 : 3);
   {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1018,10 +1033,10 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   const int x_slot = (p.BN * 128 + 1023) / 1024 * 1024;
   // raw slots of 256 k: int4 128 B per row, q4_K one 144-byte super-block per row
   // (256-byte int4 rows measured no faster on B200)
-  p.spr = 4;
+  p.spr = F == Fmt::BF16 ? 1 : 4;
   p.raw_pitch = F == Fmt::Int4 ? 128 : 144;
-  p.raw_bytes = 128 * p.raw_pitch;
-  p.NR = 3;
+  p.raw_bytes = F == Fmt::BF16 ? 0 : 128 * p.raw_pitch;  // bf16 weights go straight into the A slots
+  p.NR = F == Fmt::BF16 ? 0 : 3;
   const int budget = kSmemPerSm - 1024 - 1024;
   p.NX = std::max(2, std::min(8, (budget - kTc5NA * 16384 - p.NR * p.raw_bytes) / x_slot));
   p.off_x = kTc5NA * 16384;
@@ -1032,7 +1047,7 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   // Split K over a cluster of S CTAs (one CTA per SM) until the CTAs fill the
   // SMs; every CTA keeps a whole number of 256-k raw slots.
   const int n_tiles = (N + 127) / 128, m_tiles = (M + p.BN - 1) / p.BN;
-  const int nst = K / 64;
+  const int nst = (K + 63) / 64;  // bf16: a partial last stage reads zeros past K (TMA bounds fill)
   int S = 1;
   while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nst % (2 * p.spr * S) == 0) S *= 2;
   if (const char* s_env = std::getenv("WQ_TC5_S")) {  // tests and tuning
@@ -1050,15 +1065,18 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   int rc;
   if constexpr (F == Fmt::Int4)
     rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else if constexpr (F == Fmt::BF16)
+    rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, 2ull * K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   else
     rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (K / 256) * 144ull, N, (K / 256) * 144ull, 144, 128,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
-  rc = encode_2d(&p.tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, 2ull * K, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  rc = encode_2d(&p.tmap_x, F == Fmt::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K,
+                 M, 2ull * K, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   static std::mutex mu;
-  static bool configured[2][64] = {};
-  const int fi = F == Fmt::Int4 ? 0 : 1;
+  static bool configured[3][64] = {};
+  const int fi = F == Fmt::Int4 ? 0 : F == Fmt::Q4K ? 1 : 2;
   {
     std::lock_guard<std::mutex> lk(mu);
     int dev = 0;
@@ -1087,7 +1105,8 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   rc = launch_check("gemm_tc5 launch");
   if (rc) return rc;
   char buf[64];
-  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.bn%d.s%d", F == Fmt::Int4 ? "int4" : "q4k", p.BN, S);
+  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.bn%d.s%d", F == Fmt::Int4 ? "int4" : F == Fmt::Q4K ? "q4k" : "bf16",
+                p.BN, S);
   *label = buf;
   return WQ_OK;
 }
@@ -1106,10 +1125,11 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     // batches of 9 and more: one tcgen05 dequant-then-MMA launch (int4 canonical, q4_K)
     const char* force = forced_variant();
     const bool tc5_ok = (F == Fmt::Int4 && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0 && block_size >= 64) ||
-                        (F == Fmt::Q4K && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0);
+                        (F == Fmt::Q4K && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0) ||
+                        (F == Fmt::BF16 && K % 8 == 0 && aligned16(w));
     const bool want = force ? std::strcmp(force, "tc5") == 0 : M >= 9;
     if (tc5_ok && want && aligned16(x)) {
-      if constexpr (F == Fmt::Int4 || F == Fmt::Q4K) {
+      if constexpr (F == Fmt::Int4 || F == Fmt::Q4K || F == Fmt::BF16) {
         rc = launch_tc5<F>(x, w, scales, zeros, y, M, N, K, nb, zb, block_size, di.sms, st, &label);
         if (rc) return rc;
         set_last_kernel(label);

@@ -61,9 +61,10 @@ __device__ __forceinline__ uint64_t umma_smem_desc_sw128(uint32_t saddr) {
          (2ull << 61);
 }
 
-// kind::f16 instruction descriptor: D f32, A/B f16, both K-major, N = bn, M = 128.
-__host__ __device__ __forceinline__ uint32_t umma_idesc_f16(int bn) {
-  return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+// kind::f16 instruction descriptor: D f32, A/B f16 (or both bf16), both K-major, N = bn, M = 128.
+__host__ __device__ __forceinline__ uint32_t umma_idesc_f16(int bn, bool bf16 = false) {
+  return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | (static_cast<uint32_t>(bn >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
       mbar_init(&x_empty[i], 1);  // tcgen05.commit
     }
     for (int i = 0; i < kTc5NA; ++i) {
-      mbar_init(&a_full[i], 8);
+      mbar_init(&a_full[i], F == Fmt::BF16 ? 1 : 8);  // bf16: the producer's TMA fills A directly
       mbar_init(&a_empty[i], 1);
     }
     mbar_init(done, 1);
@@ -281,7 +282,16 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
       int rs = 0, ru = 0, xs = 0, xu = 0;  // slot index and use count of each ring
       for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
         const int gs = s_begin + ls;
-        if ((ls & (p.spr - 1)) == 0) {
+        if constexpr (F == Fmt::BF16) {
+          // bf16 weights are the MMA operand as stored: 128 rows × 64 k straight into an A slot
+          const int a = ls & (kTc5NA - 1), au = ls / kTc5NA;
+          if (au > 0 && !mbar_wait_bounded(&a_empty[a], static_cast<uint32_t>((au - 1) & 1))) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&a_full[a], 16384u);
+          tma_load_2d(smem + a * 16384, &p.tmap_w, gs * 64, n0, &a_full[a]);
+        } else if ((ls & (p.spr - 1)) == 0) {
           if (ru > 0 && !mbar_wait_bounded(&raw_empty[rs], static_cast<uint32_t>((ru - 1) & 1))) {
             *abort_flag = 1;
             break;
@@ -309,7 +319,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_f16(p.BN);
+      const uint32_t idesc = umma_idesc_f16(p.BN, F == Fmt::BF16);
       int xs = 0, xu = 0;
       for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
         const int a = ls & (kTc5NA - 1), au = ls / kTc5NA;
@@ -346,7 +356,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
       for (int i = 0; i < kTc5SzAhead; ++i) szr[i] = i < nks ? fetch_sz(p, row, s_begin + i) : 0u;
     }
     int rs = 0, ru = 0;
-    for (int s0 = 0; s0 < nks; s0 += kTc5SzAhead) {
+    for (int s0 = 0; s0 < (F == Fmt::BF16 ? 0 : nks); s0 += kTc5SzAhead) {
 #pragma unroll
       for (int i = 0; i < kTc5SzAhead; ++i) {
         const int ls = s0 + i;
@@ -368,7 +378,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
         const uint8_t* rrow = smem + p.off_raw + rs * p.raw_bytes + rl * p.raw_pitch;
         const uint8_t* codes = F == Fmt::Int4 ? rrow + 32 * (ls & (p.spr - 1)) : rrow + 16 + 32 * (ls & 3);
         uint32_t o[16];
-        dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, o);
+        if constexpr (F != Fmt::BF16) dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, o);
         uint8_t* at = smem + a * 16384;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -397,7 +407,13 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
   const int cols_per = split_cols ? p.BN / 2 : p.BN;
   const int c_begin = split_cols ? ch * cols_per : 0;
   const bool reads = warp < 8 && (split_cols || ch == 0);
-  __half* y = reinterpret_cast<__half*>(p.y);
+  // fp16 y (int4, q4_K) or bf16 y (bf16 weights and activations)
+  auto store_y = [&](long long o, float v) {
+    if constexpr (F == Fmt::BF16)
+      reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
+    else
+      reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(v);
+  };
   // the two accumulator tiles of a 16-column group, added (fixed order)
   auto acc16 = [&](int c0, float (&v)[16]) {
     uint32_t r0[16], r1[16];
@@ -415,7 +431,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = m0 + c0 + j;
-          if (m < p.M && yrow < p.N) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(v[j]);
+          if (m < p.M && yrow < p.N) store_y(static_cast<long long>(m) * p.N + yrow, v[j]);
         }
       }
     }
@@ -440,7 +456,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
       float sum = 0.f;
       for (int q = 0; q < p.S; ++q) sum += tc5_dsmem_ld(acc + rr * p.BN + c, static_cast<uint32_t>(q));
       const int m = m0 + c, yrow = n0 + rr;
-      if (m < p.M && yrow < p.N && !*abort_flag) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(sum);
+      if (m < p.M && yrow < p.N && !*abort_flag) store_y(static_cast<long long>(m) * p.N + yrow, sum);
     }
     tc5_cluster_sync();
   }

@@ -49,7 +49,7 @@ struct V1KParams {
   int off_x;         // activations [M][K] fp16
   int off_zero;      // 256 zero bytes
   int off_xs;        // Σx table [k-units][8] fp32 (int4: per tile, ×2^-24; q4_K: per 32-k chunk)
-  int off_red;       // [2][kNS][W][16][Mp] fp32 warp partials
+  int off_red;       // [kRedSlots][kNS][W][16][Mp] fp32 warp partials
   int off_bar;       // full[NS], empty[NS], x barrier, abort word
 };
 
@@ -102,6 +102,26 @@ __device__ __forceinline__ void q4k_tile_fma(const uint8_t* tp, const uint8_t* x
     v1d::mma16816(dl[c % MP2], a0 & 0x000F000Fu, a1 & 0x000F000Fu, a08 & 0x000F000Fu, a18 & 0x000F000Fu, xv.x, xv.z);
     v1d::mma16816(dh[c % MP2], a0 & 0x00F000F0u, a1 & 0x00F000F0u, a08 & 0x00F000F0u, a18 & 0x00F000F0u, xv.y, xv.w);
   }
+  // At MP2 = 1 the chunk sums come from the activations themselves: lane
+  // (g, t) holds 8 of the 32 of chunk g; four lanes add up the chunk, and the
+  // lane receiving chunk c reads the sum from lane 4c.
+  float xown[2] = {0.f, 0.f};
+  if constexpr (MP2 == 1) {
+    float ps = 0.f;
+    if (xrow) {
+      const uint4 xo = *reinterpret_cast<const uint4*>(xt + 64 * g);
+      const uint32_t u[4] = {xo.x, xo.y, xo.z, xo.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[e]));
+        ps += f.x + f.y;
+      }
+    }
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+    xown[0] = __shfl_sync(0xffffffffu, ps, 8 * t);      // chunk 2t
+    xown[1] = __shfl_sync(0xffffffffu, ps, 8 * t + 4);  // chunk 2t + 1
+  }
   // coefficients of the chunks this lane receives, rows g and g + 8
   const uint32_t dd0 = *reinterpret_cast<const uint32_t*>(tp + 2048 + 4 * g);
   const uint32_t dd1 = *reinterpret_cast<const uint32_t*>(tp + 2048 + 4 * (g + 8));
@@ -117,13 +137,79 @@ __device__ __forceinline__ void q4k_tile_fma(const uint8_t* tp, const uint8_t* x
       const int hi = c & 1;
       const float sc0 = static_cast<float>((en0 >> (6 * hi)) & 63u), sc1 = static_cast<float>((en1 >> (6 * hi)) & 63u);
       const float mn0 = static_cast<float>((en0 >> (12 + 6 * hi)) & 63u), mn1 = static_cast<float>((en1 >> (12 + 6 * hi)) & 63u);
-      const float X = xc[c * 8 + m];
+      const float X = MP2 == 1 ? xown[e] : xc[c * 8 + m];
       // y += d·sc·Σqx − dmin·m·Σx  (codes ×2^-24 in the MMA, ×2^24 folded into d)
       y[e] = fmaf(d0 * sc0, fmaf(dh[S][e], 0.0625f, dl[S][e]), fmaf(-(m0 * mn0), X, y[e]));
       y[2 + e] = fmaf(d1 * sc1, fmaf(dh[S][2 + e], 0.0625f, dl[S][2 + e]), fmaf(-(m1 * mn1), X, y[2 + e]));
     }
   }
 }
+
+// int4 B200_V1 tile with the zero-point taken out of the MMA operand: a nibble
+// masked under the fp16 pattern of 1024 (low nibbles) or 64 (high nibbles) is
+// 1024 + q or 64 + q exactly; subtracting 1024 + z or 64 + z (one HSUB2 per
+// pair) leaves the exact integer q − z.  The MMA then forms Σ (q − z)·x
+// directly: no Σx table, no prologue, one fp32 FMA by the scale per output.
+__device__ __forceinline__ uint32_t v1k_lop3_or(uint32_t v, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(magic));  // (v & mask) | magic
+  return r;
+}
+__device__ __forceinline__ uint32_t v1k_hsub2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ void tile_fma_zq(const uint8_t* tp, const uint8_t* xt, int lane, int g, float (&y)[4]) {
+  const uint4 qa = *reinterpret_cast<const uint4*>(tp + lane * 16);
+  const uint4 qb = *reinterpret_cast<const uint4*>(tp + 512 + lane * 16);
+  uint4 xv[4];
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) xv[gi] = *reinterpret_cast<const uint4*>(xt + 64 * gi);
+  const uint16_t* sc = reinterpret_cast<const uint16_t*>(tp + 1024);
+  const uint32_t sb0 = sc[g], sb1 = sc[g + 8];
+  const uint2 zz = *reinterpret_cast<const uint2*>(tp + 1056);
+  const uint32_t z0 = (zz.x >> (4 * g)) & 15u, z1 = (zz.y >> (4 * g)) & 15u;
+  const uint32_t zl0 = (0x6400u | z0) * 0x00010001u, zl1 = (0x6400u | z1) * 0x00010001u;
+  const uint32_t zh0 = (0x5400u | (z0 << 4)) * 0x00010001u, zh1 = (0x5400u | (z1 << 4)) * 0x00010001u;
+  const uint32_t v0[4] = {qa.x, qa.z, qb.x, qb.z}, v1[4] = {qa.y, qa.w, qb.y, qb.w};
+  float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};  // two chains: even / odd 32-k groups
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) {
+    const uint32_t a0 = v0[gi], a1 = v1[gi], a08 = a0 >> 8, a18 = a1 >> 8;
+    float(&d)[4] = (gi & 1) ? db : da;
+    v1d::mma16816(d, v1k_hsub2(v1k_lop3_or(a0, 0x000F000Fu, 0x64006400u), zl0),
+                  v1k_hsub2(v1k_lop3_or(a1, 0x000F000Fu, 0x64006400u), zl1),
+                  v1k_hsub2(v1k_lop3_or(a08, 0x000F000Fu, 0x64006400u), zl0),
+                  v1k_hsub2(v1k_lop3_or(a18, 0x000F000Fu, 0x64006400u), zl1), xv[gi].x, xv[gi].z);
+    v1d::mma16816(d, v1k_hsub2(v1k_lop3_or(a0, 0x00F000F0u, 0x54005400u), zh0),
+                  v1k_hsub2(v1k_lop3_or(a1, 0x00F000F0u, 0x54005400u), zh1),
+                  v1k_hsub2(v1k_lop3_or(a08, 0x00F000F0u, 0x54005400u), zh0),
+                  v1k_hsub2(v1k_lop3_or(a18, 0x00F000F0u, 0x54005400u), zh1), xv[gi].y, xv[gi].w);
+  }
+  const float s0 = h16_to_f32(sb0), s1 = h16_to_f32(sb1);
+  y[0] = fmaf(s0, da[0] + db[0], y[0]);
+  y[1] = fmaf(s0, da[1] + db[1], y[1]);
+  y[2] = fmaf(s1, da[2] + db[2], y[2]);
+  y[3] = fmaf(s1, da[3] + db[3], y[3]);
+}
+
+// Split-band counters: one atomic with acquire-release semantics both
+// publishes this piece's partial sums (written by the warp before a
+// __syncwarp) and, for the last piece, makes the other pieces visible.
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Band partial slots between the consumer warps and the reducer: a ring of
+// kRedSlots, so a slow fix-up of one band does not hold the consumers back.
+constexpr int kRedSlots = 4;
+constexpr int kBarRedFull = 1;   // named barriers 1..4: slot s holds a band's warp partials
+constexpr int kBarRedFree = 5;   // named barriers 5..8: slot s is free again
+constexpr int kBarPrologue = 9;  // consumers only
 
 // CTA of tile t when CTA i owns [floor(i·T/G), floor((i+1)·T/G)).
 __device__ __forceinline__ int v1k_cta_of(long long t, long long T, int G) {
@@ -140,13 +226,16 @@ __device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.f + 
 // each tile of the stream is a gate tile followed by the up tile of the same
 // 16 rows and 128 k (the fused gate-up stream); the CTA keeps both sums and
 // writes y = silu(x·Wgᵀ)·(x·Wuᵀ).
-template <Fmt F, int MP2, bool DUAL = false>
+template <Fmt F, int MP2, bool DUAL = false, bool ZQ = false>
 __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1KParams p) {
   constexpr bool kQ4K = F == Fmt::Q4K;
+  // the Σx table is needed for the q4_K mins (MP2 > 1; at MP2 = 1 the tile forms its
+  // chunk sums itself) and for the int4 Σx zero-point term (unless ZQ)
+  constexpr bool kSumX = kQ4K ? MP2 > 1 : !ZQ;
   constexpr int kNS = DUAL ? 2 : 1;  // sums kept per output (gate and up for the fused stream)
   constexpr int kUnit = kQ4K ? 32 : 128;             // k per Σx entry (a q4_K chunk, an int4 tile)
   constexpr int kUnitsPerTile = kQ4K ? 8 : 1;
-  constexpr float kYScale = kQ4K ? 1.f : 16777216.f;  // int4 partials are in units of 2^-24
+  constexpr float kYScale = !kQ4K && !ZQ ? 16777216.f : 1.f;  // subnormal-code int4 partials are ×2^-24
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int W = p.W, G = gridDim.x, cta = blockIdx.x;
@@ -240,8 +329,8 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
     grid_wait_prior();  // y, the counters and the partials may be in use by the previous kernel
     __half* y = reinterpret_cast<__half*>(p.y);
     for (int bl = 0; bl < n_bl; ++bl) {
-      const int s = bl & 1;
-      v1d::bar_sync(v1d::kBarFull0 + s, nthr_all);
+      const int s = bl % kRedSlots;
+      v1d::bar_sync(kBarRedFull + s, nthr_all);
       const float* rs = red + s * red_slot;
       const int b = band_at(bl);
       const long long bt0 = static_cast<long long>(b) * p.tpb, bt1 = bt0 + p.tpb;
@@ -268,14 +357,12 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
       if (!whole) {
         // fix-up of a band cut by CTA boundaries: count this piece; the last
         // piece adds all pieces in CTA order and writes y
-        __threadfence();
         __syncwarp();
         int seen = 0;
-        if (lane == 0) seen = atomicAdd(&p.counters[b], 1);
+        if (lane == 0) seen = atom_add_acq_rel(&p.counters[b], 1);
         seen = __shfl_sync(0xffffffffu, seen, 0);
         const int c0 = v1k_cta_of(bt0, p.T, G), c1 = v1k_cta_of(bt1 - 1, p.T, G);
         if (seen == c1 - c0) {
-          __threadfence();
           for (int o = lane; o < 16 * p.M; o += 32) {
             const int row = o / p.M, n = o - row * p.M;
             float sum[kNS];
@@ -296,7 +383,7 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
           if (lane == 0) p.counters[b] = 0;
         }
       }
-      if (bl + 2 < n_bl) v1d::bar_arrive(v1d::kBarFree0 + s, nthr_all);
+      if (bl + kRedSlots < n_bl) v1d::bar_arrive(kBarRedFree + s, nthr_all);
     }
     return;
   }
@@ -317,7 +404,7 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
     // units.
     constexpr int kTpu = kUnit / 8;
     const int n_units = p.tpb * kUnitsPerTile;
-    const int items = n_units * p.M * kTpu;
+    const int items = kSumX ? n_units * p.M * kTpu : 0;
     const int rounds = (items + nthr - 1) / nthr;
     for (int r = 0; r < rounds; ++r) {
       const int i = r * nthr + tid;
@@ -342,7 +429,7 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
       if ((i & 7) >= p.M) xs[i] = 0.f;
     for (int i = tid; i < 64; i += nthr) reinterpret_cast<uint32_t*>(zbuf)[i] = 0u;
   }
-  v1d::bar_sync(v1d::kBarCons, nthr);
+  v1d::bar_sync(kBarPrologue, nthr);
 
   // int4: the lane's B column is batch row g; q4_K: batch row g % MP2 (see q4k_tile_fma)
   const int mrow = kQ4K ? g % (MP2 > 0 ? MP2 : 1) : g;
@@ -372,8 +459,8 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
   int bl = 0, ti = 0;
   locate(vw, bl, ti);
   auto flush = [&](int b) {
-    const int s = b & 1;
-    if (b >= 2) v1d::bar_sync(v1d::kBarFree0 + s, nthr_all);
+    const int s = b % kRedSlots;
+    if (b >= kRedSlots) v1d::bar_sync(kBarRedFree + s, nthr_all);
     float* rs = red + s * red_slot + warp * 16 * p.Mp;
     if constexpr (kQ4K && MP2 < 8) {
       // columns 2t, 2t+1 of a lane hold batch rows (2t + e) % MP2 of different
@@ -413,7 +500,7 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
       put(rs, yacc[0], yacc[1], yacc[2], yacc[3]);
       if constexpr (DUAL) put(rs + W * 16 * p.Mp, yacc2[0], yacc2[1], yacc2[2], yacc2[3]);
     }
-    v1d::bar_arrive(v1d::kBarFull0 + s, nthr_all);
+    v1d::bar_arrive(kBarRedFull + s, nthr_all);
     yacc[0] = yacc[1] = yacc[2] = yacc[3] = 0.f;
     yacc2[0] = yacc2[1] = yacc2[2] = yacc2[3] = 0.f;
   };
@@ -439,7 +526,10 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
       if (ok) {
         if constexpr (kQ4K)
           q4k_tile_fma<MP2>(st + u * p.tb, xbase + ti * xstep, xrow, zbuf, xs + ti * 64, lane, g, t, yacc);
-        else if constexpr (DUAL) {
+        else if constexpr (ZQ) {
+          tile_fma_zq(st + u * p.tb, xbase + ti * xstep, lane, g, yacc);
+          if constexpr (DUAL) tile_fma_zq(st + u * p.tb + p.tb / 2, xbase + ti * xstep, lane, g, yacc2);
+        } else if constexpr (DUAL) {
           v1d::tile_fma(st + u * p.tb, xbase + ti * xstep, xsl + ti * 8, lane, g, yacc);
           v1d::tile_fma(st + u * p.tb + p.tb / 2, xbase + ti * xstep, xsl + ti * 8, lane, g, yacc2);
         } else
