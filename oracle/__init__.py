@@ -24,6 +24,10 @@ from .q4 import (  # noqa: F401
     bound,
     dequant_bf16,
     dequant_int4,
+    dequant_mxfp4,
+    e2m1_value,
+    e8m0_value,
+    MXFP4_BLOCK,
     dequant_q4k,
     dequant_q4k_from_plane,
     exact_in_f32,

@@ -188,6 +188,50 @@ def dequant_q4k_from_plane(raw, plane, N: int, K: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# mxfp4 blockwise (named by the block_quantized_matmul / _moe mxfp4 rows of the
+# CPU criterion bench block in onnx-genai PR #1000; the page does not print
+# the format, so the reading taken is the OCP microscaling FP4 definition:
+# blocks of 32 along K share one E8M0 scale 2^(E - 127), elements are E2M1)
+# --------------------------------------------------------------------------
+
+MXFP4_BLOCK = 32
+
+
+def e2m1_value(code) -> np.ndarray:
+    """Value of a 4-bit E2M1 code: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa.
+
+    Exponent field 0 is the subnormal range (0 or 0.5); otherwise the value is
+    2^(e - 1)·(1 + m/2).
+    """
+    c = np.asarray(code).astype(np.int64)
+    sign = np.where(c & 8, -1.0, 1.0)
+    e = (c >> 1) & 3
+    m = (c & 1).astype(np.float64)
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.ldexp(1.0, np.maximum(e - 1, 0)))
+    return sign * mag
+
+
+def e8m0_value(byte) -> np.ndarray:
+    """2^(E - 127) for an E8M0 scale byte (255 is NaN)."""
+    b = np.asarray(byte).astype(np.int64)
+    return np.where(b == 255, np.nan, np.ldexp(1.0, b - 127))
+
+
+def dequant_mxfp4(w_packed, scales, N: int, K: int) -> np.ndarray:
+    """W[n, k] = 2^(E[n, k // 32] - 127) · e2m1(q[n, k]) in float64 (exact).
+
+    Codes [N][K/2] bytes, two per byte, low nibble = even k (the int4 reading);
+    scales [N][K/32] E8M0 bytes.
+    """
+    if K % MXFP4_BLOCK:
+        raise ValueError("mxfp4 needs K % 32 == 0")
+    q = int4_codes(w_packed, N, K)
+    E = np.asarray(scales, dtype=np.uint8).reshape(N, K // MXFP4_BLOCK)
+    blk = np.arange(K) // MXFP4_BLOCK
+    return e8m0_value(E)[:, blk] * e2m1_value(q)
+
+
+# --------------------------------------------------------------------------
 # bf16 (AstrAI commit log, uint4-anchoring bullet: any K, any 2-byte offset)
 # --------------------------------------------------------------------------
 

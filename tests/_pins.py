@@ -339,6 +339,56 @@ def pin_exact_in_f32(o):
     assert not o.exact_in_f32(np.array([1.0 + 2.0 ** -30]))
 
 
+# ---------------------------------------------------------------- mxfp4 pins
+
+# The sixteen E2M1 values in code order (sign bit 3, exponent bits 2..1,
+# mantissa bit 0): the format's value table, typed out, not computed.
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def pin_e2m1_table(o):
+    got = o.e2m1_value(np.arange(16))
+    assert [float(v) for v in got] == E2M1_TABLE
+    assert all(math.copysign(1.0, float(g)) == math.copysign(1.0, t) for g, t in zip(got, E2M1_TABLE))
+
+
+def pin_e8m0_scales(o):
+    """E8M0 byte E is 2^(E - 127); 255 is NaN."""
+    cases = {127: 1.0, 128: 2.0, 126: 0.5, 0: 2.0 ** -127, 254: 2.0 ** 127, 120: 1.0 / 128}
+    for b, v in cases.items():
+        assert float(o.e8m0_value(b)) == v, b
+    assert math.isnan(float(o.e8m0_value(255)))
+
+
+def pin_mxfp4_hand(o):
+    """Two blocks of one row: block 0 scale byte 128 (x2) with first codes 1, 2
+    (0.5, 1.0 -> 1.0, 2.0); block 1 scale byte 125 (x1/4) with first codes
+    15, 8 (-6, -0 -> -1.5, -0); every other code 0."""
+    w = np.zeros((1, 32), dtype=np.uint8)
+    w[0, 0] = 0x21                   # k0 = code 1, k1 = code 2
+    w[0, 16] = 0x8F                  # k32 = code 15, k33 = code 8
+    sc = np.array([[128, 125]], dtype=np.uint8)
+    W = o.dequant_mxfp4(w, sc, 1, 64)
+    assert W[0, 0] == 1.0 and W[0, 1] == 2.0 and W[0, 32] == -1.5 and W[0, 33] == 0.0
+    assert np.count_nonzero(W) == 3
+
+
+def pin_mxfp4_brute(o):
+    """Element by element through the typed value table on a small random tensor."""
+    rng = np.random.default_rng(91)
+    N, K = 3, 96
+    w = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sc = rng.integers(110, 140, (N, K // 32), dtype=np.uint8)
+    W = o.dequant_mxfp4(w, sc, N, K)
+    for n in range(N):
+        for k in range(K):
+            byte = int(w[n, k // 2])
+            code = byte & 15 if k % 2 == 0 else byte >> 4
+            want = E2M1_TABLE[code] * 2.0 ** (int(sc[n, k // 32]) - 127)
+            assert W[n, k] == want, (n, k)
+    assert o.exact_in_f32(W)
+
+
 # ---------------------------------------------------------------- SwiGLU pins
 
 def pin_silu_closed_forms(o):
@@ -413,6 +463,10 @@ ALL_PINS = [
     pin_gemv_fsum,
     pin_accept_threshold,
     pin_exact_in_f32,
+    pin_e2m1_table,
+    pin_e8m0_scales,
+    pin_mxfp4_hand,
+    pin_mxfp4_brute,
     pin_silu_closed_forms,
     pin_silu_reflection_and_slope,
     pin_swiglu_hand,

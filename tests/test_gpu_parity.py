@@ -216,15 +216,18 @@ def test_gemv_int4_v1_layout(M, N, K, bs, zeros):
     assert labels["cc"] == "unsupported" and ".simple." in labels["simple"], labels
 
 @gpu
+@pytest.mark.parametrize("zq", [0, 1])
 @pytest.mark.parametrize("C", [1, 2, 4])
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("N,K,bs,zeros", [(37, 2048, 128, True), (1000, 1536, 256, False), (300, 512, 128, True),
                                           (4100, 1024, 128, True), (16, 4096, 256, True)])
-def test_gemv_int4_v1_cluster_split(C, M, N, K, bs, zeros, monkeypatch):
-    """The B200_V1 kernel with subnormal codes and a per-tile Σx zero-point term,
-    with the k-tiles of every band split over clusters of C CTAs (partials added
+def test_gemv_int4_v1_cluster_split(zq, C, M, N, K, bs, zeros, monkeypatch):
+    """The B200_V1 band kernel, both tile forms (zq=1: exact q − z in the MMA
+    operand; zq=0: subnormal codes with a per-tile Σx zero-point term), with
+    the k-tiles of every band split over clusters of C CTAs (partials added
     through distributed shared memory).  Two calls in a row must agree bit for bit."""
     monkeypatch.setenv("WQ_FORCE_KERNEL", "v1s")
+    monkeypatch.setenv("WQ_V1_ZQ", str(zq))
     monkeypatch.setenv("WQ_V1_C", str(C))
     c = Int4Case(M, N, K, bs, zeros, workload=23, layout=wq.WQ_LAYOUT_B200_V1)
     y1 = c.run()
@@ -289,7 +292,7 @@ def test_gemv_int4_v1_default_kernel_full_size():
     c = Int4Case(1, 4096, 14336, 128, True, workload=3, layout=wq.WQ_LAYOUT_B200_V1)
     rows = sample_rows(4096)
     y = c.run()
-    assert ".gemv.v1k." in wq.last_kernel(), wq.last_kernel()
+    assert ".gemv.v1s." in wq.last_kernel(), wq.last_kernel()
     W = oracle.dequant_int4(c.w[rows], c.s[rows], c.z[rows], len(rows), 14336, 128)
     check(y[:, rows], W, c.x, "B200_V1 4096x14336 sampled rows")
 

@@ -123,6 +123,30 @@ def _swiglu_tolerance_no_up_term(a, b, Ba, Bb, rel=2e-3, abs_=1e-3):
     return prop + 2.0 ** -10 * (np.abs(oq.silu(a) * b) + prop) + abs_
 
 
+def _e2m1_exponent_unbiased(code):
+    c = np.asarray(code).astype(np.int64)
+    sign = np.where(c & 8, -1.0, 1.0)
+    e = (c >> 1) & 3
+    m = (c & 1).astype(np.float64)
+    return sign * np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.ldexp(1.0, e))
+
+
+def _e2m1_unsigned(code):
+    return np.abs(_orig["e2m1_value"](code))
+
+
+def _e8m0_bias_128(byte):
+    b = np.asarray(byte).astype(np.int64)
+    return np.where(b == 255, np.nan, np.ldexp(1.0, b - 128))
+
+
+def _mxfp4_block_16(w_packed, scales, N, K):
+    q = oq.int4_codes(w_packed, N, K)
+    E = np.asarray(scales, dtype=np.uint8).reshape(N, K // 32)
+    blk = np.minimum(np.arange(K) // 16, K // 32 - 1)
+    return oq.e8m0_value(E)[:, blk] * oq.e2m1_value(q)
+
+
 MUTANTS = {
     "int4 nibbles high-first": ("int4_codes", _int4_codes_high_first),
     "int4 default zero-point 0": ("int4_zero_points", _zero_points_default_zero),
@@ -138,6 +162,10 @@ MUTANTS = {
     "bound without abs": ("bound", _bound_no_abs),
     "acceptance twice as loose": ("accept", _accept_loose),
     "bf16 offset ignored": ("dequant_bf16", _dequant_bf16_ignores_offset),
+    "e2m1 exponent without its bias": ("e2m1_value", _e2m1_exponent_unbiased),
+    "e2m1 sign dropped": ("e2m1_value", _e2m1_unsigned),
+    "e8m0 bias 128": ("e8m0_value", _e8m0_bias_128),
+    "mxfp4 blocks of 16": ("dequant_mxfp4", _mxfp4_block_16),
     "silu without the a factor": ("silu", _silu_without_a),
     "silu reflected": ("silu", _silu_reflected),
     "swiglu gate and up swapped": ("swiglu_gemv", _swiglu_gate_up_swapped),

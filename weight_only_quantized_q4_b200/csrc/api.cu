@@ -505,7 +505,7 @@ int v1_max_clusters(int C, int smem, int threads, int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(&gemv_v1_kernel), &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(&gemv_v1_kernel<true>), &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -513,18 +513,31 @@ int v1_max_clusters(int C, int smem, int threads, int sms) {
   return n;
 }
 
+// WQ_V1_ZQ=0/1 picks the B200_V1 band kernel's tile arithmetic (A/B runs):
+// 1 (default) forms the exact q − z in the MMA operand, 0 uses subnormal
+// codes with a per-tile Σx zero-point term.
+bool v1_zq() {
+  const char* v = std::getenv("WQ_V1_ZQ");
+  return !(v && std::atoi(v) == 0);
+}
+
+using V1Kernel = void (*)(const V1Params);
+V1Kernel v1_kernel_fn() { return v1_zq() ? &gemv_v1_kernel<true> : &gemv_v1_kernel<false>; }
+
 int v1_configure() {
   static std::mutex mu;
-  static bool configured[64] = {};
+  static bool configured[2][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(mu);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemv_v1_kernel),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
-    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-    configured[dev] = true;
-  }
+  const V1Kernel fns[2] = {&gemv_v1_kernel<false>, &gemv_v1_kernel<true>};
+  for (int z = 0; z < 2; ++z)
+    if (dev >= 0 && dev < 64 && !configured[z][dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fns[z]),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[z][dev] = true;
+    }
   return WQ_OK;
 }
 
@@ -751,7 +764,7 @@ int launch_v1(const V1Plan& plan, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemv_v1_kernel, plan.p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, v1_kernel_fn(), plan.p);
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemv_v1 launch: ") + cudaGetErrorString(e));
   return launch_check("gemv_v1 launch");
 }
@@ -1049,7 +1062,8 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   const int n_tiles = (N + 127) / 128, m_tiles = (M + p.BN - 1) / p.BN;
   const int nst = (K + 63) / 64;  // bf16: a partial last stage reads zeros past K (TMA bounds fill)
   int S = 1;
-  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nst % (2 * p.spr * S) == 0) S *= 2;
+  // the largest power-of-two split that still fits one wave, every CTA keeping an even number of raw slots
+  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nst % (2 * p.spr * S * 2) == 0) S *= 2;
   if (const char* s_env = std::getenv("WQ_TC5_S")) {  // tests and tuning
     const int sf = std::atoi(s_env);
     if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
@@ -1177,8 +1191,10 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
         label = buf;
         continue;
       }
+      // (the stream-K kernel measured slower than the band kernel for int4 on
+      // B200 at the 4096x14336 class shapes: it runs on request only)
       V1KPlan kplan;
-      const bool want_v1k = force ? std::strcmp(force, "v1k") == 0 : true;
+      const bool want_v1k = force ? std::strcmp(force, "v1k") == 0 : false;
       if (want_v1k && layout == WQ_LAYOUT_B200_V1 && aligned16(xc) &&
           plan_v1k(Fmt::Int4, mc, N, K, block_size, di.sms, &kplan)) {
         kplan.p.x = xc;

@@ -114,6 +114,56 @@ __device__ __forceinline__ void tile_fma(const uint8_t* tp, const uint8_t* xt, c
   y[3] = fmaf(s1, fmaf(-z1, X.y, fmaf(dh[3], 0.0625f, dl[3])), y[3]);
 }
 
+// int4 B200_V1 tile with the zero-point taken out of the MMA operand: a nibble
+// masked under the fp16 pattern of 1024 (low nibbles) or 64 (high nibbles) is
+// 1024 + q or 64 + q exactly; subtracting 1024 + z or 64 + z (one HSUB2 per
+// pair) leaves the exact integer q − z.  The MMA then forms Σ (q − z)·x
+// directly: no Σx table, no prologue, one fp32 FMA by the scale per output.
+__device__ __forceinline__ uint32_t v1k_lop3_or(uint32_t v, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(magic));  // (v & mask) | magic
+  return r;
+}
+__device__ __forceinline__ uint32_t v1k_hsub2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ void tile_fma_zq(const uint8_t* tp, const uint8_t* xt, int lane, int g, float (&y)[4]) {
+  const uint4 qa = *reinterpret_cast<const uint4*>(tp + lane * 16);
+  const uint4 qb = *reinterpret_cast<const uint4*>(tp + 512 + lane * 16);
+  uint4 xv[4];
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) xv[gi] = *reinterpret_cast<const uint4*>(xt + 64 * gi);
+  const uint16_t* sc = reinterpret_cast<const uint16_t*>(tp + 1024);
+  const uint32_t sb0 = sc[g], sb1 = sc[g + 8];
+  const uint2 zz = *reinterpret_cast<const uint2*>(tp + 1056);
+  const uint32_t z0 = (zz.x >> (4 * g)) & 15u, z1 = (zz.y >> (4 * g)) & 15u;
+  const uint32_t zl0 = (0x6400u | z0) * 0x00010001u, zl1 = (0x6400u | z1) * 0x00010001u;
+  const uint32_t zh0 = (0x5400u | (z0 << 4)) * 0x00010001u, zh1 = (0x5400u | (z1 << 4)) * 0x00010001u;
+  const uint32_t v0[4] = {qa.x, qa.z, qb.x, qb.z}, v1[4] = {qa.y, qa.w, qb.y, qb.w};
+  float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};  // two chains: even / odd 32-k groups
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) {
+    const uint32_t a0 = v0[gi], a1 = v1[gi], a08 = a0 >> 8, a18 = a1 >> 8;
+    float(&d)[4] = (gi & 1) ? db : da;
+    mma16816(d, v1k_hsub2(v1k_lop3_or(a0, 0x000F000Fu, 0x64006400u), zl0),
+                  v1k_hsub2(v1k_lop3_or(a1, 0x000F000Fu, 0x64006400u), zl1),
+                  v1k_hsub2(v1k_lop3_or(a08, 0x000F000Fu, 0x64006400u), zl0),
+                  v1k_hsub2(v1k_lop3_or(a18, 0x000F000Fu, 0x64006400u), zl1), xv[gi].x, xv[gi].z);
+    mma16816(d, v1k_hsub2(v1k_lop3_or(a0, 0x00F000F0u, 0x54005400u), zh0),
+                  v1k_hsub2(v1k_lop3_or(a1, 0x00F000F0u, 0x54005400u), zh1),
+                  v1k_hsub2(v1k_lop3_or(a08, 0x00F000F0u, 0x54005400u), zh0),
+                  v1k_hsub2(v1k_lop3_or(a18, 0x00F000F0u, 0x54005400u), zh1), xv[gi].y, xv[gi].w);
+  }
+  const float s0 = h16_to_f32(sb0), s1 = h16_to_f32(sb1);
+  y[0] = fmaf(s0, da[0] + db[0], y[0]);
+  y[1] = fmaf(s0, da[1] + db[1], y[1]);
+  y[2] = fmaf(s1, da[2] + db[2], y[2]);
+  y[3] = fmaf(s1, da[3] + db[3], y[3]);
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -134,7 +184,11 @@ __device__ __forceinline__ float dsmem_ld(const float* local, uint32_t rank) {
 
 constexpr int kV1MaxWarps = 26;  // consumer warps + producer + reducer
 
+// ZQ: tiles through v1d::tile_fma_zq (exact q − z in the MMA operand, no Σx
+// table or prologue); otherwise subnormal codes with the per-tile Σx term.
+template <bool ZQ = false>
 __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Params p) {
+  constexpr float kYScale = ZQ ? 1.f : 16777216.f;  // subnormal-code partials are in units of 2^-24
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int W = p.W;
@@ -255,7 +309,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
         if (p.C > 1) {
           part[(bl * 16 + row) * p.M + n] = sum;
         } else if (r0 + row < p.N && !*abort_flag) {
-          reinterpret_cast<__half*>(p.y)[static_cast<long long>(n) * p.N + r0 + row] = __float2half_rn(sum * 16777216.f);
+          reinterpret_cast<__half*>(p.y)[static_cast<long long>(n) * p.N + r0 + row] = __float2half_rn(sum * kYScale);
         }
       }
       if (bl + 2 < n_bl) v1d::bar_arrive(v1d::kBarFree0 + s, nthr_all);
@@ -272,7 +326,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
     bool ok = mbar_wait_bounded(xbar, 0u);
     if (!ok) *abort_flag = 1;
     {
-      const int items = p.tpc * p.M * 4;
+      const int items = ZQ ? 0 : p.tpc * p.M * 4;
       for (int b0 = 0; b0 < items; b0 += nthr) {
         const int i = b0 + tid;
         float sum = 0.f;
@@ -349,7 +403,12 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
           flush(cur_bl);
           ++cur_bl;
         }
-        if (ok) v1d::tile_fma(st + u * p.tb, xbase + ti * xstep, xsl + ti * 8, lane, g, yacc);
+        if (ok) {
+          if constexpr (ZQ)
+            v1d::tile_fma_zq(st + u * p.tb, xbase + ti * xstep, lane, g, yacc);
+          else
+            v1d::tile_fma(st + u * p.tb, xbase + ti * xstep, xsl + ti * 8, lane, g, yacc);
+        }
         ti += W;
         while (ti >= p.tpc) {
           ti -= p.tpc;
@@ -384,7 +443,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
       float sum = 0.f;
       for (int c = 0; c < p.C; ++c) sum += v1d::dsmem_ld(part + i, static_cast<uint32_t>(c));
       if (r < p.N && !*abort_flag)
-        reinterpret_cast<__half*>(p.y)[static_cast<long long>(n) * p.N + r] = __float2half_rn(sum * 16777216.f);
+        reinterpret_cast<__half*>(p.y)[static_cast<long long>(n) * p.N + r] = __float2half_rn(sum * kYScale);
     }
     v1d::cluster_sync();
   }

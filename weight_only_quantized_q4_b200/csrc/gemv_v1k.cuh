@@ -145,56 +145,6 @@ __device__ __forceinline__ void q4k_tile_fma(const uint8_t* tp, const uint8_t* x
   }
 }
 
-// int4 B200_V1 tile with the zero-point taken out of the MMA operand: a nibble
-// masked under the fp16 pattern of 1024 (low nibbles) or 64 (high nibbles) is
-// 1024 + q or 64 + q exactly; subtracting 1024 + z or 64 + z (one HSUB2 per
-// pair) leaves the exact integer q − z.  The MMA then forms Σ (q − z)·x
-// directly: no Σx table, no prologue, one fp32 FMA by the scale per output.
-__device__ __forceinline__ uint32_t v1k_lop3_or(uint32_t v, uint32_t mask, uint32_t magic) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(magic));  // (v & mask) | magic
-  return r;
-}
-__device__ __forceinline__ uint32_t v1k_hsub2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-__device__ __forceinline__ void tile_fma_zq(const uint8_t* tp, const uint8_t* xt, int lane, int g, float (&y)[4]) {
-  const uint4 qa = *reinterpret_cast<const uint4*>(tp + lane * 16);
-  const uint4 qb = *reinterpret_cast<const uint4*>(tp + 512 + lane * 16);
-  uint4 xv[4];
-#pragma unroll
-  for (int gi = 0; gi < 4; ++gi) xv[gi] = *reinterpret_cast<const uint4*>(xt + 64 * gi);
-  const uint16_t* sc = reinterpret_cast<const uint16_t*>(tp + 1024);
-  const uint32_t sb0 = sc[g], sb1 = sc[g + 8];
-  const uint2 zz = *reinterpret_cast<const uint2*>(tp + 1056);
-  const uint32_t z0 = (zz.x >> (4 * g)) & 15u, z1 = (zz.y >> (4 * g)) & 15u;
-  const uint32_t zl0 = (0x6400u | z0) * 0x00010001u, zl1 = (0x6400u | z1) * 0x00010001u;
-  const uint32_t zh0 = (0x5400u | (z0 << 4)) * 0x00010001u, zh1 = (0x5400u | (z1 << 4)) * 0x00010001u;
-  const uint32_t v0[4] = {qa.x, qa.z, qb.x, qb.z}, v1[4] = {qa.y, qa.w, qb.y, qb.w};
-  float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};  // two chains: even / odd 32-k groups
-#pragma unroll
-  for (int gi = 0; gi < 4; ++gi) {
-    const uint32_t a0 = v0[gi], a1 = v1[gi], a08 = a0 >> 8, a18 = a1 >> 8;
-    float(&d)[4] = (gi & 1) ? db : da;
-    v1d::mma16816(d, v1k_hsub2(v1k_lop3_or(a0, 0x000F000Fu, 0x64006400u), zl0),
-                  v1k_hsub2(v1k_lop3_or(a1, 0x000F000Fu, 0x64006400u), zl1),
-                  v1k_hsub2(v1k_lop3_or(a08, 0x000F000Fu, 0x64006400u), zl0),
-                  v1k_hsub2(v1k_lop3_or(a18, 0x000F000Fu, 0x64006400u), zl1), xv[gi].x, xv[gi].z);
-    v1d::mma16816(d, v1k_hsub2(v1k_lop3_or(a0, 0x00F000F0u, 0x54005400u), zh0),
-                  v1k_hsub2(v1k_lop3_or(a1, 0x00F000F0u, 0x54005400u), zh1),
-                  v1k_hsub2(v1k_lop3_or(a08, 0x00F000F0u, 0x54005400u), zh0),
-                  v1k_hsub2(v1k_lop3_or(a18, 0x00F000F0u, 0x54005400u), zh1), xv[gi].y, xv[gi].w);
-  }
-  const float s0 = h16_to_f32(sb0), s1 = h16_to_f32(sb1);
-  y[0] = fmaf(s0, da[0] + db[0], y[0]);
-  y[1] = fmaf(s0, da[1] + db[1], y[1]);
-  y[2] = fmaf(s1, da[2] + db[2], y[2]);
-  y[3] = fmaf(s1, da[3] + db[3], y[3]);
-}
-
 // Split-band counters: one atomic with acquire-release semantics both
 // publishes this piece's partial sums (written by the warp before a
 // __syncwarp) and, for the last piece, makes the other pieces visible.
@@ -527,8 +477,8 @@ __global__ void __launch_bounds__(kV1KMaxWarps * 32, 1) gemv_v1k_kernel(const V1
         if constexpr (kQ4K)
           q4k_tile_fma<MP2>(st + u * p.tb, xbase + ti * xstep, xrow, zbuf, xs + ti * 64, lane, g, t, yacc);
         else if constexpr (ZQ) {
-          tile_fma_zq(st + u * p.tb, xbase + ti * xstep, lane, g, yacc);
-          if constexpr (DUAL) tile_fma_zq(st + u * p.tb + p.tb / 2, xbase + ti * xstep, lane, g, yacc2);
+          v1d::tile_fma_zq(st + u * p.tb, xbase + ti * xstep, lane, g, yacc);
+          if constexpr (DUAL) v1d::tile_fma_zq(st + u * p.tb + p.tb / 2, xbase + ti * xstep, lane, g, yacc2);
         } else if constexpr (DUAL) {
           v1d::tile_fma(st + u * p.tb, xbase + ti * xstep, xsl + ti * 8, lane, g, yacc);
           v1d::tile_fma(st + u * p.tb + p.tb / 2, xbase + ti * xstep, xsl + ti * 8, lane, g, yacc2);
