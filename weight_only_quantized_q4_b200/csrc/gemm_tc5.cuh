@@ -414,13 +414,19 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
     else
       reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(v);
   };
-  // the two accumulator tiles of a 16-column group, added (fixed order)
+  // the two accumulator tiles of a 16-column group, added (fixed order); a CTA
+  // with a single stage (bf16, K <= 64) never wrote the odd tile
   auto acc16 = [&](int c0, float (&v)[16]) {
     uint32_t r0[16], r1[16];
     tmem_ld16(lane_base + c0, r0);
-    tmem_ld16(lane_base + p.BN + c0, r1);
+    if (nks > 1) {
+      tmem_ld16(lane_base + p.BN + c0, r1);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
+      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]);
+    }
   };
   if (p.S == 1) {
     if (ok && reads) {
