@@ -157,6 +157,26 @@ int gemv_int4_swiglu(const void* x_f16, const void* w_gate_up, void* y_f16, int 
 int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K,
              int layout, void* stream);
 
+/* gemv_q4k for the B200_V1 q4_K stream, for callers that must not allocate
+ * device memory.  No counterpart on the pages: it exists because the ordinary
+ * call sets up a small split-band workspace with cudaMalloc the first time it
+ * runs on a stream, and some callers cannot allow that: programs that own all
+ * device memory through their own pool or a fixed budget, and programs that
+ * must not let a library call block or synchronize the device the way
+ * cudaMalloc can.  This call instead uses one fixed array in the library's
+ * own device memory (about 272 KB, reserved on every GPU that loads the
+ * library and held until the process exits); it never calls cudaMalloc or
+ * cudaFree.  Its first call on a device looks up the array's device address;
+ * make that first call before any stream capture.  Limits: layout must be
+ * WQ_LAYOUT_B200_V1, N <= 65536 (larger N returns WQ_ERR_ARG); the other
+ * arguments are those of gemv_q4k.  The array keeps the last call's contents
+ * and each call clears the part that must start at zero, so calls that
+ * overlap on the GPU (for example on two streams at once) race: run them one
+ * after another.  Errors: WQ_ERR_ARG, WQ_ERR_ALIGN, WQ_ERR_LAYOUT,
+ * WQ_ERR_UNSUPPORTED, WQ_ERR_DEVICE, WQ_ERR_CUDA. */
+int gemv_q4k_noalloc(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K, int layout,
+                     void* stream);
+
 /* As gemv_q4k, but the per-chunk coefficients come from the W_dsc plane w_dsc
  * ((K/32)·N float2, chunk-major, N·K/4 bytes; build it with wq_build_q4k_dsc or
  * wq_build_q4k_dsc_device).  Only the code bytes of w_q4k are read. */

@@ -19,6 +19,7 @@ from .api import (  # noqa: F401
     gemv_int4_swiglu,
     gemv_q4k,
     gemv_q4k_dsc,
+    gemv_q4k_noalloc,
     last_error,
     last_kernel,
     wq_build_q4k_dsc,

@@ -31,6 +31,7 @@ _vp, _i, _sz, _cp = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_cha
 SIGNATURES = {
     "gemv_int4_blockwise": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "gemv_q4k": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "gemv_q4k_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "gemv_q4k_dsc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "gemv_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "gemv_int4_swiglu": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),

@@ -43,6 +43,18 @@ def gemv_q4k(x, w_q4k, y, M, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
     _check(lib().gemv_q4k(_ptr(x), _ptr(w_q4k), _ptr(y), M, N, K, layout, _stream(stream)), "gemv_q4k")
 
 
+def gemv_q4k_noalloc(x, w_q4k, y, M, N, K, layout=WQ_LAYOUT_B200_V1, stream=None):
+    """gemv_q4k over the B200_V1 stream that never allocates device memory.
+
+    For callers that own all device memory (their own pool, a fixed budget) or
+    must not let a library call block the device the way cudaMalloc can.  Its
+    scratch is one fixed array in the library's device memory (about 272 KB
+    per GPU, held until exit) shared by every call: calls that overlap on the
+    GPU race.  The first call on a device looks up that array's address, so
+    make it before any stream capture.  N is limited to 65536 rows."""
+    _check(lib().gemv_q4k_noalloc(_ptr(x), _ptr(w_q4k), _ptr(y), M, N, K, layout, _stream(stream)), "gemv_q4k_noalloc")
+
+
 def gemv_q4k_dsc(x, w_q4k, w_dsc, y, M, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
     _check(lib().gemv_q4k_dsc(_ptr(x), _ptr(w_q4k), _ptr(w_dsc), _ptr(y), M, N, K, layout, _stream(stream)),
            "gemv_q4k_dsc")

@@ -824,6 +824,39 @@ int reset_workspaces() {
 }
 
 // ---------------------------------------------------------------------------
+// Allocation-free variant of the split-band workspace (gemv_q4k_noalloc): a
+// fixed array in the library's own device memory, reserved when the library
+// is loaded and kept until the process exits, so that a call never allocates.
+// It serves at most kNaMaxBands bands (N <= 16 · kNaMaxBands rows) and
+// kNaMaxCtas CTAs.  Every such call on every stream uses this one array.
+// ---------------------------------------------------------------------------
+constexpr int kNaMaxBands = 4096;  // rows up to 65,536
+constexpr int kNaMaxCtas = 256;
+constexpr size_t kNaBytes = static_cast<size_t>(kNaMaxBands) * 4 + static_cast<size_t>(kNaMaxCtas) * 2 * 128 * 4;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNaBytes];
+
+// The array's device address, looked up once per device with that device
+// current (in host code the symbol is only a host-side handle).
+int noalloc_scratch(uint8_t** out) {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(WQ_ERR_DEVICE, "device ordinal out of range");
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(WQ_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return WQ_OK;
+}
+
+// ---------------------------------------------------------------------------
 // B200_V1 int4 GEMV, stream-K: planner and launcher
 // ---------------------------------------------------------------------------
 struct V1KPlan {
@@ -928,7 +961,7 @@ bool plan_v1k(Fmt f, int M, int N, int K, int block_size, int sms, V1KPlan* out,
   return true;
 }
 
-int launch_v1k(V1KPlan& plan, cudaStream_t st) {
+int launch_v1k(V1KPlan& plan, cudaStream_t st, bool use_stream_workspace = true) {
   static std::mutex mu;
   static bool configured[8][64] = {};
   const V1KKernel fn = v1k_kernel(plan.fmt, plan.mp2, plan.dual);
@@ -945,8 +978,10 @@ int launch_v1k(V1KPlan& plan, cudaStream_t st) {
       configured[ki][dev] = true;
     }
   }
-  int rc = split_workspace(st, &plan.p.counters, &plan.p.partials);
-  if (rc) return rc;
+  if (use_stream_workspace) {
+    int rc = split_workspace(st, &plan.p.counters, &plan.p.partials);
+    if (rc) return rc;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.grid, 1, 1);
   cfg.blockDim = dim3(plan.threads, 1, 1);
@@ -1352,6 +1387,48 @@ int gemv_q4k(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, in
   return run_gemv<Fmt::Q4K>("q4k", x_f16, static_cast<const uint8_t*>(w_q4k), nullptr, nullptr, nullptr, y_f16, M,
                             N, K, static_cast<long long>(K / 256) * 144, 0, 0, 0, true,
                             static_cast<cudaStream_t>(stream), layout);
+}
+
+int gemv_q4k_noalloc(const void* x_f16, const void* w_q4k, void* y_f16, int M, int N, int K, int layout,
+                     void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (layout != WQ_LAYOUT_B200_V1)
+    return fail(WQ_ERR_LAYOUT, "gemv_q4k_noalloc: reads the B200_V1 q4_K stream (wq_repack_q4k) only");
+  if (K % 256) return fail(WQ_ERR_ARG, "gemv_q4k_noalloc: K must be a multiple of 256");
+  if ((N + 15) / 16 > kNaMaxBands)
+    return fail(WQ_ERR_ARG, "gemv_q4k_noalloc: N above the fixed scratch maximum of 65536 rows");
+  if (!x_f16 || !w_q4k || !y_f16) return fail(WQ_ERR_ARG, "gemv_q4k_noalloc: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_q4k) || !aligned16(y_f16))
+    return fail(WQ_ERR_ALIGN, "gemv_q4k_noalloc: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  uint8_t* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n_bands = (N + 15) / 16;
+  // counters start each call at zero (a call that gave up may have left some set)
+  cudaError_t e = cudaMemsetAsync(scratch, 0, static_cast<size_t>(n_bands) * 4, st);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("scratch clear: ") + cudaGetErrorString(e));
+  std::string label;
+  for (int m0 = 0; m0 < M; m0 += 8) {
+    const int mc = std::min(8, M - m0);
+    V1KPlan plan;
+    if (!plan_v1k(Fmt::Q4K, mc, N, K, 0, di.sms, &plan))
+      return fail(WQ_ERR_UNSUPPORTED, "gemv_q4k_noalloc: the activations of this call do not fit the kernel");
+    plan.grid = std::min(plan.grid, kNaMaxCtas);
+    plan.p.counters = reinterpret_cast<int*>(scratch);
+    plan.p.partials = reinterpret_cast<float*>(scratch + static_cast<size_t>(kNaMaxBands) * 4);
+    plan.p.x = static_cast<const uint8_t*>(x_f16) + static_cast<long long>(m0) * K * 2;
+    plan.p.w = static_cast<const uint8_t*>(w_q4k);
+    plan.p.y = static_cast<uint8_t*>(y_f16) + static_cast<long long>(m0) * N * 2;
+    if ((rc = launch_v1k(plan, st, false))) return rc;
+    char buf[64];
+    std::snprintf(buf, sizeof(buf), "q4k.gemv.v1k.noalloc.m%d.g%d%s", mc, plan.grid, M > 8 ? ".chunked" : "");
+    label = buf;
+  }
+  set_last_kernel(label);
+  return WQ_OK;
 }
 
 int gemv_q4k_dsc(const void* x_f16, const void* w_q4k, const void* w_dsc, void* y_f16, int M, int N, int K,
