@@ -30,6 +30,14 @@
  *    with no synchronization in between.  A following kernel that itself
  *    uses programmatic dependent launch must wait (griddepcontrol.wait)
  *    before reading y, as usual.
+ *  - The tensor-core family (M >= 9) forms each weight in fp16 (q4_K, int4)
+ *    before the MMA, rounded once (relative error <= 2^-11 per weight).  A
+ *    weight row whose bound could pass the fp16 range (15·max|s| for int4,
+ *    max(|d|·945 + |dmin|·63) over the super-blocks for q4_K, above 65504)
+ *    is formed as w·2^-e with the least such e, and its fp32 result is
+ *    multiplied by 2^e: no finite weight becomes infinite.  In such a row a
+ *    weight that falls below the fp16 normal range after the scaling keeps
+ *    an absolute error of at most 2^(e-25).
  *  - The first call on a device configures kernel attributes and looks up the
  *    driver's tensor-map encoder; make it before capturing a CUDA graph.
  *  - Environment variables read at each call, for tests and tuning only:

@@ -420,6 +420,39 @@ def test_gemm_tcgen05_cluster_split_k(S, M, fmt, monkeypatch):
 
 
 @gpu
+@pytest.mark.parametrize("S", [1, 4])
+@pytest.mark.parametrize("fmt", ["int4", "q4k"])
+def test_gemm_tcgen05_weights_beyond_fp16_range(fmt, S, monkeypatch):
+    """Half the rows dequantize beyond the fp16 range (int4 scales up to 9000,
+    |w| up to 135000; q4_K d up to 100, |w| up to about 95000) beside ordinary
+    rows.  The tcgen05 path forms such rows as w·2^-e and rescales their fp32
+    result, so every output stays finite and within the tolerance (small
+    activations keep y itself inside fp16)."""
+    monkeypatch.setenv("WQ_TC5_S", str(S))
+    M, N, K = 16, 300, 2048
+    rng = np.random.default_rng(32)
+    big = rng.random(N) < 0.5
+    if fmt == "int4":
+        c = Int4Case(M, N, K, 128, True, workload=32)
+        c.s[big] = rng.uniform(5000, 9000, (int(big.sum()), K // 128)).astype(np.float16)
+        c.ds = dev(c.s)
+        run = c.run
+    else:
+        c = Q4KCase(M, N, K, workload=32)
+        d = rng.uniform(50, 100, (int(big.sum()), K // 256)).astype(np.float16)
+        c.raw[big, :, 0:2] = d.view(np.uint8).reshape(int(big.sum()), K // 256, 2)
+        c.draw = c.dw = dev(c.raw)
+        run = lambda: c.run(False)  # noqa: E731
+    c.x = (c.x.astype(np.float32) * 1e-4).astype(np.float16)
+    c.dx = dev(c.x)
+    y = run()
+    label = wq.last_kernel()
+    assert ".gemm.tc5." in label and label.endswith(f".s{S}"), label
+    assert np.isfinite(y).all()
+    check(y, c.W(), c.x, f"tcgen05 {fmt} beyond fp16 range S={S}")
+
+
+@gpu
 def test_gemm_tcgen05_forced_split_follows_the_automatic_rule(monkeypatch):
     """A forced cluster split must give every CTA an even number of 256-k raw
     slots (the rule of the automatic choice); K = 2048 with S = 8 gives one."""

@@ -124,7 +124,7 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // scale bits | zero-point << 16.
 template <Fmt F>
 __device__ __forceinline__ void dequant_stage(int s, int h, const uint8_t* raw, const uint8_t* hdr, uint32_t sz,
-                                              uint32_t (&o)[16]) {
+                                              float down, uint32_t (&o)[16]) {
   if constexpr (F == Fmt::Int4) {
     const uint4 c = *reinterpret_cast<const uint4*>(raw + 16 * h);
     const uint32_t sbits = sz & 0xFFFFu, z = sz >> 16;
@@ -148,7 +148,7 @@ __device__ __forceinline__ void dequant_stage(int s, int h, const uint8_t* raw, 
     const int pp = ((s * 64) & 255) >> 6;
     uint32_t sc2, mn2;
     q4k_scale_min_pair(hd.y, hd.z, hd.w, static_cast<uint32_t>(pp & 1), static_cast<uint32_t>(pp >> 1), sc2, mn2);
-    const float d = h16_to_f32(hd.x), dm = h16_to_f32(hd.x >> 16);
+    const float d = h16_to_f32(hd.x) * down, dm = h16_to_f32(hd.x >> 16) * down;  // ×2^-e: exact
     // half 0: chunk 2pp (low nibbles), half 1: chunk 2pp+1 (high nibbles)
     const uint32_t scv = h ? (sc2 >> 8) : (sc2 & 0xFFu), mnv = h ? (mn2 >> 8) : (mn2 & 0xFFu);
     const float A = __fmul_rn(d, static_cast<float>(scv)), B = -__fmul_rn(dm, static_cast<float>(mnv));
@@ -163,6 +163,59 @@ __device__ __forceinline__ void dequant_stage(int s, int h, const uint8_t* raw, 
       o[wd * 2 + 0] = pack_f16x2(f[0], f[1]);
       o[wd * 2 + 1] = pack_f16x2(f[2], f[3]);
     }
+  }
+}
+
+// fp16 range of the weight tile.  A dequantized weight must be finite in fp16
+// (|w| <= 65504) to enter the MMA; the bound of a row is 15·max|s| (int4) or
+// max(|d|·63·15 + |dmin|·63) (q4_K).  A row whose bound is above 65504 is
+// dequantized as w·2^-e, with the least e that brings the bound within range,
+// and its fp32 result is multiplied by 2^e (both exact).  Rows within range
+// (every row of ordinary weights) have e = 0 and are unchanged.  Non-finite
+// scales are left out of the bound: they propagate as in IEEE arithmetic.
+template <Fmt F>
+__device__ __forceinline__ int row_exponent(const TC5Params& p, int row) {
+  if constexpr (F == Fmt::BF16) {
+    return 0;
+  } else {
+    if (row >= p.N) return 0;
+    float bound = 0.f;
+    if constexpr (F == Fmt::Int4) {
+      const unsigned short* sr = reinterpret_cast<const unsigned short*>(p.scales) + static_cast<long long>(row) * p.nb;
+      uint32_t mx = 0;
+      auto take = [&](uint32_t bits) {
+        const uint32_t m = bits & 0x7FFFu;
+        if (m < 0x7C00u && m > mx) mx = m;
+      };
+      if ((p.nb & 7) == 0) {  // whole 16-byte groups (the scale array is 16-byte aligned)
+        const uint4* s4 = reinterpret_cast<const uint4*>(sr);
+#pragma unroll 4
+        for (int b = 0; b < p.nb / 8; ++b) {
+          const uint4 v = __ldg(s4 + b);
+          take(v.x), take(v.x >> 16), take(v.y), take(v.y >> 16);
+          take(v.z), take(v.z >> 16), take(v.w), take(v.w >> 16);
+        }
+      } else {
+#pragma unroll 8
+        for (int b = 0; b < p.nb; ++b) take(__ldg(sr + b));
+      }
+      bound = 15.f * h16_to_f32(mx);
+    } else {
+      const int nsb = p.K / 256;
+      const uint8_t* wr = p.w + static_cast<long long>(row) * nsb * 144;
+#pragma unroll 8
+      for (int j = 0; j < nsb; ++j) {
+        const uint32_t dd = __ldg(reinterpret_cast<const unsigned int*>(wr + 144ll * j));
+        const float b = fabsf(h16_to_f32(dd)) * 945.f + fabsf(h16_to_f32(dd >> 16)) * 63.f;
+        if (b <= 3.0e38f && b > bound) bound = b;  // finite d and dmin only
+      }
+    }
+    int e = 0;
+    while (bound > 65504.f) {
+      bound *= 0.5f;
+      ++e;
+    }
+    return e;
   }
 }
 
@@ -275,6 +328,9 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // dequant / epilogue warps: thread tid handles weight row n0 + (tid & 127) in both roles
+  const int row_e = warp < 8 ? row_exponent<F>(p, n0 + (tid & 127)) : 0;
+  const float row_up = __int_as_float((127 + row_e) << 23);  // 2^e
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -350,6 +406,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
     // ------------------------------------------------------------ dequant warps
     const int rl = tid & 127, h = tid >> 7;  // weight row (TMEM lane) and which 32 k of a stage
     const int row = n0 + rl;
+    const float down = __int_as_float((127 - row_e) << 23);  // 2^-e of this row
     uint32_t szr[kTc5SzAhead];
     if constexpr (F == Fmt::Int4) {
 #pragma unroll
@@ -374,11 +431,15 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
         if constexpr (F == Fmt::Int4) {
           sz = szr[i];
           if (ls + kTc5SzAhead < nks) szr[i] = fetch_sz(p, row, s_begin + ls + kTc5SzAhead);
+          if (row_e) {  // s·2^-e, rounded to fp16 (exact unless it falls below the normal range)
+            const uint32_t sb = __half_as_ushort(__float2half_rn(h16_to_f32(sz) * down));
+            sz = (sz & 0xFFFF0000u) | sb;
+          }
         }
         const uint8_t* rrow = smem + p.off_raw + rs * p.raw_bytes + rl * p.raw_pitch;
         const uint8_t* codes = F == Fmt::Int4 ? rrow + 32 * (ls & (p.spr - 1)) : rrow + 16 + 32 * (ls & 3);
         uint32_t o[16];
-        if constexpr (F != Fmt::BF16) dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, o);
+        if constexpr (F != Fmt::BF16) dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, down, o);
         uint8_t* at = smem + a * 16384;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -437,7 +498,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = m0 + c0 + j;
-          if (m < p.M && yrow < p.N) store_y(static_cast<long long>(m) * p.N + yrow, v[j]);
+          if (m < p.M && yrow < p.N) store_y(static_cast<long long>(m) * p.N + yrow, v[j] * row_up);
         }
       }
     }
@@ -451,7 +512,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
         float v[16];
         if (ok) acc16(c0, v);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[trow * p.BN + c0 + j] = ok ? v[j] : 0.f;
+        for (int j = 0; j < 16; ++j) acc[trow * p.BN + c0 + j] = ok ? v[j] * row_up : 0.f;
       }
     }
     tc5_cluster_sync();
