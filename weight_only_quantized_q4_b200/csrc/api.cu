@@ -344,7 +344,7 @@ bool plan_tc(Fmt f, int M, int N, int K, long long row_bytes, int nb, int zb, in
     seg_full = 0;
   } else if (f == Fmt::Int4) {
     if (block_size < 32 || K % 128) return false;
-    Kc = std::max(std::max(block_size, 128), kc_req > 0 ? kc_req / 256 * 256 : 1024);
+    Kc = std::max(std::max(block_size, 128), kc_req > 0 ? kc_req / 256 * 256 : 4096);
     Kc = std::min(Kc, K);
     seg_full = Kc / 2;
   } else if (f == Fmt::BF16) {
@@ -353,7 +353,7 @@ bool plan_tc(Fmt f, int M, int N, int K, long long row_bytes, int nb, int zb, in
     seg_full = 2ll * Kc;
   } else {
     if (K % 256) return false;
-    Kc = std::min(kc_req > 0 ? std::max(256, kc_req / 256 * 256) : 1024, K);
+    Kc = std::min(kc_req > 0 ? std::max(256, kc_req / 256 * 256) : (f == Fmt::Q4K && M <= 2 ? 2048 : 1024), K);
     seg_full = (Kc / 256) * 144;
   }
   TCParams& p = plan->p;
@@ -386,9 +386,14 @@ bool plan_tc(Fmt f, int M, int N, int K, long long row_bytes, int nb, int zb, in
   p.stage_bytes = static_cast<int>(round16(off));
   // WQ_TC_W overrides the number of consumer warps (tuning)
   // one CTA per SM for the B200_V1 stream needs 16 consumer warps (4 per
-  // scheduler) to cover the load / MMA latency chains of the tile loop
+  // scheduler) to cover the load / MMA latency chains of the tile loop;
+  // canonical int4 streams best with 12 warps over 4096-k stages, raw q4_K at
+  // M <= 2 with 12 warps over 2048 k (B200, against 8 warps over 1024 k:
+  // int4 M=1 4096x14336 22.8 -> 18.7 us, M=4 25.0 -> 20.4 us; q4_K M=1
+  // 4096x11008 20.4 -> 18.0 us; q4_K M=4 stays faster at 8 warps / 1024 k)
   const char* w_env = std::getenv("WQ_TC_W");
-  const int W = w_env ? std::max(1, std::min(16, std::atoi(w_env))) : (layout == WQ_LAYOUT_B200_V1 ? 16 : 8);
+  const int w_def = layout == WQ_LAYOUT_B200_V1 ? 16 : (f == Fmt::Int4 || (f == Fmt::Q4K && M <= 2)) ? 12 : 8;
+  const int W = w_env ? std::max(1, std::min(16, std::atoi(w_env))) : w_def;
   p.W = W;
   long long meta = 0;
   if (f == Fmt::Int4 && layout == WQ_LAYOUT_B200_V1) {
