@@ -71,12 +71,14 @@ for _M in (1, 2, 4, 8):
 for _M in (16, 32, 64, 128):
     for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336), (32000, 4096)):
         WORKLOADS[f"batched_int4_b128_zp_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 5, 0.002, 0.01)
+        WORKLOADS[f"batched_int4_b128_zp_v1_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 5, 0.002, 0.01,
+                                                                       layout=1)
         WORKLOADS[f"batched_q4k_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=False, workload=5)
 
 DEFAULT_WORKLOAD = "int4_b128_zp_v1_m1_4096x14336"
 METRIC = "achieved HBM GB/s and \u00b5s/call per quantized GEMV at M=1..8 vs ~8 TB/s peak"
-SWEEP_BATCHED = [f"batched_{f}_m{m}_{n}x{k}" for f in ("int4_b128_zp", "q4k") for m in (16, 64, 128)
-                 for n, k in ((4096, 4096), (14336, 4096), (32000, 4096))]
+SWEEP_BATCHED = [f"batched_{f}_m{m}_{n}x{k}" for f in ("int4_b128_zp_v1", "int4_b128_zp", "q4k")
+                 for m in (16, 32, 64, 128) for n, k in ((4096, 4096), (14336, 4096), (4096, 14336), (32000, 4096))]
 SWEEP = ["q4k_v1_m1_4096x11008", "q4k_v1_m4_4096x11008", "q4k_v1_m1_11008x4096", "int4_b128_zp_v1_m1_4096x14336", "int4_b128_zp_v1_m2_4096x14336", "int4_b128_zp_v1_m4_4096x14336", "int4_b128_zp_v1_m8_4096x14336",
          "int4_b128_zp_v1_m1_14336x4096", "int4_b128_zp_v1_m1_4096x4096",
          "int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",

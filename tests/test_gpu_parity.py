@@ -619,3 +619,95 @@ def test_full_batched_sampled(fmt, N, K):
         g.check(f"batched {fmt} {N}x{K} M={M}")
         y = g.t.cpu().numpy().astype(np.float64)
         check(y[:, rows], Wr, x, f"batched {fmt} {N}x{K} M={M} [{label}]")
+
+
+# ----------------------------------------------------- tcgen05 over the B200_V1 stream
+
+@gpu
+@pytest.mark.parametrize("M", [9, 16, 33, 64, 128, 200])
+@pytest.mark.parametrize("N,K,bs", [(300, 1024, 128), (37, 4096, 256), (1000, 384, 128), (16, 128, 128)])
+def test_gemm_v1tc_batched(M, N, K, bs):
+    """Batches of 9 and more over B200_V1 int4 weights run the tcgen05 kernel
+    that reads the band stream: ragged row tiles (N = 300, 37, 1000), an odd
+    number of 128-k steps (K = 384), a single step (K = 128), two batch tiles
+    (M = 200).  Guard bands around every output; two calls agree bit for bit."""
+    c = Int4Case(M, N, K, bs, True, workload=40, layout=wq.WQ_LAYOUT_B200_V1)
+    y = c.run()
+    assert ".gemm.v1tc." in wq.last_kernel(), wq.last_kernel()
+    check(y, c.W(), c.x, f"v1tc M={M} N={N} K={K} bs={bs}")
+    assert np.array_equal(y, c.run())
+
+
+@gpu
+@pytest.mark.parametrize("S", [1, 2, 4, 8])
+@pytest.mark.parametrize("M", [16, 48, 128])
+def test_gemm_v1tc_cluster_split_k(S, M, monkeypatch):
+    """K split over a cluster of S CTAs whose fp32 accumulators are added
+    through distributed shared memory in rank order."""
+    monkeypatch.setenv("WQ_V1TC_S", str(S))
+    c = Int4Case(M, 300, 4096, 128, True, workload=41, layout=wq.WQ_LAYOUT_B200_V1)
+    y = c.run()
+    label = wq.last_kernel()
+    assert ".gemm.v1tc." in label and label.endswith(f".s{S}"), label
+    check(y, c.W(), c.x, f"v1tc M={M} S={S}")
+    assert np.array_equal(y, c.run())
+
+
+@gpu
+def test_gemm_v1tc_forced_split_follows_the_rule(monkeypatch):
+    """A forced split must leave every CTA an even number of 128-k steps."""
+    monkeypatch.setenv("WQ_V1TC_S", "4")
+    c = Int4Case(16, 300, 768, 128, True, workload=41, layout=wq.WQ_LAYOUT_B200_V1)
+    with pytest.raises(wq.WQError) as e:
+        c.run()
+    assert e.value.code == wq.WQ_ERR_ARG
+
+
+@gpu
+@pytest.mark.parametrize("S", [1, 4])
+def test_gemm_v1tc_weights_beyond_fp16_range(S, monkeypatch):
+    """Half the rows with scales up to 9000 (|w| up to 135000): formed as
+    w·2^-e and rescaled in fp32, every output finite and within tolerance."""
+    monkeypatch.setenv("WQ_V1TC_S", str(S))
+    M, N, K = 16, 300, 2048
+    rng = np.random.default_rng(42)
+    big = rng.random(N) < 0.5
+    t = synth.int4_weights(N, K, 128, scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=42)
+    s = t["scales"].copy()
+    s[big] = rng.uniform(5000, 9000, (int(big.sum()), K // 128)).astype(np.float16)
+    g = Guarded((wq.wq_int4_packed_bytes(N, K, 128),), torch.uint8)
+    wq.wq_repack_int4(dev(t["w_packed"]), dev(s), dev(t["zeros"]), g.t, N, K, 128)
+    x = (synth.activations_f16(M, K, workload=42).astype(np.float32) * 1e-4).astype(np.float16)
+    gy = Guarded((M, N), torch.float16)
+    wq.gemv_int4_blockwise(dev(x), g.t, None, None, gy.t, M, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1)
+    torch.cuda.synchronize()
+    gy.check("v1tc large-scale y")
+    label = wq.last_kernel()
+    assert ".gemm.v1tc." in label and label.endswith(f".s{S}"), label
+    y = gy.t.cpu().numpy().astype(np.float64)
+    assert np.isfinite(y).all()
+    check(y, oracle.dequant_int4(t["w_packed"], s, t["zeros"], N, K, 128), x, f"v1tc beyond fp16 range S={S}")
+
+
+@gpu
+@pytest.mark.parametrize("N,K", FULL_BATCHED)
+def test_full_batched_v1tc_sampled(N, K):
+    """The batched int4 workload in the B200_V1 layout at its full sizes
+    (M = 16, 32, 64, 128) in the default launch configuration; sampled rows
+    vs the oracle, guard bands around every output."""
+    t = synth.int4_weights(N, K, 128, scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=5)
+    g = Guarded((wq.wq_int4_packed_bytes(N, K, 128),), torch.uint8)
+    wq.wq_repack_int4(dev(t["w_packed"]), dev(t["scales"]), dev(t["zeros"]), g.t, N, K, 128)
+    torch.cuda.synchronize()
+    rows = sample_rows(N)
+    Wr = oracle.dequant_int4(t["w_packed"][rows], t["scales"][rows], t["zeros"][rows], len(rows), K, 128)
+    for M in (16, 32, 64, 128):
+        x = synth.activations_f16(M, K, workload=5)
+        gy = Guarded((M, N), torch.float16)
+        wq.gemv_int4_blockwise(dev(x), g.t, None, None, gy.t, M, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1)
+        torch.cuda.synchronize()
+        label = wq.last_kernel()
+        assert ".gemm.v1tc." in label, label
+        gy.check(f"v1tc full {N}x{K} M={M}")
+        y = gy.t.cpu().numpy().astype(np.float64)
+        check(y[:, rows], Wr, x, f"v1tc full {N}x{K} M={M} [{label}]")

@@ -25,6 +25,7 @@
 #include "gemv_v1.cuh"
 #include "gemv_v1k.cuh"
 #include "gemm_tc5.cuh"
+#include "gemm_v1tc.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -567,6 +568,11 @@ bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clust
   const char* sk_env = std::getenv("WQ_V1_STAGE_KB");
   const int stage_budget = (sk_env ? std::max(1, std::atoi(sk_env)) : stage_kb) * 1024;
   p.tps = W * std::max(1, stage_budget / (W * p.tb));
+  // first stage: WQ_V1_FIRST tiles (tuning; rounded to whole multiples of W)
+  const char* f_env = std::getenv("WQ_V1_FIRST");
+  // (a first stage of one tile per warp lands sooner after the wait: B200, M=1
+  // 4096x14336 12.08 -> 11.98 us, 4096x4096 5.21 -> 5.01 us)
+  p.tps0 = f_env ? std::max(W, std::min(p.tps, std::atoi(f_env) / W * W)) : W;
   // Before waiting for the previous kernel: an L2 prefetch of the head of the
   // CTA's stream (safe whatever that kernel wrote; WQ_V1_PFKB, KB), or ring
   // stages copied to shared memory (WQ_V1_PRE, stages; only correct when the
@@ -575,6 +581,8 @@ bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clust
   p.pre = pre_env ? std::max(0, std::atoi(pre_env)) : 0;
   const char* pf_env = std::getenv("WQ_V1_PFKB");
   p.pf_bytes = p.pre > 0 ? 0 : (pf_env ? std::max(0, std::atoi(pf_env)) : 96) * 1024;
+  const char* pfd_env = std::getenv("WQ_V1_PFD");  // L2 prefetch distance in stages (tuning)
+  p.pfd = pfd_env ? std::max(0, std::atoi(pfd_env)) : 0;
   const char* h_env = std::getenv("WQ_V1_HINT");
   p.hint = h_env ? (std::atoi(h_env) != 0) : 1;
   p.stage_bytes = p.tps * p.tb;
@@ -1118,7 +1126,7 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   p.nks = nst / S;
   int rc;
   if constexpr (F == Fmt::Int4)
-    rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   else if constexpr (F == Fmt::BF16)
     rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, 2ull * K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   else
@@ -1165,6 +1173,99 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   return WQ_OK;
 }
 
+// tcgen05 batched GEMM over the int4 B200_V1 stream (blocks >= 128): planner and launcher
+int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, int block_size, int sms,
+                cudaStream_t st, std::string* label) {
+  if (K % 128 || block_size < 128) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: needs K % 128 == 0 and blocks >= 128");
+  V1TCParams p{};
+  p.w = w;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_bands = (N + 15) / 16;
+  p.tpb = K / 128;
+  p.tb = int4_v1_tile_bytes(block_size);
+  p.BN = std::min(128, (M + 15) / 16 * 16);
+  int cols = 32;
+  while (cols < 2 * p.BN) cols *= 2;  // two accumulator tiles (even / odd steps)
+  p.tmem_cols = cols;
+  const int n_tiles = (p.n_bands + 7) / 8, m_tiles = (M + p.BN - 1) / p.BN;
+  // Split K over a cluster of S CTAs (one CTA per SM) while the CTAs still fit
+  // one wave; every CTA keeps an even number of 128-k steps.
+  int S = 1;
+  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && p.tpb % (4 * S) == 0) S *= 2;
+  if (const char* s_env = std::getenv("WQ_V1TC_S")) {  // tests and tuning
+    const int sf = std::atoi(s_env);
+    if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
+      if (sf > 1 && p.tpb % (2 * sf)) return fail(WQ_ERR_ARG, "WQ_V1TC_S does not split K into an even number of steps per CTA");
+      S = sf;
+    }
+  }
+  p.S = S;
+  p.nks = p.tpb / S;
+  // shared memory: NA A slots (32 KB), NX activation slots, NR raw slots of T
+  // steps (one bulk copy of T tiles per band: few, large copies keep the
+  // copy engine streaming), row exponents, barriers
+  const int x_slot = p.BN * 256;
+  p.NA = 2;
+  p.NX = p.BN <= 32 ? 4 : p.BN <= 64 ? 3 : 2;
+  const int budget = kSmemPerSm + 4096 - 1024;
+  p.off_x = p.NA * 32768;
+  p.off_raw = p.off_x + p.NX * x_slot;
+  const int fixed = 512 + 16 + 8 * (2 * 4 + 2 * p.NX + 2 * p.NA + 1) + 16;
+  const char* t_env = std::getenv("WQ_V1TC_T");  // steps per raw slot (tuning)
+  p.NR = 3;
+  p.T = std::min(16, (budget - p.off_raw - fixed) / (p.NR * 8 * p.tb));
+  if (p.T < 2) {
+    p.NR = 2;
+    p.T = std::min(16, (budget - p.off_raw - fixed) / (p.NR * 8 * p.tb));
+  }
+  if (t_env) p.T = std::max(1, std::min(p.T, std::atoi(t_env)));
+  p.T = std::max(1, std::min(p.T, p.nks));
+  if (p.T < 1 || p.NR < 2) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: shared memory plan too large");
+  p.off_rowe = static_cast<int>(round16(static_cast<long long>(p.off_raw) + static_cast<long long>(p.NR) * 8 * p.T * p.tb));
+  p.off_bar = p.off_rowe + 512;
+  const int smem = 1024 + p.off_bar + 8 * (2 * p.NR + 2 * p.NX + 2 * p.NA + 1) + 16;
+  if (smem > kSmemPerSm + 4096) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: shared memory plan too large");
+  if (S > 1 && 512 * p.BN > p.off_raw) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: cluster partials do not fit");
+  int rc = encode_2d(&p.tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, 2ull * K, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  {
+    static std::mutex mu;
+    static bool configured[64] = {};
+    std::lock_guard<std::mutex> lk(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemm_v1tc_kernel),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles * S, m_tiles, 1);
+  cfg.blockDim = dim3(kV1TCWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemm_v1tc_kernel, p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_v1tc launch: ") + cudaGetErrorString(e));
+  rc = launch_check("gemm_v1tc launch");
+  if (rc) return rc;
+  char buf[64];
+  std::snprintf(buf, sizeof(buf), "int4.gemm.v1tc.bn%d.t%d.s%d", p.BN, p.T, S);
+  *label = buf;
+  return WQ_OK;
+}
+
 // Run one format over all M in chunks of at most 8 rows of x.
 template <Fmt F>
 int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros,
@@ -1182,6 +1283,17 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
                         (F == Fmt::Q4K && layout == WQ_LAYOUT_CANONICAL && K % 256 == 0) ||
                         (F == Fmt::BF16 && K % 8 == 0 && aligned16(w));
     const bool want = force ? std::strcmp(force, "tc5") == 0 : M >= 9;
+    if constexpr (F == Fmt::Int4) {
+      // B200_V1 int4 with blocks of at least 128: the tcgen05 kernel reads the band stream itself
+      const bool v1tc_ok = layout == WQ_LAYOUT_B200_V1 && K % 128 == 0 && block_size >= 128 && aligned16(x);
+      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : M >= 9;
+      if (v1tc_ok && want_v1tc) {
+        rc = launch_v1tc(x, w, y, M, N, K, block_size, di.sms, st, &label);
+        if (rc) return rc;
+        set_last_kernel(label);
+        return WQ_OK;
+      }
+    }
     if (tc5_ok && want && aligned16(x)) {
       if constexpr (F == Fmt::Int4 || F == Fmt::Q4K || F == Fmt::BF16) {
         rc = launch_tc5<F>(x, w, scales, zeros, y, M, N, K, nb, zb, block_size, di.sms, st, &label);

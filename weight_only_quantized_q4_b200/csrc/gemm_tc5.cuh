@@ -126,7 +126,7 @@ template <Fmt F>
 __device__ __forceinline__ void dequant_stage(int s, int h, const uint8_t* raw, const uint8_t* hdr, uint32_t sz,
                                               float down, uint32_t (&o)[16]) {
   if constexpr (F == Fmt::Int4) {
-    const uint4 c = *reinterpret_cast<const uint4*>(raw + 16 * h);
+    const uint4 c = *reinterpret_cast<const uint4*>(raw);  // this thread's 16 code bytes (32 k)
     const uint32_t sbits = sz & 0xFFFFu, z = sz >> 16;
     const uint32_t s2 = sbits | (sbits << 16);
     // (1024 + z, 64 + z): subtracted from (1024 + q_even, 64 + q_odd) gives (q - z) exactly
@@ -219,13 +219,24 @@ __device__ __forceinline__ int row_exponent(const TC5Params& p, int row) {
   }
 }
 
-// int4 scale and zero-point of stage s of weight row `row` (packed fp16 | z << 16)
-__device__ __forceinline__ uint32_t fetch_sz(const TC5Params& p, int row, int s) {
-  if (row >= p.N) return 8u << 16;
+// int4 scale and zero-point of stage s of weight row `row`, as the two loaded
+// words (fp16 scale bits; the zero-point byte holding blocks 2j and 2j+1).
+// Nothing here uses the loaded values, so the loads stay in flight until the
+// stage that needs them (sz_of combines them there): an operation on a load's
+// result at issue time would stall the thread for the whole load latency.
+// Rows past N read row N-1 (their outputs are never stored).
+__device__ __forceinline__ void fetch_sz(const TC5Params& p, int row, int s, uint32_t& sraw, uint32_t& zraw) {
+  const long long r = row < p.N ? row : p.N - 1;
   const int b = (s * 64) >> p.block_shift;  // blocks of >= 64 k: one scale / zero-point per stage
-  uint32_t z = 8u;
-  if (p.zeros) z = (__ldg(p.zeros + static_cast<long long>(row) * p.zb + (b >> 1)) >> ((b & 1) * 4)) & 15u;
-  return __ldg(reinterpret_cast<const unsigned short*>(p.scales) + static_cast<long long>(row) * p.nb + b) | (z << 16);
+  const uint8_t* zp = p.zeros ? p.zeros + r * p.zb + (b >> 1) : p.scales;  // any readable byte without zeros
+  sraw = __ldg(reinterpret_cast<const unsigned short*>(p.scales) + r * p.nb + b);
+  zraw = __ldg(zp);
+}
+// packed fp16 scale | z << 16 of stage s from its two loaded words
+__device__ __forceinline__ uint32_t sz_of(const TC5Params& p, int s, uint32_t sraw, uint32_t zraw) {
+  const int b = (s * 64) >> p.block_shift;
+  const uint32_t z = p.zeros ? (zraw >> ((b & 1) * 4)) & 15u : 8u;
+  return (sraw & 0xFFFFu) | (z << 16);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t bytes) {
@@ -407,10 +418,13 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
     const int rl = tid & 127, h = tid >> 7;  // weight row (TMEM lane) and which 32 k of a stage
     const int row = n0 + rl;
     const float down = __int_as_float((127 - row_e) << 23);  // 2^-e of this row
-    uint32_t szr[kTc5SzAhead];
+    uint32_t sra[kTc5SzAhead], zra[kTc5SzAhead];
     if constexpr (F == Fmt::Int4) {
 #pragma unroll
-      for (int i = 0; i < kTc5SzAhead; ++i) szr[i] = i < nks ? fetch_sz(p, row, s_begin + i) : 0u;
+      for (int i = 0; i < kTc5SzAhead; ++i) {
+        sra[i] = zra[i] = 0u;
+        if (i < nks) fetch_sz(p, row, s_begin + i, sra[i], zra[i]);
+      }
     }
     int rs = 0, ru = 0;
     for (int s0 = 0; s0 < (F == Fmt::BF16 ? 0 : nks); s0 += kTc5SzAhead) {
@@ -429,15 +443,18 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
         }
         uint32_t sz = 0u;
         if constexpr (F == Fmt::Int4) {
-          sz = szr[i];
-          if (ls + kTc5SzAhead < nks) szr[i] = fetch_sz(p, row, s_begin + ls + kTc5SzAhead);
+          sz = sz_of(p, s_begin + ls, sra[i], zra[i]);
+          if (ls + kTc5SzAhead < nks) fetch_sz(p, row, s_begin + ls + kTc5SzAhead, sra[i], zra[i]);
           if (row_e) {  // s·2^-e, rounded to fp16 (exact unless it falls below the normal range)
             const uint32_t sb = __half_as_ushort(__float2half_rn(h16_to_f32(sz) * down));
             sz = (sz & 0xFFFF0000u) | sb;
           }
         }
         const uint8_t* rrow = smem + p.off_raw + rs * p.raw_bytes + rl * p.raw_pitch;
-        const uint8_t* codes = F == Fmt::Int4 ? rrow + 32 * (ls & (p.spr - 1)) : rrow + 16 + 32 * (ls & 3);
+        // int4 raw slots arrive 128-byte swizzled (16-byte chunk c of row r at
+        // c ^ (r & 7)): the 8 rows a quarter-warp reads fall in 8 different banks
+        const uint8_t* codes = F == Fmt::Int4 ? smem + p.off_raw + rs * p.raw_bytes + sw128(rl, 2 * (ls & 3) + h)
+                                              : rrow + 16 + 32 * (ls & 3);
         uint32_t o[16];
         if constexpr (F != Fmt::BF16) dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, down, o);
         uint8_t* at = smem + a * 16384;

@@ -1,0 +1,362 @@
+// gemm_v1tc.cuh — batched dequant-then-MMA on the tcgen05 tensor cores for
+// int4 weights in the B200_V1 band stream (quantization blocks of at least
+// 128 k, so every 16 × 128 tile carries one scale and one zero-point per row).
+//
+// y[m, n] = Σ_k W[n, k]·x[m, k] with W = (q - z)·s (onnx-genai PR #1000,
+// "What it does": int4 blockwise weights, fp16 scales, uint4 zero-points),
+// accumulated in fp32, one rounding to fp16.
+//
+// Layout of the work.  A CTA owns 128 weight rows (eight 16-row bands of the
+// stream: the UMMA M side), BN batch rows (the UMMA N side) and one slice of
+// K; the S CTAs of a cluster share the rows, split K and add their fp32
+// accumulators through distributed shared memory in rank order.  The CTA's
+// stream is consumed one 128-k step at a time (eight tiles, one per band):
+//   * producer warp: one bulk copy per band and step (the tiles of a band are
+//     contiguous in the stream, so no tensor map is needed for the weights),
+//     and two TMA copies of the BN × 128 activation slice, 128-byte swizzled
+//     into the UMMA K-major layout (no multicast);
+//   * sixteen dequant warps: warp w turns the tile of band w mod 8 of every
+//     step of parity w / 8 into fp16 A rows: (q - z) exactly through
+//     magic-number codes, times s in one fp16 rounding (as the 64-k kernel
+//     does).  The tile's codes are in warp-MMA fragment order, so a lane holds
+//     8 consecutive k of two rows per 32-bit word and writes them as one
+//     16-byte chunk of the swizzled A tile; lanes with odd row index take the
+//     two words of a pair in the opposite order, so the eight lanes of a
+//     quarter-warp always write eight different bank groups;
+//   * MMA warp: eight tcgen05.mma (K = 16) per step into one of two fp32 TMEM
+//     accumulators (even / odd steps), each commit freeing the step's A and
+//     activation slots.
+// Rows whose weights could pass the fp16 range (15·max|s| > 65504 over the
+// row's blocks) are formed as w·2^-e and their result multiplied by 2^e, as
+// in the 64-k kernel.  Every mbarrier wait is bounded (wq_device.cuh).
+#pragma once
+
+#include "gemm_tc5.cuh"
+
+namespace wq {
+
+struct V1TCParams {
+  CUtensorMap tmap_x;  // activations [M][K] fp16, box BN rows × 64, 128-byte swizzle
+  const uint8_t* w;    // B200_V1 int4 stream
+  void* y;             // [M, N] fp16
+  int M, N, K;
+  int n_bands;         // ceil(N / 16)
+  int tpb;             // tiles (128-k steps) per band
+  int tb;              // bytes per tile
+  int BN;              // batch tile (UMMA N), multiple of 16, <= 128
+  int tmem_cols;       // power of two >= max(32, 2·BN)
+  int S;               // CTAs of a cluster (K slices)
+  int nks;             // steps per CTA (tpb / S, even)
+  int NA, NR, NX;      // A slots (32 KB), raw slots (8 bands × T tiles), activation slots (BN × 256 B)
+  int T;               // 128-k steps per raw slot: one copy of T consecutive tiles per band
+  int off_x, off_raw, off_rowe, off_bar;  // shared-memory offsets (A slots start at 0)
+};
+
+constexpr int kV1TCWarps = 18;  // 16 dequant / epilogue warps, producer, MMA issuer
+constexpr int kV1TCA = 32768;   // bytes of one A slot: 128 rows × 128 k fp16 (two 64-k atoms)
+
+// One int4 B200_V1 tile (16 rows × 128 k) at tp into rows 16·band.. of the A
+// slot at ab (two 128-byte-swizzled 64-k atoms).  s2: the two rows' scales as
+// fp16 pairs (already multiplied by 2^-e where needed).
+__device__ __forceinline__ void v1tc_tile_to_a(const uint8_t* tp, uint8_t* ab, int band, int lane, uint32_t s2g,
+                                               uint32_t s2g8) {
+  const int g = lane >> 2, t = lane & 3, odd = g & 1;
+  // word pairs (row g, row g + 8) of gi = 0..3, gi ^ odd at position j
+  const uint2 w0 = *reinterpret_cast<const uint2*>(tp + lane * 16 + 8 * odd);
+  const uint2 w1 = *reinterpret_cast<const uint2*>(tp + lane * 16 + 8 * (1 - odd));
+  const uint2 w2 = *reinterpret_cast<const uint2*>(tp + 512 + lane * 16 + 8 * odd);
+  const uint2 w3 = *reinterpret_cast<const uint2*>(tp + 512 + lane * 16 + 8 * (1 - odd));
+  const uint2 zz = *reinterpret_cast<const uint2*>(tp + 1056);
+  const uint32_t z0 = (zz.x >> (4 * g)) & 15u, z1 = (zz.y >> (4 * g)) & 15u;
+  const uint32_t zl0 = (0x6400u | z0) * 0x00010001u, zl1 = (0x6400u | z1) * 0x00010001u;
+  const uint32_t zh0 = (0x5400u | (z0 << 4)) * 0x00010001u, zh1 = (0x5400u | (z1 << 4)) * 0x00010001u;
+  const uint32_t wg[4] = {w0.x, w1.x, w2.x, w3.x}, wg8[4] = {w0.y, w1.y, w2.y, w3.y};
+  const int r0 = 16 * band + g, r1 = r0 + 8;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int gi = j ^ odd;             // the word's 32-k group: k = 32·gi + 8·t .. + 7
+    const int c = 4 * (gi & 1) + t;     // its 16-byte chunk inside the 64-k atom
+    uint8_t* atom = ab + (j >> 1) * 16384;  // gi >> 1 == j >> 1
+    {
+      const uint32_t a = wg[j], a8 = a >> 8;
+      const uint4 o = make_uint4(hmul2_f(hsub2_f(lop3_or(a, 0x000F000Fu, 0x64006400u), zl0), s2g),
+                                 hmul2_f(hsub2_f(lop3_or(a, 0x00F000F0u, 0x54005400u), zh0), s2g),
+                                 hmul2_f(hsub2_f(lop3_or(a8, 0x000F000Fu, 0x64006400u), zl0), s2g),
+                                 hmul2_f(hsub2_f(lop3_or(a8, 0x00F000F0u, 0x54005400u), zh0), s2g));
+      *reinterpret_cast<uint4*>(atom + sw128(r0, c)) = o;
+    }
+    {
+      const uint32_t a = wg8[j], a8 = a >> 8;
+      const uint4 o = make_uint4(hmul2_f(hsub2_f(lop3_or(a, 0x000F000Fu, 0x64006400u), zl1), s2g8),
+                                 hmul2_f(hsub2_f(lop3_or(a, 0x00F000F0u, 0x54005400u), zh1), s2g8),
+                                 hmul2_f(hsub2_f(lop3_or(a8, 0x000F000Fu, 0x64006400u), zl1), s2g8),
+                                 hmul2_f(hsub2_f(lop3_or(a8, 0x00F000F0u, 0x54005400u), zh1), s2g8));
+      *reinterpret_cast<uint4*>(atom + sw128(r1, c)) = o;
+    }
+  }
+}
+
+// 2^-e for the fp16 range of a row whose largest |scale| has bits smax (0x7FFF-masked, finite)
+__device__ __forceinline__ int v1tc_row_exponent(uint32_t smax) {
+  float bound = 15.f * h16_to_f32(smax);
+  int e = 0;
+  while (bound > 65504.f) {
+    bound *= 0.5f;
+    ++e;
+  }
+  return e;
+}
+
+__global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __grid_constant__ V1TCParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  uint64_t* raw_empty = raw_full + p.NR;
+  uint64_t* x_full = raw_empty + p.NR;
+  uint64_t* x_empty = x_full + p.NX;
+  uint64_t* a_full = x_empty + p.NX;
+  uint64_t* a_empty = a_full + p.NA;
+  uint64_t* done = a_empty + p.NA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* rowe = reinterpret_cast<int*>(smem + p.off_rowe);  // [128] exponent e of each tile row
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = p.S > 1 ? tc5_cluster_rank() : 0u;
+  const int tile = blockIdx.x / p.S;
+  const int n0 = tile * 128, b0 = tile * 8;
+  const int nbt = min(8, p.n_bands - b0);  // bands present in this row tile
+  const int m0 = blockIdx.y * p.BN;
+  const int s_begin = static_cast<int>(rank) * p.nks;  // first 128-k step of this CTA
+  const int nks = p.nks;
+  const int x_slot = p.BN * 256;                        // two 64-k atoms of BN rows
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(p.tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 32) {
+    for (int i = 0; i < p.NR; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 16);  // every dequant warp, once per slot
+    }
+    for (int i = 0; i < p.NX; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], 1);  // tcgen05.commit
+    }
+    for (int i = 0; i < p.NA; ++i) {
+      mbar_init(&a_full[i], 8);
+      mbar_init(&a_empty[i], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 16) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const long long band_bytes = static_cast<long long>(p.tpb) * p.tb;
+      const int nslots = (nks + p.T - 1) / p.T;
+      int issued = 0;  // raw slots issued so far
+      // raw slot r (steps [r·T, r·T + T)): one copy per band of its tiles, which
+      // are contiguous in the band's stream; issued NR - 1 slots ahead of the
+      // step whose activations are being copied
+      auto issue_raw = [&](int r) {
+        const int rs = r % p.NR, ru = r / p.NR;
+        if (ru > 0 && !mbar_wait_bounded(&raw_empty[rs], static_cast<uint32_t>((ru - 1) & 1))) return false;
+        const int nt = min(p.T, nks - r * p.T);
+        mbar_arrive_expect_tx(&raw_full[rs], static_cast<uint32_t>(nbt * nt * p.tb));
+        uint8_t* dst = smem + p.off_raw + rs * 8 * p.T * p.tb;
+        for (int i = 0; i < nbt; ++i)
+          bulk_g2s(dst + i * p.T * p.tb, p.w + (b0 + i) * band_bytes + static_cast<long long>(s_begin + r * p.T) * p.tb,
+                   static_cast<uint32_t>(nt * p.tb), &raw_full[rs]);
+        return true;
+      };
+      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+        const int gs = s_begin + ls;
+        const int xs = ls % p.NX, xu = ls / p.NX;
+        if (xu > 0 && !mbar_wait_bounded(&x_empty[xs], static_cast<uint32_t>((xu - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&x_full[xs], static_cast<uint32_t>(x_slot));
+        uint8_t* xd = smem + p.off_x + xs * x_slot;
+        tma_load_2d(xd, &p.tmap_x, gs * 128, m0, &x_full[xs]);
+        tma_load_2d(xd + x_slot / 2, &p.tmap_x, gs * 128 + 64, m0, &x_full[xs]);
+        bool okr = true;
+        while (okr && issued < nslots && issued <= ls / p.T + p.NR - 1) okr = issue_raw(issued++);
+        if (!okr) {
+          *abort_flag = 1;
+          break;
+        }
+      }
+    }
+  } else if (warp == 17) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(p.BN);
+      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+        const int a = ls % p.NA, au = ls / p.NA, xs = ls % p.NX, xu = ls / p.NX;
+        if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>(au & 1)) ||
+            !mbar_wait_bounded(&x_full[xs], static_cast<uint32_t>(xu & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dacc = tmem + static_cast<uint32_t>((ls & 1) * p.BN);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // the two 64-k atoms of the step
+          const uint64_t ad = umma_smem_desc_sw128(smem_u32(smem + a * kV1TCA + h * 16384));
+          const uint64_t bd = umma_smem_desc_sw128(smem_u32(smem + p.off_x + xs * x_slot + h * (x_slot / 2)));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
+            umma_f16(dacc, ad + 2ull * j, bd + 2ull * j, idesc, (ls > 1 || h > 0 || j > 0) ? 1u : 0u);
+        }
+        umma_commit(&a_empty[a]);
+        umma_commit(&x_empty[xs]);
+      }
+      umma_commit(done);  // arrives when every MMA issued above has completed
+    }
+  } else {
+    // ------------------------------------------------------------ dequant warps
+    const int band = warp & 7, par = warp >> 3;
+    const int g = lane >> 2, t = lane & 3;
+    const bool have = band < nbt;
+    // fp16 range of the two rows this lane writes: the largest finite |scale|
+    // over every tile of the band (all of K, so that the CTAs of a cluster agree)
+    uint32_t m_g = 0, m_g8 = 0;
+    if (have && par == 0) {
+      const uint8_t* bb = p.w + static_cast<long long>(b0 + band) * p.tpb * p.tb + 1024;
+#pragma unroll 4
+      for (int j = t; j < p.tpb; j += 4) {
+        const uint32_t a = __ldg(reinterpret_cast<const unsigned short*>(bb + static_cast<long long>(j) * p.tb) + g) & 0x7FFFu;
+        const uint32_t b = __ldg(reinterpret_cast<const unsigned short*>(bb + static_cast<long long>(j) * p.tb) + g + 8) & 0x7FFFu;
+        if (a < 0x7C00u && a > m_g) m_g = a;
+        if (b < 0x7C00u && b > m_g8) m_g8 = b;
+      }
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        m_g = max(m_g, __shfl_xor_sync(0xffffffffu, m_g, o));
+        m_g8 = max(m_g8, __shfl_xor_sync(0xffffffffu, m_g8, o));
+      }
+      if (t == 0) {
+        rowe[16 * band + g] = v1tc_row_exponent(m_g);
+        rowe[16 * band + g + 8] = v1tc_row_exponent(m_g8);
+      }
+    } else if (!have && par == 0 && t == 0) {
+      rowe[16 * band + g] = 0;
+      rowe[16 * band + g + 8] = 0;
+    }
+    asm volatile("bar.sync 1, 512;" ::: "memory");  // the 16 dequant warps: row exponents in place
+    const int e0 = rowe[16 * band + g], e1 = rowe[16 * band + g + 8];
+    const float dn0 = __int_as_float((127 - e0) << 23), dn1 = __int_as_float((127 - e1) << 23);
+    // every dequant warp visits every raw slot (count 16 on its empty barrier)
+    // and converts the slot's steps of its parity
+    for (int r = 0; r * p.T < nks && !*abort_flag; ++r) {
+      const int rs = r % p.NR, ru = r / p.NR;
+      if (!mbar_wait_bounded(&raw_full[rs], static_cast<uint32_t>(ru & 1))) {
+        *abort_flag = 1;
+        break;
+      }
+      const int l_end = min(nks, (r + 1) * p.T);
+      for (int ls = r * p.T + ((r * p.T + par) & 1); ls < l_end; ls += 2) {
+        const int a = ls % p.NA, au = ls / p.NA;
+        if (au > 0 && !mbar_wait_bounded(&a_empty[a], static_cast<uint32_t>((au - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        if (have) {
+          const uint8_t* tp = smem + p.off_raw + (rs * 8 + band) * p.T * p.tb + (ls - r * p.T) * p.tb;
+          uint32_t sg = *reinterpret_cast<const unsigned short*>(tp + 1024 + 2 * g);
+          uint32_t sg8 = *reinterpret_cast<const unsigned short*>(tp + 1024 + 2 * (g + 8));
+          if (e0) sg = __half_as_ushort(__float2half_rn(h16_to_f32(sg) * dn0));
+          if (e1) sg8 = __half_as_ushort(__float2half_rn(h16_to_f32(sg8) * dn1));
+          v1tc_tile_to_a(tp, smem + a * kV1TCA, band, lane, sg * 0x00010001u, sg8 * 0x00010001u);
+          fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        }
+        __syncwarp();
+        if (lane == 0) tc5_arrive(&a_full[a]);
+      }
+      __syncwarp();
+      if (lane == 0) tc5_arrive(&raw_empty[rs]);
+    }
+  }
+
+  // ---- epilogue: every thread waits for the last MMAs, warps 0..7 read TMEM
+  // (warp w: lanes 32(w mod 4).., column half (w / 4) mod 2)
+  bool ok = !*abort_flag && mbar_wait_bounded(done, 0u);
+  tc_fence_after();
+  const int lq = warp & 3, ch = (warp >> 2) & 1;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+  const int trow = lq * 32 + lane;  // tile row this thread reads back
+  const bool split_cols = p.BN % 32 == 0;
+  const int cols_per = split_cols ? p.BN / 2 : p.BN;
+  const int c_begin = split_cols ? ch * cols_per : 0;
+  const bool reads = warp < 8 && (split_cols || ch == 0);
+  const float row_up = __int_as_float((127 + rowe[trow & 127]) << 23);  // 2^e
+  auto acc16 = [&](int c0, float (&v)[16]) {
+    uint32_t r0[16], r1[16];
+    tmem_ld16(lane_base + c0, r0);
+    if (nks > 1) {
+      tmem_ld16(lane_base + p.BN + c0, r1);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = (__uint_as_float(r0[j]) + __uint_as_float(r1[j])) * row_up;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]) * row_up;
+    }
+  };
+  __half* y = reinterpret_cast<__half*>(p.y);
+  if (p.S == 1) {
+    if (ok && reads) {
+      for (int c0 = c_begin; c0 < c_begin + cols_per; c0 += 16) {
+        float v[16];
+        acc16(c0, v);
+        const int yrow = n0 + trow;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + c0 + j;
+          if (m < p.M && yrow < p.N) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(v[j]);
+        }
+      }
+    }
+  } else {
+    // K split over the cluster: park the fp32 tile [128][BN] in this CTA's
+    // shared memory (the rings are drained), then each rank adds 128/S rows
+    // over all ranks in rank order
+    float* acc = reinterpret_cast<float*>(smem);
+    __syncthreads();
+    if (reads) {
+      for (int c0 = c_begin; c0 < c_begin + cols_per; c0 += 16) {
+        float v[16];
+        if (ok) acc16(c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[trow * p.BN + c0 + j] = ok ? v[j] : 0.f;
+      }
+    }
+    tc5_cluster_sync();
+    const int rows_per = 128 / p.S;
+    const int items = rows_per * p.BN;
+    for (int i = tid; i < items; i += kV1TCWarps * 32) {
+      const int rr = static_cast<int>(rank) * rows_per + i / p.BN, c = i % p.BN;
+      float sum = 0.f;
+      for (int q = 0; q < p.S; ++q) sum += tc5_dsmem_ld(acc + rr * p.BN + c, static_cast<uint32_t>(q));
+      const int m = m0 + c, yrow = n0 + rr;
+      if (m < p.M && yrow < p.N && !*abort_flag) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(sum);
+    }
+    tc5_cluster_sync();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols) : "memory");
+}
+
+}  // namespace wq

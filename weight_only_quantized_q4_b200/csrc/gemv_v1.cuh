@@ -43,6 +43,8 @@ struct V1Params {
   int tpb;           // tiles per band (K / 128)
   int tpc;           // tiles per band handled by one CTA (tpb / C)
   int tps;           // tiles per stage (a multiple of W)
+  int tps0;          // tiles of the first stage (a multiple of W, <= tps): a small first
+                     // stage lands sooner after the wait for the previous kernel
   int tb;            // bytes per tile
   int NS;            // ring depth
   int stage_bytes;   // tps · tb
@@ -51,6 +53,7 @@ struct V1Params {
   int hint;          // 1: weight copies carry the L2 evict-first policy
   int pre;           // stages copied to shared memory before waiting for the previous kernel
   int pf_bytes;      // bytes of the CTA's stream prefetched into L2 before that wait (pre == 0)
+  int pfd;           // after the wait: stage S + pfd is prefetched into L2 as stage S is copied (0: off)
   int Mp;            // M rounded up to even (stride of a partial row)
   int off_x;         // activations [M][tpc·128] fp16
   int off_zero;      // 256 zero bytes
@@ -203,7 +206,10 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
   const int b_end = static_cast<int>(static_cast<long long>(cid + 1) * p.n_bands / n_cl);
   const int n_bl = b_end - b_begin;
   const int n_tiles = n_bl * p.tpc;                   // this CTA's linear tile sequence
-  const int n_stages = (n_tiles + p.tps - 1) / p.tps;
+  // stage S covers tiles [stage_first(S), stage_first(S) + stage_tiles(S)) of the sequence
+  const int n_stages = n_tiles <= p.tps0 ? 1 : 1 + (n_tiles - p.tps0 + p.tps - 1) / p.tps;
+  auto stage_first = [&](int S) { return S == 0 ? 0 : p.tps0 + (S - 1) * p.tps; };
+  auto stage_tiles = [&](int S) { return min(S == 0 ? p.tps0 : p.tps, n_tiles - stage_first(S)); };
   const int Kc = p.tpc * 128;                         // this CTA's k extent
 
   if (tid == 0) {
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
           *abort_flag = 1;
           break;
         }
-        const int nt = min(p.tps, n_tiles - S * p.tps);
+        const int nt = stage_tiles(S);
         mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nt) * p.tb);
         uint8_t* dst = smem + slot * p.stage_bytes;
         for (int left = nt; left > 0;) {  // one copy per run of tiles inside one band
@@ -278,6 +284,15 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
             ti = 0;
             ++bl;
           }
+        }
+        // keep more of the stream in flight than the ring holds: move the
+        // tiles of stage S + pfd from HBM to L2 now (C = 1: the CTA's tiles
+        // are one contiguous range), so their copy into the ring later is an
+        // L2 read
+        if (p.pfd > 0 && p.C == 1 && S + p.pfd < n_stages) {
+          const uint8_t* src = base + static_cast<long long>(stage_first(S + p.pfd)) * p.tb;
+          const long long nb = static_cast<long long>(stage_tiles(S + p.pfd)) * p.tb;
+          for (long long o = 0; o < nb; o += 32768) prefetch_l2(src + o, static_cast<uint32_t>(min(nb - o, 32768ll)));
         }
         if (++slot == p.NS) {
           slot = 0;
@@ -321,35 +336,30 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
     float* xs = reinterpret_cast<float*>(smem + p.off_xs);
     uint8_t* xsm = smem + p.off_x;
     uint8_t* zbuf = smem + p.off_zero;  // 256 zero bytes: the activations of lanes past M
-    // Σx per (tile, batch column) of this CTA's k-range: four threads per tile
-    // and column, 32 k each
+    // Σx per (tile, batch column) of this CTA's k-range: sixteen threads per
+    // tile and column, each adding 8 consecutive activations (consecutive
+    // threads read consecutive 16-byte chunks: no bank conflicts), then four
+    // shuffles within the 16
     bool ok = mbar_wait_bounded(xbar, 0u);
     if (!ok) *abort_flag = 1;
     {
-      const int items = ZQ ? 0 : p.tpc * p.M * 4;
+      const int items = ZQ ? 0 : p.tpc * p.M * 16;
       for (int b0 = 0; b0 < items; b0 += nthr) {
         const int i = b0 + tid;
         float sum = 0.f;
+        const int tm = i >> 4, m = tm % p.M, ti = tm / p.M;
         if (i < items && ok) {
-          const int q = i & 3, tm = i >> 2, m = tm % p.M, ti = tm / p.M;
-          const uint4* src = reinterpret_cast<const uint4*>(xsm + (static_cast<long long>(m) * Kc + ti * 128 + q * 32) * 2);
+          const uint4 v = *reinterpret_cast<const uint4*>(xsm + (static_cast<long long>(m) * Kc + ti * 128 + (i & 15) * 8) * 2);
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 v = src[c];
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[e]));
-              sum += f.x + f.y;
-            }
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[e]));
+            sum += f.x + f.y;
           }
         }
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (i < items && (i & 3) == 0) {
-          const int tm = i >> 2, m = tm % p.M, ti = tm / p.M;
-          xs[ti * 8 + m] = sum * 5.9604644775390625e-08f;  // ×2^-24, exact
-        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (i < items && (i & 15) == 0) xs[ti * 8 + m] = sum * 5.9604644775390625e-08f;  // ×2^-24, exact
       }
       for (int i = tid; i < p.tpc * 8; i += nthr)
         if ((i & 7) >= p.M) xs[i] = 0.f;
@@ -396,7 +406,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
       } else {
         ok = false;
       }
-      const int nt = min(p.tps, n_tiles - S * p.tps);
+      const int nt = stage_tiles(S);
       const uint8_t* st = smem + slot * p.stage_bytes;
       for (int u = warp; u < nt; u += W) {
         while (cur_bl < bl) {  // this warp's tiles moved on to a later band
