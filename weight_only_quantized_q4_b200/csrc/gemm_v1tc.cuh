@@ -229,32 +229,59 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
     const int band = warp & 7, par = warp >> 3;
     const int g = lane >> 2, t = lane & 3;
     const bool have = band < nbt;
-    // fp16 range of the two rows this lane writes: the largest finite |scale|
-    // over every tile of the band (all of K, so that the CTAs of a cluster agree)
-    uint32_t m_g = 0, m_g8 = 0;
-    if (have && par == 0) {
+    // fp16 range of every row: the largest finite |scale| over every tile of
+    // the band (all of K, so that the CTAs of a cluster agree).  The two warps
+    // of a band split its tiles; each lane loads the 32 scale bytes of its
+    // tiles with two 16-byte loads, all issued before any is used; the warps
+    // reduce per row and meet in shared memory.
+    uint32_t* rmax = reinterpret_cast<uint32_t*>(rowe);  // [128] row maxima, then exponents in place
+    if (tid < 128) rmax[tid] = 0u;
+    asm volatile("bar.sync 1, 512;" ::: "memory");
+    if (have) {
       const uint8_t* bb = p.w + static_cast<long long>(b0 + band) * p.tpb * p.tb + 1024;
-#pragma unroll 4
-      for (int j = t; j < p.tpb; j += 4) {
-        const uint32_t a = __ldg(reinterpret_cast<const unsigned short*>(bb + static_cast<long long>(j) * p.tb) + g) & 0x7FFFu;
-        const uint32_t b = __ldg(reinterpret_cast<const unsigned short*>(bb + static_cast<long long>(j) * p.tb) + g + 8) & 0x7FFFu;
-        if (a < 0x7C00u && a > m_g) m_g = a;
-        if (b < 0x7C00u && b > m_g8) m_g8 = b;
+      uint32_t mx[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) mx[r] = 0u;
+      constexpr int kPer = 4;  // tiles per lane per round (loads in flight)
+      for (int j0 = 2 * lane + par; j0 < p.tpb; j0 += 64 * kPer) {
+        uint4 v[kPer][2];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int j = j0 + 64 * u;
+          if (j < p.tpb) {
+            v[u][0] = __ldg(reinterpret_cast<const uint4*>(bb + static_cast<long long>(j) * p.tb));
+            v[u][1] = __ldg(reinterpret_cast<const uint4*>(bb + static_cast<long long>(j) * p.tb + 16));
+          } else {
+            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t wv[4] = {v[u][hh].x, v[u][hh].y, v[u][hh].z, v[u][hh].w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t m = (wv[q >> 1] >> (16 * (q & 1))) & 0x7FFFu;
+              const int r = 8 * hh + q;
+              if (m < 0x7C00u && m > mx[r]) mx[r] = m;
+            }
+          }
       }
 #pragma unroll
-      for (int o = 1; o < 4; o <<= 1) {
-        m_g = max(m_g, __shfl_xor_sync(0xffffffffu, m_g, o));
-        m_g8 = max(m_g8, __shfl_xor_sync(0xffffffffu, m_g8, o));
+      for (int r = 0; r < 16; ++r) {
+        const uint32_t m = __reduce_max_sync(0xffffffffu, mx[r]);
+        if (lane == 0) atomicMax(&rmax[16 * band + r], m);
       }
-      if (t == 0) {
-        rowe[16 * band + g] = v1tc_row_exponent(m_g);
-        rowe[16 * band + g + 8] = v1tc_row_exponent(m_g8);
-      }
-    } else if (!have && par == 0 && t == 0) {
-      rowe[16 * band + g] = 0;
-      rowe[16 * band + g + 8] = 0;
     }
-    asm volatile("bar.sync 1, 512;" ::: "memory");  // the 16 dequant warps: row exponents in place
+    asm volatile("bar.sync 1, 512;" ::: "memory");
+    if (par == 0 && t == 0) {
+      const int e_g = v1tc_row_exponent(rmax[16 * band + g]), e_g8 = v1tc_row_exponent(rmax[16 * band + g + 8]);
+      __syncwarp(0x11111111u);
+      rowe[16 * band + g] = e_g;
+      rowe[16 * band + g + 8] = e_g8;
+    }
+    asm volatile("bar.sync 1, 512;" ::: "memory");  // the row exponents are in place
     const int e0 = rowe[16 * band + g], e1 = rowe[16 * band + g + 8];
     const float dn0 = __int_as_float((127 - e0) << 23), dn1 = __int_as_float((127 - e1) << 23);
     // every dequant warp visits every raw slot (count 16 on its empty barrier)
