@@ -68,6 +68,9 @@ for _M in (1, 2, 4, 8):
     for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336)):
         WORKLOADS[f"int4_b128_zp_v1_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 3, 0.002, 0.01, layout=1)
 
+for _M in (1, 2, 4, 8):
+    for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336)):
+        WORKLOADS[f"mxfp4_m{_M}_{_N}x{_K}"] = dict(fmt="mxfp4", M=_M, N=_N, K=_K, workload=6)
 for _M in (16, 32, 64, 128):
     for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336), (32000, 4096)):
         WORKLOADS[f"batched_int4_b128_zp_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 5, 0.002, 0.01)
@@ -83,7 +86,7 @@ SWEEP = ["q4k_v1_m1_4096x11008", "q4k_v1_m4_4096x11008", "q4k_v1_m1_11008x4096",
          "int4_b128_zp_v1_m1_14336x4096", "int4_b128_zp_v1_m1_4096x4096",
          "int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
          "int4_b32_m1_256x1024", "q4k_m1_4096x11008", "q4k_dsc_m1_4096x11008", "q4k_m4_11008x4096",
-         "q4k_m8_4096x4096", "bf16_m1_1536x6912", "bf16_m3_1536x6912", "bf16_m8_1536x6912", "bf16_m1_151936x1536"]
+         "q4k_m8_4096x4096", "mxfp4_m1_4096x14336", "mxfp4_m4_4096x14336", "bf16_m1_1536x6912", "bf16_m3_1536x6912", "bf16_m8_1536x6912", "bf16_m1_151936x1536"]
 
 
 def weight_bytes(w) -> int:
@@ -94,11 +97,14 @@ def weight_bytes(w) -> int:
         return N * K // 2 + 2 * N * nb + (N * ((nb + 1) // 2) if w["zeros"] else 0)
     if w["fmt"] == "q4k":
         return N * K // 2 + N * K // 4 if w["dsc"] else N * (K // 256) * 144
+    if w["fmt"] == "mxfp4":
+        return N * K // 2 + N * K // 32
     return 2 * N * K
 
 
 def dtype_of(w) -> str:
-    return {"int4": "int4xf16->f32", "q4k": "q4kxf16->f32", "bf16": "bf16xbf16->f32"}[w["fmt"]]
+    return {"int4": "int4xf16->f32", "q4k": "q4kxf16->f32", "bf16": "bf16xbf16->f32",
+            "mxfp4": "mxfp4xf16->f32"}[w["fmt"]]
 
 
 def host_inputs(w):
@@ -111,6 +117,8 @@ def host_inputs(w):
     if w["fmt"] == "q4k":
         return dict(x=synth.activations_f16(M, K, workload=w["workload"]),
                     raw=synth.q4k_weights(N, K, workload=w["workload"]))
+    if w["fmt"] == "mxfp4":
+        return dict(x=synth.activations_f16(M, K, workload=w["workload"]), **synth.mxfp4_weights(N, K, workload=w["workload"]))
     return dict(x=synth.activations_bf16_bits(M, K, workload=w["workload"]),
                 w=synth.bf16_weights_bits(N, K, workload=w["workload"]))
 
@@ -214,6 +222,12 @@ class DeviceWorkload:
                 self.copies.append(c)
             self.x = torch.from_numpy(host["x"]).to(dev)
             self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        elif w["fmt"] == "mxfp4":
+            base = [torch.from_numpy(host["w_packed"]).to(dev), torch.from_numpy(host["scales"]).to(dev)]
+            for _ in range(self.R):
+                self.copies.append([t.clone() for t in base])
+            self.x = torch.from_numpy(host["x"]).to(dev)
+            self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
         else:
             wt = torch.from_numpy(host["w"].view(np.int16)).to(dev).view(torch.bfloat16)
             for _ in range(self.R):
@@ -246,6 +260,8 @@ class DeviceWorkload:
                 wq.gemv_q4k_dsc(x, c[0], c[1], y, M, self.N, self.K, stream=stream)
             else:
                 wq.gemv_q4k(x, c[0], y, M, self.N, self.K, layout=w.get("layout", 0), stream=stream)
+        elif w["fmt"] == "mxfp4":
+            wq.gemv_mxfp4(x, c[0], c[1], y, M, self.N, self.K, stream=stream)
         else:
             wq.gemv_bf16(x, c[0], y, M, self.N, self.K, stream=stream)
 
@@ -553,6 +569,9 @@ def cpu_baseline(w, host, budget_s=15.0):
                 W = oracle.dequant_q4k_from_plane(host["raw"][r], P, len(r), K)
             else:
                 W = oracle.dequant_q4k(host["raw"][r], len(r), K)
+            xv = x.astype(np.float64)
+        elif w["fmt"] == "mxfp4":
+            W = oracle.dequant_mxfp4(host["w_packed"][r], host["scales"][r], len(r), K)
             xv = x.astype(np.float64)
         else:
             W = oracle.dequant_bf16(host["w"][r], len(r), K)

@@ -41,7 +41,7 @@
  *  - The first call on a device configures kernel attributes and looks up the
  *    driver's tensor-map encoder; make it before capturing a CUDA graph.
  *  - Environment variables read at each call, for tests and tuning only:
- *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc) pins a kernel
+ *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc | mx) pins a kernel
  *    family (a call that family cannot run returns WQ_ERR_UNSUPPORTED; there
  *    is no silent substitute), WQ_PDL=0 disables programmatic dependent
  *    launch, and WQ_V1_*, WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch
@@ -196,6 +196,21 @@ int gemv_q4k_dsc(const void* x_f16, const void* w_q4k, const void* w_dsc, void* 
 int gemv_bf16(const void* x_bf16, const void* w_bf16, void* y_bf16, int M, int N, int K,
               void* stream);
 
+/* y[M,N] fp16 = x[M,K] fp16 · W[N,K]ᵀ, W mxfp4 blockwise (onnx-genai PR #1000,
+ * CPU criterion bench block: the mxfp4 block-quantized matmul rows; the page
+ * does not print the format, the reading is the OCP microscaling FP4
+ * definition): blocks of 32 elements along K share one E8M0 scale byte E,
+ * value 2^(E - 127) (E = 255 is NaN), and every element is a 4-bit E2M1 code
+ * (bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa; values 0, 0.5,
+ * 1, 1.5, 2, 3, 4, 6 and their negatives).
+ *   w_packed     codes [N][K/2] bytes, low nibble = even k (16-byte aligned)
+ *   scales_e8m0  [N][K/32] bytes (any alignment)
+ * K % 32 == 0 (else WQ_ERR_ARG).  fp32 accumulation; each block's scale is
+ * applied in fp32.  Batches past 8 rows run in chunks of 8 (W read once per
+ * chunk).  WQ_FORCE_KERNEL other than "mx" returns WQ_ERR_UNSUPPORTED. */
+int gemv_mxfp4(const void* x_f16, const void* w_packed, const void* scales_e8m0, void* y_f16, int M, int N, int K,
+               void* stream);
+
 /* ---------------------------------------------------------------------------
  * Device dequantization exports: w_out [N,K] fp32 row-major, through the same
  * device unpacking code the GEMV kernels use.  Every value is exact (the
@@ -210,6 +225,11 @@ int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const v
  * then be NULL). */
 int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K, int layout,
                 void* stream);
+
+/* mxfp4: w_out[n][k] = 2^(E - 127)·e2m1(q) exactly in fp32 (a value past the
+ * fp32 range is ±inf; E = 255 gives NaN).  K % 32 == 0; w_packed and w_out
+ * 16-byte aligned. */
+int dequant_mxfp4(const void* w_packed, const void* scales_e8m0, float* w_out, int N, int K, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Weight packing (load time).

@@ -13,10 +13,12 @@ from .api import (  # noqa: F401
     WQ_LAYOUT_CANONICAL,
     WQError,
     dequant_int4_blockwise,
+    dequant_mxfp4,
     dequant_q4k,
     gemv_bf16,
     gemv_int4_blockwise,
     gemv_int4_swiglu,
+    gemv_mxfp4,
     gemv_q4k,
     gemv_q4k_dsc,
     gemv_q4k_noalloc,

@@ -34,11 +34,13 @@ SIGNATURES = {
     "gemv_q4k_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "gemv_q4k_dsc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "gemv_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "gemv_mxfp4": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "gemv_int4_swiglu": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "wq_repack_int4_gate_up": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "wq_int4_gate_up_packed_bytes": (_sz, [_i, _i, _i, _i]),
     "dequant_int4_blockwise": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "dequant_q4k": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "dequant_mxfp4": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
     "wq_int4_bytes": (_sz, [_i, _i, _i, _i]),
     "wq_int4_codes_bytes": (_sz, [_i, _i, _i]),
     "wq_repack_int4": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),

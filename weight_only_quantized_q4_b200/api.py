@@ -86,6 +86,14 @@ def dequant_int4_blockwise(w_packed, scales, zeros, w_out, N, K, block_size, lay
                                         layout, _stream(stream)), "dequant_int4_blockwise")
 
 
+def gemv_mxfp4(x, w_packed, scales, y, M, N, K, stream=None):
+    _check(lib().gemv_mxfp4(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(y), M, N, K, _stream(stream)), "gemv_mxfp4")
+
+
+def dequant_mxfp4(w_packed, scales, w_out, N, K, stream=None):
+    _check(lib().dequant_mxfp4(_ptr(w_packed), _ptr(scales), _ptr(w_out), N, K, _stream(stream)), "dequant_mxfp4")
+
+
 def dequant_q4k(w_q4k, w_dsc, w_out, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
     _check(lib().dequant_q4k(_ptr(w_q4k), _ptr(w_dsc), _ptr(w_out), N, K, layout, _stream(stream)), "dequant_q4k")
 

@@ -26,6 +26,7 @@
 #include "gemv_v1k.cuh"
 #include "gemm_tc5.cuh"
 #include "gemm_v1tc.cuh"
+#include "gemv_mxfp4.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -1572,6 +1573,56 @@ int gemv_bf16(const void* x_bf16, const void* w_bf16, void* y_bf16, int M, int N
   const bool fast = aligned16(x_bf16) && aligned16(w_bf16) && (K % 8) == 0;
   return run_gemv<Fmt::BF16>("bf16", x_bf16, static_cast<const uint8_t*>(w_bf16), nullptr, nullptr, nullptr, y_bf16,
                              M, N, K, 2ll * K, 0, 0, 0, fast, static_cast<cudaStream_t>(stream));
+}
+
+int gemv_mxfp4(const void* x_f16, const void* w_packed, const void* scales_e8m0, void* y_f16, int M, int N, int K,
+               void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (K % 32) return fail(WQ_ERR_ARG, "gemv_mxfp4: K must be a multiple of 32");
+  if (!x_f16 || !w_packed || !scales_e8m0 || !y_f16) return fail(WQ_ERR_ARG, "gemv_mxfp4: null pointer");
+  if (!aligned16(x_f16) || !aligned16(w_packed) || !aligned2(y_f16))
+    return fail(WQ_ERR_ALIGN, "gemv_mxfp4: x and w_packed must be 16-byte aligned, y 2-byte aligned");
+  if (const char* force = forced_variant())
+    if (std::strcmp(force, "mx") != 0)
+      return fail(WQ_ERR_UNSUPPORTED, std::string("WQ_FORCE_KERNEL=") + force + ": mxfp4 has one kernel family (mx)");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int m0 = 0; m0 < M; m0 += 8) {  // batches past 8 rows run in chunks of 8 (W is read once per chunk)
+    MXParams p{};
+    p.x = static_cast<const uint8_t*>(x_f16) + static_cast<long long>(m0) * K * 2;
+    p.w = static_cast<const uint8_t*>(w_packed);
+    p.scales = static_cast<const uint8_t*>(scales_e8m0);
+    p.y = static_cast<uint8_t*>(y_f16) + static_cast<long long>(m0) * N * 2;
+    p.M = std::min(8, M - m0);
+    p.N = N;
+    p.K = K;
+    gemv_mxfp4_kernel<<<(N + 15) / 16, kMXWarps * 32, 0, st>>>(p);
+    if ((rc = launch_check("gemv_mxfp4 launch"))) return rc;
+  }
+  char buf[64];
+  std::snprintf(buf, sizeof(buf), "mxfp4.gemv.mx.m%d%s", std::min(8, M), M > 8 ? ".chunked" : "");
+  set_last_kernel(buf);
+  return WQ_OK;
+}
+
+int dequant_mxfp4(const void* w_packed, const void* scales_e8m0, float* w_out, int N, int K, void* stream) {
+  int rc = check_dims(1, N, K);
+  if (rc) return rc;
+  if (K % 32) return fail(WQ_ERR_ARG, "dequant_mxfp4: K must be a multiple of 32");
+  if (!w_packed || !scales_e8m0 || !w_out) return fail(WQ_ERR_ARG, "dequant_mxfp4: null pointer");
+  if (!aligned16(w_packed) || !aligned16(w_out))
+    return fail(WQ_ERR_ALIGN, "dequant_mxfp4: w_packed and w_out must be 16-byte aligned");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  const long long bytes = static_cast<long long>(N) * (K / 2);
+  const int grid = static_cast<int>(std::min<long long>((bytes + 255) / 256, di.sms * 32ll));
+  dequant_mxfp4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_packed), static_cast<const uint8_t*>(scales_e8m0), w_out, N, K);
+  if ((rc = launch_check("dequant_mxfp4 launch"))) return rc;
+  set_last_kernel("mxfp4.dequant");
+  return WQ_OK;
 }
 
 int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const void* zeros_u4, float* w_out, int N,

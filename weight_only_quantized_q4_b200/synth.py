@@ -114,3 +114,14 @@ def with_element_offset(a: np.ndarray, offset: int) -> tuple[np.ndarray, np.ndar
     buf = np.zeros(flat.size + offset + 8, dtype=flat.dtype)
     buf[offset:offset + flat.size] = flat
     return buf, buf[offset:offset + flat.size].reshape(a.shape)
+
+
+def mxfp4_weights(N: int, K: int, *, workload: int = 6, e_lo: int = 121, e_hi: int = 129) -> dict:
+    """mxfp4 blockwise weights: codes uint8 [N, K/2] (uniform bytes: every E2M1
+    code, both signs), E8M0 scale bytes uint8 [N, K/32] uniform in [e_lo, e_hi]
+    (2^-6 .. 2^2 with the defaults)."""
+    if K % 32:
+        raise ValueError("mxfp4 needs K % 32 == 0")
+    w = _rng(workload, TENSOR_W).integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = _rng(workload, TENSOR_SCALE).integers(e_lo, e_hi + 1, size=(N, K // 32), dtype=np.uint8)
+    return {"w_packed": w, "scales": s}
