@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kMXWarps * 32) gemv_mxfp4_kernel(const MXParam
   const bool xrow = g < p.M;
   const __half* xr = reinterpret_cast<const __half*>(p.x) + static_cast<long long>(xrow ? g : 0) * p.K + 8 * t;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  constexpr int kU = 4;  // blocks in flight per warp
+  constexpr int kU = 8;  // blocks in flight per warp
   for (int b0 = warp; b0 < nb; b0 += kMXWarps * kU) {
     uint32_t c0[kU], c1[kU], e0[kU], e1[kU];
     uint4 xv[kU];
