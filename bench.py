@@ -71,6 +71,7 @@ for _M in (1, 2, 4, 8):
 for _M in (1, 2, 4, 8):
     for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336)):
         WORKLOADS[f"mxfp4_m{_M}_{_N}x{_K}"] = dict(fmt="mxfp4", M=_M, N=_N, K=_K, workload=6)
+    WORKLOADS[f"swiglu_b128_zp_m{_M}_14336x4096"] = dict(fmt="swiglu", M=_M, N=14336, K=4096, bs=128, workload=7)
 for _M in (16, 32, 64, 128):
     for _N, _K in ((4096, 4096), (14336, 4096), (4096, 14336), (32000, 4096)):
         WORKLOADS[f"batched_int4_b128_zp_m{_M}_{_N}x{_K}"] = _int4(_M, _N, _K, 128, True, 5, 0.002, 0.01)
@@ -99,12 +100,15 @@ def weight_bytes(w) -> int:
         return N * K // 2 + N * K // 4 if w["dsc"] else N * (K // 256) * 144
     if w["fmt"] == "mxfp4":
         return N * K // 2 + N * K // 32
+    if w["fmt"] == "swiglu":  # gate and up: two int4 tensors of N x K
+        nb = K // w["bs"]
+        return 2 * (N * K // 2 + 2 * N * nb + N * ((nb + 1) // 2))
     return 2 * N * K
 
 
 def dtype_of(w) -> str:
     return {"int4": "int4xf16->f32", "q4k": "q4kxf16->f32", "bf16": "bf16xbf16->f32",
-            "mxfp4": "mxfp4xf16->f32"}[w["fmt"]]
+            "mxfp4": "mxfp4xf16->f32", "swiglu": "int4xf16->f32"}[w["fmt"]]
 
 
 def host_inputs(w):
@@ -119,6 +123,10 @@ def host_inputs(w):
                     raw=synth.q4k_weights(N, K, workload=w["workload"]))
     if w["fmt"] == "mxfp4":
         return dict(x=synth.activations_f16(M, K, workload=w["workload"]), **synth.mxfp4_weights(N, K, workload=w["workload"]))
+    if w["fmt"] == "swiglu":
+        g = synth.int4_weights(N, K, w["bs"], scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=w["workload"])
+        u = synth.int4_weights(N, K, w["bs"], scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=w["workload"] + 50)
+        return dict(x=synth.activations_f16(M, K, workload=w["workload"]), gate=g, up=u)
     return dict(x=synth.activations_bf16_bits(M, K, workload=w["workload"]),
                 w=synth.bf16_weights_bits(N, K, workload=w["workload"]))
 
@@ -222,6 +230,14 @@ class DeviceWorkload:
                 self.copies.append(c)
             self.x = torch.from_numpy(host["x"]).to(dev)
             self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        elif w["fmt"] == "swiglu":
+            d = {h: [torch.from_numpy(host[h][k]).to(dev) for k in ("w_packed", "scales", "zeros")] for h in ("gate", "up")}
+            packed = torch.empty(wq.wq_int4_gate_up_packed_bytes(N, K, w["bs"]), dtype=torch.uint8, device=dev)
+            wq.wq_repack_int4_gate_up(*d["gate"], *d["up"], packed, N, K, w["bs"])
+            for _ in range(self.R):
+                self.copies.append([packed.clone()])
+            self.x = torch.from_numpy(host["x"]).to(dev)
+            self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
         elif w["fmt"] == "mxfp4":
             base = [torch.from_numpy(host["w_packed"]).to(dev), torch.from_numpy(host["scales"]).to(dev)]
             for _ in range(self.R):
@@ -262,6 +278,8 @@ class DeviceWorkload:
                 wq.gemv_q4k(x, c[0], y, M, self.N, self.K, layout=w.get("layout", 0), stream=stream)
         elif w["fmt"] == "mxfp4":
             wq.gemv_mxfp4(x, c[0], c[1], y, M, self.N, self.K, stream=stream)
+        elif w["fmt"] == "swiglu":
+            wq.gemv_int4_swiglu(x, c[0], y, M, self.N, self.K, w["bs"], stream=stream)
         else:
             wq.gemv_bf16(x, c[0], y, M, self.N, self.K, stream=stream)
 
@@ -573,6 +591,13 @@ def cpu_baseline(w, host, budget_s=15.0):
         elif w["fmt"] == "mxfp4":
             W = oracle.dequant_mxfp4(host["w_packed"][r], host["scales"][r], len(r), K)
             xv = x.astype(np.float64)
+        elif w["fmt"] == "swiglu":
+            Wg = oracle.dequant_int4(host["gate"]["w_packed"][r], host["gate"]["scales"][r], host["gate"]["zeros"][r],
+                                     len(r), K, w["bs"])
+            W = oracle.dequant_int4(host["up"]["w_packed"][r], host["up"]["scales"][r], host["up"]["zeros"][r],
+                                    len(r), K, w["bs"])
+            xv = x.astype(np.float64)
+            oracle.swiglu_gemv(Wg, W, xv)
         else:
             W = oracle.dequant_bf16(host["w"][r], len(r), K)
             xv = oracle.dequant_bf16(x, M, K)
