@@ -77,10 +77,14 @@ def int4_zero_points(zeros, N: int, n_blocks: int) -> np.ndarray:
 
 
 def dequant_int4(w_packed, scales, zeros, N: int, K: int, block_size: int) -> np.ndarray:
-    """W[n, k] = (q[n,k] - z[n, k//bs]) · s[n, k//bs] in float64 (exact)."""
-    if block_size <= 0 or K % block_size:
-        raise ValueError("K must be a positive multiple of block_size")
-    nb = K // block_size
+    """W[n, k] = (q[n,k] - z[n, k//bs]) · s[n, k//bs] in float64 (exact).
+
+    A row has nb = ceil(K/bs) blocks; when bs does not divide K the last one
+    covers the remaining K - (nb-1)·bs codes (ragged last block; the code
+    array keeps K/2 bytes per row, no padding)."""
+    if block_size <= 0:
+        raise ValueError("block_size must be positive")
+    nb = -(-K // block_size)
     q = int4_codes(w_packed, N, K)
     s = f16_bits_to_f64(np.asarray(scales).view(np.uint16).reshape(N, nb))
     z = int4_zero_points(zeros, N, nb)

@@ -206,7 +206,7 @@ def pin_int4_hand(o):
 
 def _brute_int4(w, s, z, N, K, bs):
     out = np.zeros((N, K))
-    nb = K // bs
+    nb = (K + bs - 1) // bs  # a shorter last block when bs does not divide K
     for n in range(N):
         for k in range(K):
             byte = int(w[n, k // 2])
@@ -229,6 +229,31 @@ def pin_int4_brute(o):
                                with_zeros=with_zeros, workload=904)
         W = o.dequant_int4(t["w_packed"], t["scales"], t["zeros"], 3, 96, 32)
         assert np.array_equal(W, _brute_int4(t["w_packed"], t["scales"], t["zeros"], 3, 96, 32))
+
+
+def pin_int4_ragged_brute(o):
+    """A ragged last block (K not a multiple of the block): element by element,
+    odd and even block counts (80 = 32+32+16, 48 = 32+16, 144 = 128+16)."""
+    for N, K, bs in ((3, 80, 32), (2, 48, 32), (2, 144, 128)):
+        for with_zeros in (True, False):
+            t = synth.int4_weights(N, K, bs, scale_lo=0.005, scale_hi=0.02,
+                                   with_zeros=with_zeros, workload=907)
+            assert t["scales"].shape == (N, -(-K // bs))
+            W = o.dequant_int4(t["w_packed"], t["scales"], t["zeros"], N, K, bs)
+            assert np.array_equal(W, _brute_int4(t["w_packed"], t["scales"], t["zeros"], N, K, bs))
+
+
+def pin_int4_ragged_is_a_prefix(o):
+    """Cutting K to a ragged length keeps the first K columns of the full-block
+    matrix: same scales and zero-points, each row's first K/2 code bytes."""
+    N, bs = 3, 64
+    Kf = 4 * bs
+    t = synth.int4_weights(N, Kf, bs, scale_lo=0.005, scale_hi=0.02, with_zeros=True, workload=908)
+    Wf = o.dequant_int4(t["w_packed"], t["scales"], t["zeros"], N, Kf, bs)
+    for K in (Kf - 16, Kf - bs + 2, 3 * bs + 32):
+        w = np.ascontiguousarray(t["w_packed"][:, :K // 2])
+        W = o.dequant_int4(w, t["scales"], t["zeros"], N, K, bs)
+        assert np.array_equal(W, Wf[:, :K])
 
 
 def pin_int4_zero_equals_code(o):
@@ -456,6 +481,8 @@ ALL_PINS = [
     pin_q4k_codes_layout,
     pin_int4_hand,
     pin_int4_brute,
+    pin_int4_ragged_brute,
+    pin_int4_ragged_is_a_prefix,
     pin_int4_zero_equals_code,
     pin_bf16_offsets_and_odd_k,
     pin_gemv_one_hot,

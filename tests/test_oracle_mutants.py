@@ -102,6 +102,15 @@ def _dequant_int4_block_off_by_one(w_packed, scales, zeros, N, K, block_size):
     return (q - z[:, blk]).astype(np.float64) * s[:, blk]
 
 
+def _dequant_int4_ragged_tail_in_last_full_block(w_packed, scales, zeros, N, K, block_size):
+    nb = -(-K // block_size)
+    q = oq.int4_codes(w_packed, N, K)
+    s = oq.f16_bits_to_f64(np.asarray(scales).view(np.uint16).reshape(N, nb))
+    z = oq.int4_zero_points(zeros, N, nb)
+    blk = np.minimum(np.arange(K) // block_size, max(K // block_size - 1, 0))
+    return (q - z[:, blk]).astype(np.float64) * s[:, blk]
+
+
 def _silu_without_a(a):
     a = np.asarray(a, dtype=np.float64)
     return 1.0 / (1.0 + np.exp(-a))
@@ -151,6 +160,7 @@ MUTANTS = {
     "int4 nibbles high-first": ("int4_codes", _int4_codes_high_first),
     "int4 default zero-point 0": ("int4_zero_points", _zero_points_default_zero),
     "int4 block index off by one": ("dequant_int4", _dequant_int4_block_off_by_one),
+    "int4 ragged tail read with the last full block": ("dequant_int4", _dequant_int4_ragged_tail_in_last_full_block),
     "6-bit min from byte j-4": ("get_scale_min_k4", _scale_min_wrong_byte),
     "6-bit nibbles swapped": ("get_scale_min_k4", _scale_min_nibbles_swapped),
     "q4_K codes sequential": ("q4k_codes", _codes_sequential),

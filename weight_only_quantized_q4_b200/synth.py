@@ -62,12 +62,12 @@ def int4_weights(N: int, K: int, block_size: int, *, scale_lo: float, scale_hi: 
 
     Returns a dict with
       w_packed [N, K/2] uint8   (two codes per byte, low nibble = even k)
-      scales   [N, K/block] float16
-      zeros    [N, ceil((K/block)/2)] uint8 or None (None means z = 8)
+      scales   [N, nb] float16, nb = ceil(K/block) (the last block may be shorter)
+      zeros    [N, ceil(nb/2)] uint8 or None (None means z = 8)
     """
-    if K % block_size:
-        raise ValueError("K must be a multiple of block_size")
-    nb = K // block_size
+    if K % 2:
+        raise ValueError("K must be even (two codes per byte)")
+    nb = -(-K // block_size)
     w = _rng(workload, TENSOR_W).integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     s = _rng(workload, TENSOR_SCALE).uniform(scale_lo, scale_hi, size=(N, nb)).astype(np.float16)
     z = None
