@@ -50,10 +50,12 @@
  * Weight formats (canonical byte layouts, layout version WQ_LAYOUT_CANONICAL):
  *  - int4 MatMulNBits-style blocks (onnx-genai PR #1000, "What it does": int4
  *    blockwise weights with fp16 scales and zero-points).  w_packed is
- *    [N][K/2] bytes, two 4-bit codes per byte, low nibble = even k.  scales
- *    is [N][K/block_size] fp16.  zeros is [N][ceil((K/block_size)/2)] bytes,
- *    two uint4 zero-points per byte, low nibble = even block; NULL means
- *    z = 8 for every block.  w = (q - z)·s.
+ *    [N][K/2] bytes, two 4-bit codes per byte, low nibble = even k.  A row
+ *    has nb = ceil(K/block_size) blocks along K; when K is not a multiple of
+ *    block_size the last one is shorter (K - (nb-1)·block_size codes, no
+ *    padding in the code array).  scales is [N][nb] fp16.  zeros is
+ *    [N][ceil(nb/2)] bytes, two uint4 zero-points per byte, low nibble = even
+ *    block; NULL means z = 8 for every block.  w = (q - z)·s.
  *  - q4_K super-blocks (minfer doc 62 "r59 — q4_K W_dsc plane", §3.2): row n
  *    holds K/256 blocks of 144 bytes: fp16 d (bytes 0-1), fp16 dmin (2-3),
  *    12 bytes of packed 6-bit scales and mins (4-15), 128 bytes of 4-bit
@@ -135,7 +137,8 @@ extern "C" {
  * ------------------------------------------------------------------------- */
 
 /* y[M,N] fp16 = x[M,K] fp16 · dequant(int4)ᵀ.
- * block_size: a power of two in [16, 256] with K % block_size == 0.
+ * block_size: a power of two in [16, 256]; K % 16 == 0 (K need not be a
+ * multiple of block_size: the last block of a row is then shorter).
  * zeros_u4 may be NULL (z = 8).  layout: WQ_LAYOUT_CANONICAL, or
  * WQ_LAYOUT_B200_V1 for weights rewritten by wq_repack_int4 (then w_packed is
  * the repacked buffer and scales_f16 / zeros_u4 are ignored).

@@ -103,7 +103,11 @@ def test_size_queries():
     assert wq.wq_int4_bytes(4096, 14336, 128, 1) == 256 * 112 * 1072
     assert wq.wq_int4_bytes(256, 1024, 32) == 256 * 512 + 256 * 32 * 2 + 256 * 16
     assert wq.wq_int4_bytes(4, 96, 32) == 4 * 48 + 4 * 3 * 2 + 4 * 2  # odd block count: zero-point bytes round up
-    assert wq.wq_int4_bytes(4, 100, 32) == 0
+    assert wq.wq_int4_bytes(4, 100, 32) == 0  # K % 16 != 0
+    # a ragged last block: 80 = 32 + 32 + 16 (three blocks), 896 = 3 x 256 + 128
+    assert wq.wq_int4_bytes(4, 80, 32) == 4 * 40 + 4 * 3 * 2 + 4 * 2
+    assert wq.wq_int4_bytes(2, 896, 256) == 2 * 448 + 2 * 4 * 2 + 2 * 2
+    assert wq.wq_int4_packed_bytes(21, 896, 256) == 2 * 7 * 1072
     assert wq.wq_q4k_bytes(4096, 4096) == 4096 * 16 * 144
     assert wq.wq_q4k_dsc_bytes(4096, 11008) == 4096 * 11008 // 4
     assert wq.wq_q4k_dsc_bytes(4, 100) == 0

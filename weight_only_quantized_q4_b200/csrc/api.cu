@@ -1447,7 +1447,8 @@ int check_int4(int K, int block_size, int layout) {
     return fail(WQ_ERR_LAYOUT, "unknown int4 layout version");
   if (block_size < 16 || block_size > 256 || (block_size & (block_size - 1)))
     return fail(WQ_ERR_ARG, "block_size must be a power of two in [16, 256]");
-  if (K % block_size) return fail(WQ_ERR_ARG, "K must be a multiple of block_size");
+  // the last block of a row may be shorter (K - (nb - 1)·block_size codes)
+  if (K % 16) return fail(WQ_ERR_ARG, "int4 needs K % 16 == 0");
   if (layout == WQ_LAYOUT_B200_V1 && (K % 128 || block_size < 32))
     return fail(WQ_ERR_ARG, "the B200_V1 int4 layout needs K % 128 == 0 and block_size >= 32");
   return WQ_OK;
@@ -1483,7 +1484,7 @@ int gemv_int4_blockwise(const void* x_f16, const void* w_packed, const void* sca
   if (!aligned16(x_f16) || !aligned16(w_packed) || (scales_f16 && !aligned16(scales_f16)) || !aligned16(y_f16) ||
       (zeros_u4 && !aligned16(zeros_u4)))
     return fail(WQ_ERR_ALIGN, "gemv_int4_blockwise: device pointers must be 16-byte aligned");
-  const int nb = K / block_size;
+  const int nb = (K + block_size - 1) / block_size;
   const int zb = (nb + 1) / 2;
   const long long row_bytes = K / 2;
   const bool fast = (row_bytes % 16) == 0;
@@ -1641,7 +1642,7 @@ int dequant_int4_blockwise(const void* w_packed, const void* scales_f16, const v
     return fail(WQ_ERR_ALIGN, "dequant_int4_blockwise: device pointers must be 16-byte aligned");
   DeviceInfo di;
   if ((rc = device_info(&di))) return rc;
-  const int nb = K / block_size;
+  const int nb = (K + block_size - 1) / block_size;
   const long long words = static_cast<long long>(N) * (K / 8);
   const int grid = static_cast<int>(std::min<long long>((words + 255) / 256, di.sms * 32ll));
   dequant_int4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -1688,7 +1689,7 @@ int wq_repack_int4(const void* w_canonical, const void* scales_f16, const void* 
   if (N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "wq_repack_int4: need N, K > 0");
   if (!w_canonical || !scales_f16 || !w_out) return fail(WQ_ERR_ARG, "wq_repack_int4: null pointer");
   if (to_layout != WQ_LAYOUT_B200_V1) return fail(WQ_ERR_LAYOUT, "wq_repack_int4: target layout must be B200_V1");
-  if (block_size < 32 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size)
+  if (block_size < 32 || block_size > 256 || (block_size & (block_size - 1)) || K % 128)
     return fail(WQ_ERR_ARG, "wq_repack_int4: B200_V1 needs a power-of-two block in [32, 256] and K % 128 == 0");
   if (!aligned16(w_canonical) || !aligned16(scales_f16) || (zeros_u4 && !aligned16(zeros_u4)) || !aligned16(w_out))
     return fail(WQ_ERR_ALIGN, "wq_repack_int4: device pointers must be 16-byte aligned");
@@ -1718,7 +1719,7 @@ int wq_repack_int4_gate_up(const void* w_gate, const void* scales_gate, const vo
     return fail(WQ_ERR_ARG, "wq_repack_int4_gate_up: null pointer");
   if (to_layout != WQ_LAYOUT_B200_V1)
     return fail(WQ_ERR_LAYOUT, "wq_repack_int4_gate_up: target layout must be B200_V1");
-  if (block_size < 128 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size)
+  if (block_size < 128 || block_size > 256 || (block_size & (block_size - 1)) || K % 128)
     return fail(WQ_ERR_ARG, "wq_repack_int4_gate_up: needs block_size 128 or 256 and K % 128 == 0");
   if (!aligned16(w_gate) || !aligned16(scales_gate) || (zeros_gate && !aligned16(zeros_gate)) || !aligned16(w_up) ||
       !aligned16(scales_up) || (zeros_up && !aligned16(zeros_up)) || !aligned16(w_out))
@@ -1751,7 +1752,7 @@ int gemv_int4_swiglu(const void* x_f16, const void* w_gate_up, void* y_f16, int 
   if (rc) return rc;
   if (layout != WQ_LAYOUT_B200_V1)
     return fail(WQ_ERR_LAYOUT, "gemv_int4_swiglu: the fused gate-up stream exists in the B200_V1 layout only");
-  if (block_size < 128 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size)
+  if (block_size < 128 || block_size > 256 || (block_size & (block_size - 1)) || K % 128)
     return fail(WQ_ERR_ARG, "gemv_int4_swiglu: needs block_size 128 or 256 and K % 128 == 0");
   if (!x_f16 || !w_gate_up || !y_f16) return fail(WQ_ERR_ARG, "gemv_int4_swiglu: null pointer");
   if (!aligned16(x_f16) || !aligned16(w_gate_up) || !aligned16(y_f16))

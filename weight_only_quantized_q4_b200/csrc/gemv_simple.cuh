@@ -337,7 +337,7 @@ __global__ void repack_int4_v1_meta_kernel(const uint8_t* scales, const uint8_t*
   const int tpb = K / 128;
   const int bpt = int4_v1_bpt(bs);
   const int tb = int4_v1_tile_bytes(bs);
-  const int nb = K / bs, zb = (nb + 1) / 2;
+  const int nb = (K + bs - 1) / bs, zb = (nb + 1) / 2;  // a shorter last block is allowed
   const long long items = n_bands * tpb * bpt * 8;
   for (long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
        it += static_cast<long long>(gridDim.x) * blockDim.x) {

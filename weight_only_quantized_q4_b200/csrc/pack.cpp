@@ -72,7 +72,7 @@ extern "C" size_t wq_int4_codes_bytes(int N, int K, int layout) {
 
 extern "C" size_t wq_int4_packed_bytes(int N, int K, int block_size, int layout) {
   if (N <= 0 || K <= 0 || layout != WQ_LAYOUT_B200_V1) return 0;
-  if (block_size < 32 || block_size > 256 || (block_size & (block_size - 1)) || K % 128 || K % block_size) return 0;
+  if (block_size < 32 || block_size > 256 || (block_size & (block_size - 1)) || K % 128) return 0;
   return static_cast<size_t>((N + 15) / 16) * (K / 128) * WQ_INT4_V1_TILE_BYTES(block_size);
 }
 
@@ -88,10 +88,10 @@ extern "C" size_t wq_q4k_packed_bytes(int N, int K, int layout) {
 
 extern "C" size_t wq_int4_bytes(int N, int K, int block_size, int layout) {
   if (N <= 0 || K <= 0) return 0;
-  if (block_size < 16 || block_size > 256 || (block_size & (block_size - 1)) || K % block_size) return 0;
+  if (block_size < 16 || block_size > 256 || (block_size & (block_size - 1)) || K % 16) return 0;
   if (layout == WQ_LAYOUT_B200_V1) return wq_int4_packed_bytes(N, K, block_size, layout);
   if (layout != WQ_LAYOUT_CANONICAL) return 0;
-  const size_t nb = K / block_size;
+  const size_t nb = (K + block_size - 1) / block_size;  // the last block may be shorter
   return static_cast<size_t>(N) * (K / 2) + static_cast<size_t>(N) * nb * 2 + static_cast<size_t>(N) * ((nb + 1) / 2);
 }
 
