@@ -30,16 +30,20 @@ from .q4 import (  # noqa: F401
     MXFP4_BLOCK,
     dequant_q4k,
     dequant_q4k_from_plane,
+    dequant_q8,
     exact_in_f32,
     f16_bits_to_f64,
     gemv,
     get_scale_min_k4,
     int4_codes,
     int4_zero_points,
+    mmq_q4k,
+    Q8_CHUNK,
     q4k_codes,
     q4k_fields,
     q4k_plane,
     q4k_scales_mins,
+    quantize_q8,
     SILU_MAX_SLOPE,
     silu,
     swiglu_gemv,

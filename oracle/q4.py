@@ -13,6 +13,9 @@ TEST INFRASTRUCTURE ONLY (see the package docstring).  Sources, by page:
   d·sc and -dmin·m), §2.2 (the chunk-major float2 plane and its size), §2.3
   (bit-identity rules), §3.2 (super-block byte offsets and the 6-bit
   scale/min unpacking rule).
+* the same page, §3.2 (the MMQ dispatch arm: an int8 prepass over the
+  activations feeding an integer GEMM rescaled per (chunk, row) pair as in
+  §2.1): ``quantize_q8`` and ``mmq_q4k``; the prepass format is a reading.
 * AstrAI commit log (astrai/extension/backend), the uint4-anchoring bullet:
   the bf16 GEMV is defined for any K >= 1 and any 2-byte storage offset.
 
@@ -309,3 +312,66 @@ def swiglu_tolerance(a, b, Ba, Bb, rel: float = 2e-3, abs_: float = 1e-3) -> np.
     eb = rel * np.asarray(Bb, dtype=np.float64) + abs_
     prop = SILU_MAX_SLOPE * ea * (np.abs(b) + eb) + np.abs(silu(a)) * eb
     return prop + 2.0 ** -10 * (np.abs(silu(a) * b) + prop) + abs_
+
+
+# --------------------------------------------------------------------------
+# int8-activation batched q4_K (minfer doc 62 "r59 — q4_K W_dsc plane": §2.1
+# the rank-1 rescale of each (chunk, row) pair by (d·sc, −dmin·m); §3.2 the
+# MMQ dispatch arm, which quantizes the activations to int8 in a prepass and
+# hands the GEMM the int8 values and their scales)
+# --------------------------------------------------------------------------
+
+Q8_CHUNK = 32  # activations sharing one int8 scale (one q4_K chunk)
+
+
+def quantize_q8(x, M: int, K: int):
+    """The q8 prepass over fp16 activations x [M, K].
+
+    The pages name the prepass but print no format; the reading taken: per
+    row m and 32-element chunk c (the q4_K chunk), in IEEE binary32 with each
+    operation rounded once (numpy float32 arithmetic, no contraction):
+      amax = max |x|            (exact: fp16 values widen exactly),
+      d    = amax / 127,
+      q    = x / d rounded to the nearest integer, ties to even (0 when d = 0),
+      s    = d · Σ q            (Σ q is an exact integer).
+    Returns qa int8 [M, K], d float32 [M, K/32], s float32 [M, K/32].
+    """
+    if K % Q8_CHUNK:
+        raise ValueError("the q8 prepass needs K % 32 == 0")
+    x32 = np.asarray(x, dtype=np.float16).reshape(M, K // Q8_CHUNK, Q8_CHUNK).astype(np.float32)
+    amax = np.max(np.abs(x32), axis=2)
+    d = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(d > 0, d, np.float32(1.0)).astype(np.float32)
+    q = np.rint((x32 / safe[..., None]).astype(np.float32))
+    q = np.where(d[..., None] > 0, q, 0.0).astype(np.int64)
+    s = (d * q.sum(axis=2).astype(np.float32)).astype(np.float32)
+    return q.reshape(M, K).astype(np.int8), d, s
+
+
+def dequant_q8(qa, d, M: int, K: int) -> np.ndarray:
+    """The activations the int8 path multiplies by: d[m, c]·q[m, k] in float64 (exact)."""
+    q = np.asarray(qa, dtype=np.int8).astype(np.float64).reshape(M, K // Q8_CHUNK, Q8_CHUNK)
+    return (q * np.asarray(d, dtype=np.float32).astype(np.float64)[..., None]).reshape(M, K)
+
+
+def mmq_q4k(raw, qa, d, s, M: int, N: int, K: int) -> np.ndarray:
+    """y[m, n] = Σ_c (d·sc)[n,c]·d[m,c]·I[m,n,c] + (−dmin·m)[n,c]·s[m,c] in float64.
+
+    I[m, n, c] = Σ_{k in chunk c} q[n, k]·qa[m, k] is the exact integer dot
+    product of the chunk's 4-bit weight codes and int8 activations; the two
+    coefficients of each (chunk, row) pair are the W_dsc plane entries (§2.2:
+    one fp32 multiply each), and (d, s) are the prepass's per-chunk activation
+    scale and scaled code sum.  Since w = (d·sc)·q − dmin·m on every element
+    of a chunk, this is Σ_k w[n,k]·d[m,c]·qa[m,k] up to the rounding of s.
+    """
+    C = K // Q8_CHUNK
+    P = q4k_plane(raw, N, K).astype(np.float64)                # [C, N, 2]
+    _, _, _, qs = q4k_fields(raw, N, K)
+    q = q4k_codes(qs).reshape(N, C, Q8_CHUNK)                   # int64 codes 0..15
+    a = np.asarray(qa, dtype=np.int8).astype(np.int64).reshape(M, C, Q8_CHUNK)
+    isum = np.einsum("ncj,mcj->mnc", q, a)                      # exact int64
+    dd = np.asarray(d, dtype=np.float32).astype(np.float64).reshape(M, C)
+    ss = np.asarray(s, dtype=np.float32).astype(np.float64).reshape(M, C)
+    scale_term = np.einsum("cn,mc,mnc->mn", P[:, :, 0], dd, isum.astype(np.float64))
+    min_term = np.einsum("cn,mc->mn", P[:, :, 1], ss)
+    return scale_term + min_term

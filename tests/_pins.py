@@ -471,6 +471,111 @@ def pin_swiglu_tolerance_covers_worst_case(o):
                 assert np.all(np.abs(yp * r - y) <= tol)
 
 
+# ---------------------------------------------------------------- q8 prepass and int8-activation q4_K
+
+def _golden_q8():
+    g = _golden("q8_prepass_hand.json")
+    x = np.zeros((1, 32 * len(g["x_chunks"])), dtype=np.float16)
+    q = np.zeros(x.shape, dtype=np.int64)
+    for c, (xs, qs) in enumerate(zip(g["x_chunks"], g["q_chunks"])):
+        x[0, 32 * c:32 * c + len(xs)] = xs
+        q[0, 32 * c:32 * c + len(qs)] = qs
+    bits = lambda v: np.array([int(b, 16) for b in v], dtype=np.uint32).view(np.float32)  # noqa: E731
+    return x, q, bits(g["d_bits"]), bits(g["s_bits"])
+
+
+def pin_q8_golden(o):
+    """Hand-worked chunks: exact scales, ties to even, zero chunk, a scale that rounds."""
+    x, q, d, s = _golden_q8()
+    qa, dd, ss = o.quantize_q8(x, 1, x.shape[1])
+    assert qa.dtype == np.int8 and np.array_equal(qa.astype(np.int64), q)
+    assert np.array_equal(dd.reshape(-1).view(np.uint32), d.view(np.uint32))
+    assert np.array_equal(ss.reshape(-1).view(np.uint32), s.view(np.uint32))
+
+
+def pin_q8_properties(o):
+    """On random fp16 rows (plus a tiny-valued and a large-valued row): |q| <= 127,
+    the largest |q| of every non-zero chunk is 127, |x - d·q| <= d·(1/2 + 2^-16)
+    (one rounding of the quotient), and s is d·Σq rounded once."""
+    M, K = 5, 1024
+    x = synth.activations_f16(M, K, workload=910)
+    x[3] = (x[3].astype(np.float64) * 1e-6).astype(np.float16)    # fp16 subnormal range
+    x[4] = (x[4].astype(np.float64) * 1.5e4).astype(np.float16)
+    x[2, 64:96] = 0
+    qa, d, s = o.quantize_q8(x, M, K)
+    q = qa.astype(np.int64).reshape(M, K // 32, 32)
+    xc = x.astype(np.float64).reshape(M, K // 32, 32)
+    dd = d.astype(np.float64)[..., None]
+    assert np.all(np.abs(q) <= 127)
+    nz = np.max(np.abs(xc), axis=2) > 0
+    assert np.all(np.max(np.abs(q), axis=2)[nz] == 127) and np.all(q[~nz] == 0) and np.all(d[~nz] == 0)
+    assert np.all(np.abs(xc - dd * q) <= dd * (0.5 + 2.0 ** -16))
+    exact = d.astype(np.float64) * q.sum(axis=2)
+    assert np.all(np.abs(s.astype(np.float64) - exact) <= 2.0 ** -24 * np.abs(exact))
+
+
+def _brute_mmq(raw, qa, d, s, M, N, K):
+    """y by the definition, in pure Python: per chunk, the exact integer dot
+    product of the nibble codes and the int8 values, times d·sc and the
+    activation scale, plus −dmin·m times s (d·sc and dmin·m are exact: an fp16
+    times a 6-bit integer)."""
+    raw = np.asarray(raw, dtype=np.uint8).reshape(N, K // 256, 144)
+    y = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            terms = []
+            for sb in range(K // 256):
+                blk = [int(v) for v in raw[n, sb]]
+                dw = float(np.array([blk[0] | (blk[1] << 8)], dtype=np.uint16).view(np.float16)[0])
+                dmin = float(np.array([blk[2] | (blk[3] << 8)], dtype=np.uint16).view(np.float16)[0])
+                sc = blk[4:16]
+                for c in range(8):
+                    if c < 4:
+                        sv, mv = sc[c] & 63, sc[c + 4] & 63
+                    else:
+                        sv = (sc[c + 4] & 15) | ((sc[c - 4] >> 6) << 4)
+                        mv = (sc[c + 4] >> 4) | ((sc[c] >> 6) << 4)
+                    isum = 0
+                    for i in range(32):
+                        byte = blk[16 + 32 * (c // 2) + i]
+                        code = (byte & 15) if c % 2 == 0 else (byte >> 4)
+                        isum += code * int(qa[m, 256 * sb + 32 * c + i])
+                    gc = 8 * sb + c
+                    terms.append(dw * sv * float(d[m, gc]) * isum)
+                    terms.append(-(dmin * mv) * float(s[m, gc]))
+            y[m, n] = math.fsum(terms)
+    return y
+
+
+def pin_mmq_brute(o):
+    """The int8-activation q4_K product equals the definition evaluated term by term."""
+    M, N, K = 2, 3, 512
+    raw = synth.q4k_weights(N, K, workload=911)
+    qa, d, s = o.quantize_q8(synth.activations_f16(M, K, workload=911), M, K)
+    y = o.mmq_q4k(raw, qa, d, s, M, N, K)
+    yb = _brute_mmq(raw, qa, d, s, M, N, K)
+    assert np.all(np.abs(y - yb) <= 1e-12 * (1 + np.abs(yb))), np.abs(y - yb).max()
+
+
+def pin_mmq_is_the_gemv_of_the_quantized_activations(o):
+    """Since w = d·sc·q − dmin·m on every element of a chunk, the factored
+    product equals W·(d·qa) except for the one rounding of s: the difference
+    is at most Σ_c |dmin·m|·|s − d·Σqa| (plus fp64 noise)."""
+    M, N, K = 3, 40, 1024
+    raw = synth.q4k_weights(N, K, workload=912)
+    x = synth.activations_f16(M, K, workload=912)
+    qa, d, s = o.quantize_q8(x, M, K)
+    y = o.mmq_q4k(raw, qa, d, s, M, N, K)
+    W = _brute_q4k(raw, N, K)
+    xd = qa.astype(np.float64) * np.repeat(d.astype(np.float64), 32, axis=1)
+    y2 = xd @ W.T
+    P = o.q4k_plane(raw, N, K).astype(np.float64)                       # [C, N, 2]
+    ds = np.abs(s.astype(np.float64) - d.astype(np.float64) * qa.astype(np.int64).reshape(M, -1, 32).sum(axis=2))
+    slack = ds @ np.abs(P[:, :, 1]) + 1e-12 * (np.abs(xd) @ np.abs(W).T)
+    assert np.all(np.abs(y - y2) <= slack)
+    assert np.array_equal(o.dequant_q8(qa, d, M, K), xd)
+
+
 ALL_PINS = [
     pin_scale_min_golden,
     pin_scale_min_bijection,
@@ -498,4 +603,8 @@ ALL_PINS = [
     pin_silu_reflection_and_slope,
     pin_swiglu_hand,
     pin_swiglu_tolerance_covers_worst_case,
+    pin_q8_golden,
+    pin_q8_properties,
+    pin_mmq_brute,
+    pin_mmq_is_the_gemv_of_the_quantized_activations,
 ]

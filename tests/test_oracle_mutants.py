@@ -156,6 +156,32 @@ def _mxfp4_block_16(w_packed, scales, N, K):
     return oq.e8m0_value(E)[:, blk] * oq.e2m1_value(q)
 
 
+def _q8_variant(x, M, K, *, half_away=False, div=127.0, s_without_d=False):
+    x32 = np.asarray(x, dtype=np.float16).reshape(M, K // 32, 32).astype(np.float32)
+    amax = np.max(np.abs(x32), axis=2)
+    d = (amax / np.float32(div)).astype(np.float32)
+    safe = np.where(d > 0, d, np.float32(1.0)).astype(np.float32)
+    v = (x32 / safe[..., None]).astype(np.float32)
+    q = np.sign(v) * np.floor(np.abs(v) + 0.5) if half_away else np.rint(v)
+    q = np.clip(np.where(d[..., None] > 0, q, 0.0), -127, 127).astype(np.int64)
+    qs = q.sum(axis=2).astype(np.float32)
+    s = qs if s_without_d else (d * qs).astype(np.float32)
+    return q.reshape(M, K).astype(np.int8), d, s
+
+
+def _mmq_variant(raw, qa, d, s, M, N, K, *, min_sign=-1.0, shift_qa=0, shift_d=0):
+    C = K // 32
+    P = oq.q4k_plane(raw, N, K).astype(np.float64)
+    _, _, _, qs = oq.q4k_fields(raw, N, K)
+    q = oq.q4k_codes(qs).reshape(N, C, 32)
+    a = np.roll(np.asarray(qa, dtype=np.int8).astype(np.int64), shift_qa, axis=1).reshape(M, C, 32)
+    isum = np.einsum("ncj,mcj->mnc", q, a)
+    dd = np.roll(np.asarray(d, dtype=np.float32).astype(np.float64).reshape(M, C), shift_d, axis=1)
+    ss = np.asarray(s, dtype=np.float32).astype(np.float64).reshape(M, C)
+    return (np.einsum("cn,mc,mnc->mn", P[:, :, 0], dd, isum.astype(np.float64))
+            - min_sign * np.einsum("cn,mc->mn", P[:, :, 1], ss))
+
+
 MUTANTS = {
     "int4 nibbles high-first": ("int4_codes", _int4_codes_high_first),
     "int4 default zero-point 0": ("int4_zero_points", _zero_points_default_zero),
@@ -180,6 +206,12 @@ MUTANTS = {
     "silu reflected": ("silu", _silu_reflected),
     "swiglu gate and up swapped": ("swiglu_gemv", _swiglu_gate_up_swapped),
     "swiglu tolerance without the up error": ("swiglu_tolerance", _swiglu_tolerance_no_up_term),
+    "q8 ties away from zero": ("quantize_q8", lambda x, M, K: _q8_variant(x, M, K, half_away=True)),
+    "q8 scale amax/128": ("quantize_q8", lambda x, M, K: _q8_variant(x, M, K, div=128.0)),
+    "q8 code sum without the scale": ("quantize_q8", lambda x, M, K: _q8_variant(x, M, K, s_without_d=True)),
+    "mmq min term sign": ("mmq_q4k", lambda *a: _mmq_variant(*a, min_sign=1.0)),
+    "mmq activations one k late": ("mmq_q4k", lambda *a: _mmq_variant(*a, shift_qa=1)),
+    "mmq activation scale of the next chunk": ("mmq_q4k", lambda *a: _mmq_variant(*a, shift_d=-1)),
 }
 
 
