@@ -41,7 +41,7 @@
  *  - The first call on a device configures kernel attributes and looks up the
  *    driver's tensor-map encoder; make it before capturing a CUDA graph.
  *  - Environment variables read at each call, for tests and tuning only:
- *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc | mx) pins a kernel
+ *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc | mx | mmq) pins a kernel
  *    family (a call that family cannot run returns WQ_ERR_UNSUPPORTED; there
  *    is no silent substitute), WQ_PDL=0 disables programmatic dependent
  *    launch, and WQ_V1_*, WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch
@@ -233,6 +233,38 @@ int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K
  * fp32 range is ±inf; E = 255 gives NaN).  K % 32 == 0; w_packed and w_out
  * 16-byte aligned. */
 int dequant_mxfp4(const void* w_packed, const void* scales_e8m0, float* w_out, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * int8-activation batched q4_K (minfer doc 62 "r59 — q4_K W_dsc plane", §3.2:
+ * the MMQ dispatch arm quantizes the activations to int8 in a prepass and
+ * runs an integer GEMM whose (chunk, row) pairs are rescaled by the §2.1
+ * coefficients).  Numerically this is a different product from gemv_q4k: x is
+ * replaced by its int8 quantization.
+ * ------------------------------------------------------------------------- */
+
+/* The q8 prepass.  For every token m and 32-element chunk c of x [M][K] fp16
+ * (binary32, one rounding per operation): amax = max|x|, d = amax / 127,
+ * q = x / d rounded to nearest, ties to even (0 when d = 0; |q| <= 127),
+ * s = d·Σq.  Writes qa8 int8 [M][K] (token-major, wq_q8_bytes) and sda
+ * float2 [K/32][Mp] = (d, s), Mp = M rounded up to 16, entries of tokens
+ * M..Mp-1 zero (chunk-major, wq_q8_scale_bytes).  K % 32 == 0; every pointer
+ * 16-byte aligned; x finite (the result for inf / NaN inputs is unspecified).
+ * Errors: WQ_ERR_ARG, WQ_ERR_ALIGN, WQ_ERR_DEVICE, WQ_ERR_CUDA. */
+int quantize_q8(const void* x_f16, void* qa8, void* sda, int M, int K, void* stream);
+size_t wq_q8_bytes(int M, int K);       /* M·K, 0 if invalid */
+size_t wq_q8_scale_bytes(int M, int K); /* 8·(K/32)·Mp, 0 if invalid */
+
+/* y[M,N] fp16 = Σ_c (d·sc)[n,c]·d[m,c]·I[m,n,c] + (−dmin·m)[n,c]·s[m,c],
+ * I[m,n,c] = Σ_{k in chunk c} q4[n,k]·qa8[m,k] (exact), fp32 accumulation,
+ * for canonical q4_K weights (w_q4k [N][K/256][144]) and the prepass output
+ * (qa8, sda).  w_dsc (nullable): the W_dsc plane of the same weights, read
+ * for the coefficients instead of decoding them (the results are bit-
+ * identical).  tcgen05 kind::i8 GEMM.  K % 256 == 0; qa8, sda, w_q4k and
+ * w_dsc 16-byte aligned, y 2-byte aligned.  WQ_FORCE_KERNEL other than "mmq"
+ * returns WQ_ERR_UNSUPPORTED.  Errors: WQ_ERR_ARG, WQ_ERR_ALIGN,
+ * WQ_ERR_UNSUPPORTED, WQ_ERR_DEVICE, WQ_ERR_CUDA. */
+int gemm_q4k_q8(const void* qa8, const void* sda, const void* w_q4k, const void* w_dsc, void* y_f16, int M, int N,
+                int K, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Weight packing (load time).

@@ -41,6 +41,10 @@ SIGNATURES = {
     "dequant_int4_blockwise": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "dequant_q4k": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "dequant_mxfp4": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
+    "quantize_q8": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
+    "gemm_q4k_q8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "wq_q8_bytes": (_sz, [_i, _i]),
+    "wq_q8_scale_bytes": (_sz, [_i, _i]),
     "wq_int4_bytes": (_sz, [_i, _i, _i, _i]),
     "wq_int4_codes_bytes": (_sz, [_i, _i, _i]),
     "wq_repack_int4": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),

@@ -94,6 +94,23 @@ def dequant_mxfp4(w_packed, scales, w_out, N, K, stream=None):
     _check(lib().dequant_mxfp4(_ptr(w_packed), _ptr(scales), _ptr(w_out), N, K, _stream(stream)), "dequant_mxfp4")
 
 
+def quantize_q8(x, qa8, sda, M, K, stream=None):
+    _check(lib().quantize_q8(_ptr(x), _ptr(qa8), _ptr(sda), M, K, _stream(stream)), "quantize_q8")
+
+
+def gemm_q4k_q8(qa8, sda, w_q4k, w_dsc, y, M, N, K, stream=None):
+    _check(lib().gemm_q4k_q8(_ptr(qa8), _ptr(sda), _ptr(w_q4k), _ptr(w_dsc), _ptr(y), M, N, K, _stream(stream)),
+           "gemm_q4k_q8")
+
+
+def wq_q8_bytes(M, K) -> int:
+    return int(lib().wq_q8_bytes(M, K))
+
+
+def wq_q8_scale_bytes(M, K) -> int:
+    return int(lib().wq_q8_scale_bytes(M, K))
+
+
 def dequant_q4k(w_q4k, w_dsc, w_out, N, K, layout=WQ_LAYOUT_CANONICAL, stream=None):
     _check(lib().dequant_q4k(_ptr(w_q4k), _ptr(w_dsc), _ptr(w_out), N, K, layout, _stream(stream)), "dequant_q4k")
 

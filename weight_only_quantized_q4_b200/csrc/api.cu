@@ -27,6 +27,7 @@
 #include "gemm_tc5.cuh"
 #include "gemm_v1tc.cuh"
 #include "gemv_mxfp4.cuh"
+#include "gemm_mmq.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -1267,6 +1268,88 @@ int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, i
   return WQ_OK;
 }
 
+// int8-activation q4_K GEMM: BN = M rounded up to 16 (at most 128), clusters
+// of S CTAs splitting the super-blocks while the CTAs fit one wave.
+template <int BN>
+int launch_mmq_bn(const void* qa8, const void* sda, const void* w, const void* plane, void* y, int M, int N, int K,
+                  int sms, cudaStream_t st, std::string* label) {
+  using SH = MMQShape<BN>;
+  MMQParams p{};
+  p.plane = static_cast<const float*>(plane);
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  const int Mp = (M + 15) / 16 * 16;
+  const int nsb_total = K / 256;
+  const int n_tiles = (N + 127) / 128, m_tiles = (M + BN - 1) / BN;
+  int S = 1;
+  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nsb_total % (2 * S) == 0) S *= 2;
+  if (const char* s_env = std::getenv("WQ_MMQ_S")) {  // tests and tuning
+    const int sf = std::atoi(s_env);
+    if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
+      if (nsb_total % sf) return fail(WQ_ERR_ARG, "WQ_MMQ_S does not divide the super-blocks of K");
+      S = sf;
+    }
+  }
+  p.S = S;
+  p.nsb = nsb_total / S;
+  p.stage_bytes = (SH::STAGE + 1023) / 1024 * 1024;
+  p.a_bytes = (SH::A_SLOT + 1023) / 1024 * 1024;
+  p.NA = 2;
+  const int bars = 8 * (2 * 8 + 2 * p.NA + 5) + 16;
+  const int budget = kSmemPerSm + 4096 - 1024 - bars;
+  p.NS = std::min(4, (budget - p.NA * p.a_bytes) / p.stage_bytes);
+  if (const char* ns_env = std::getenv("WQ_MMQ_NS")) p.NS = std::max(2, std::min(p.NS, std::atoi(ns_env)));
+  if (p.NS < 2) return fail(WQ_ERR_UNSUPPORTED, "gemm_q4k_q8: shared memory plan too large");
+  p.off_a = p.NS * p.stage_bytes;
+  p.off_bar = p.off_a + p.NA * p.a_bytes;
+  const int smem = 1024 + p.off_bar + 8 * (2 * p.NS + 2 * p.NA + 5) + 16;
+  if (smem > kSmemPerSm + 4096) return fail(WQ_ERR_UNSUPPORTED, "gemm_q4k_q8: shared memory plan too large");
+  if (S > 1 && 512 * BN > p.off_a) return fail(WQ_ERR_UNSUPPORTED, "gemm_q4k_q8: cluster partials do not fit");
+  const unsigned long long row_bytes = 144ull * nsb_total;
+  int rc = encode_2d(&p.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, row_bytes, N, row_bytes, 144, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  if ((rc = encode_2d(&p.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa8, K, M, K, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  if ((rc = encode_2d(&p.tmap_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sda, 2ull * Mp, K / 32, 8ull * Mp, 2 * BN, 8,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)))
+    return rc;
+  {
+    static std::mutex mu;
+    static bool configured[64] = {};
+    std::lock_guard<std::mutex> lk(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemm_mmq_kernel<BN>),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles * S, m_tiles, 1);
+  cfg.blockDim = dim3(kMMQWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemm_mmq_kernel<BN>, p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_q4k_q8 launch: ") + cudaGetErrorString(e));
+  if ((rc = launch_check("gemm_q4k_q8 launch"))) return rc;
+  char buf[64];
+  std::snprintf(buf, sizeof(buf), "q4k.mmq.bn%d.ns%d.s%d%s", BN, p.NS, S, plane ? ".dsc" : "");
+  *label = buf;
+  return WQ_OK;
+}
+
 // Run one format over all M in chunks of at most 8 rows of x.
 template <Fmt F>
 int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros,
@@ -1605,6 +1688,64 @@ int gemv_mxfp4(const void* x_f16, const void* w_packed, const void* scales_e8m0,
   char buf[64];
   std::snprintf(buf, sizeof(buf), "mxfp4.gemv.mx.m%d%s", std::min(8, M), M > 8 ? ".chunked" : "");
   set_last_kernel(buf);
+  return WQ_OK;
+}
+
+size_t wq_q8_bytes(int M, int K) {
+  if (M <= 0 || K <= 0 || K % 32) return 0;
+  return static_cast<size_t>(M) * K;
+}
+
+size_t wq_q8_scale_bytes(int M, int K) {
+  if (M <= 0 || K <= 0 || K % 32) return 0;
+  return static_cast<size_t>(K / 32) * ((M + 15) / 16 * 16) * 8;
+}
+
+int quantize_q8(const void* x_f16, void* qa8, void* sda, int M, int K, void* stream) {
+  int rc = check_dims(M, 1, K);
+  if (rc) return rc;
+  if (K % 32) return fail(WQ_ERR_ARG, "quantize_q8: K must be a multiple of 32");
+  if (!x_f16 || !qa8 || !sda) return fail(WQ_ERR_ARG, "quantize_q8: null pointer");
+  if (!aligned16(x_f16) || !aligned16(qa8) || !aligned16(sda))
+    return fail(WQ_ERR_ALIGN, "quantize_q8: device pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  const int Mp = (M + 15) / 16 * 16;
+  const long long items = static_cast<long long>(K / 32) * Mp;
+  const int grid = static_cast<int>(std::min<long long>((items + 255) / 256, di.sms * 16ll));
+  quantize_q8_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half*>(x_f16), static_cast<int8_t*>(qa8), static_cast<float2*>(sda), M, Mp, K);
+  if ((rc = launch_check("quantize_q8 launch"))) return rc;
+  set_last_kernel("q8.quantize");
+  return WQ_OK;
+}
+
+int gemm_q4k_q8(const void* qa8, const void* sda, const void* w_q4k, const void* w_dsc, void* y_f16, int M, int N,
+                int K, void* stream) {
+  int rc = check_dims(M, N, K);
+  if (rc) return rc;
+  if (K % 256) return fail(WQ_ERR_ARG, "gemm_q4k_q8: q4_K needs K % 256 == 0");
+  if (!qa8 || !sda || !w_q4k || !y_f16) return fail(WQ_ERR_ARG, "gemm_q4k_q8: null pointer");
+  if (!aligned16(qa8) || !aligned16(sda) || !aligned16(w_q4k) || (w_dsc && !aligned16(w_dsc)) || !aligned2(y_f16))
+    return fail(WQ_ERR_ALIGN, "gemm_q4k_q8: qa8, sda, w_q4k and w_dsc must be 16-byte aligned, y 2-byte aligned");
+  if (const char* force = forced_variant())
+    if (std::strcmp(force, "mmq") != 0)
+      return fail(WQ_ERR_UNSUPPORTED, std::string("WQ_FORCE_KERNEL=") + force + ": the int8-activation GEMM has one kernel family (mmq)");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::string label;
+  const int bn = std::min(128, (M + 15) / 16 * 16);
+  if (bn == 16)
+    rc = launch_mmq_bn<16>(qa8, sda, w_q4k, w_dsc, y_f16, M, N, K, di.sms, st, &label);
+  else if (bn == 32)
+    rc = launch_mmq_bn<32>(qa8, sda, w_q4k, w_dsc, y_f16, M, N, K, di.sms, st, &label);
+  else if (bn <= 64)
+    rc = launch_mmq_bn<64>(qa8, sda, w_q4k, w_dsc, y_f16, M, N, K, di.sms, st, &label);
+  else
+    rc = launch_mmq_bn<128>(qa8, sda, w_q4k, w_dsc, y_f16, M, N, K, di.sms, st, &label);
+  if (rc) return rc;
+  set_last_kernel(label);
   return WQ_OK;
 }
 
