@@ -79,10 +79,17 @@ for _M in (16, 32, 64, 128):
                                                                        layout=1)
         WORKLOADS[f"batched_q4k_m{_M}_{_N}x{_K}"] = dict(fmt="q4k", M=_M, N=_N, K=_K, dsc=False, workload=5)
 
+# int8-activation q4_K (one step = the q8 prepass + the kind::i8 GEMM)
+for _M in (16, 32, 64, 128, 512):
+    for _N, _K in ((4096, 4096), (11008, 4096), (4096, 11008), (14336, 4096), (32000, 4096)):
+        WORKLOADS[f"mmq_q4k_m{_M}_{_N}x{_K}"] = dict(fmt="mmq", M=_M, N=_N, K=_K, workload=5)
+
 DEFAULT_WORKLOAD = "int4_b128_zp_v1_m1_4096x14336"
 METRIC = "achieved HBM GB/s and \u00b5s/call per quantized GEMV at M=1..8 vs ~8 TB/s peak"
 SWEEP_BATCHED = [f"batched_{f}_m{m}_{n}x{k}" for f in ("int4_b128_zp_v1", "int4_b128_zp", "q4k")
                  for m in (16, 32, 64, 128) for n, k in ((4096, 4096), (14336, 4096), (4096, 14336), (32000, 4096))]
+SWEEP_BATCHED += [f"mmq_q4k_m{m}_{n}x{k}" for m in (16, 32, 64, 128, 512)
+                  for n, k in ((4096, 4096), (11008, 4096), (4096, 11008), (32000, 4096))]
 SWEEP = ["q4k_v1_m1_4096x11008", "q4k_v1_m4_4096x11008", "q4k_v1_m1_11008x4096", "int4_b128_zp_v1_m1_4096x14336", "int4_b128_zp_v1_m2_4096x14336", "int4_b128_zp_v1_m4_4096x14336", "int4_b128_zp_v1_m8_4096x14336",
          "int4_b128_zp_v1_m1_14336x4096", "int4_b128_zp_v1_m1_4096x4096",
          "int4_b128_zp_m1_4096x14336", "int4_b128_zp_m4_4096x14336", "int4_b128_zp_m1_14336x4096",
@@ -98,6 +105,8 @@ def weight_bytes(w) -> int:
         return N * K // 2 + 2 * N * nb + (N * ((nb + 1) // 2) if w["zeros"] else 0)
     if w["fmt"] == "q4k":
         return N * K // 2 + N * K // 4 if w["dsc"] else N * (K // 256) * 144
+    if w["fmt"] == "mmq":
+        return N * (K // 256) * 144
     if w["fmt"] == "mxfp4":
         return N * K // 2 + N * K // 32
     if w["fmt"] == "swiglu":  # gate and up: two int4 tensors of N x K
@@ -108,7 +117,7 @@ def weight_bytes(w) -> int:
 
 def dtype_of(w) -> str:
     return {"int4": "int4xf16->f32", "q4k": "q4kxf16->f32", "bf16": "bf16xbf16->f32",
-            "mxfp4": "mxfp4xf16->f32", "swiglu": "int4xf16->f32"}[w["fmt"]]
+            "mxfp4": "mxfp4xf16->f32", "swiglu": "int4xf16->f32", "mmq": "q4kxs8->s32->f32"}[w["fmt"]]
 
 
 def host_inputs(w):
@@ -123,6 +132,8 @@ def host_inputs(w):
                     raw=synth.q4k_weights(N, K, workload=w["workload"]))
     if w["fmt"] == "mxfp4":
         return dict(x=synth.activations_f16(M, K, workload=w["workload"]), **synth.mxfp4_weights(N, K, workload=w["workload"]))
+    if w["fmt"] == "mmq":
+        return dict(x=synth.activations_f16(M, K, workload=w["workload"]), raw=synth.q4k_weights(N, K, workload=w["workload"]))
     if w["fmt"] == "swiglu":
         g = synth.int4_weights(N, K, w["bs"], scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=w["workload"])
         u = synth.int4_weights(N, K, w["bs"], scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=w["workload"] + 50)
@@ -204,6 +215,7 @@ class DeviceWorkload:
         if copies > 0:
             self.R = copies
         self.copies = []
+        self.launches_per_call = 1
         if w["fmt"] == "int4":
             base = [torch.from_numpy(host["w_packed"]).to(dev), torch.from_numpy(host["scales"]).to(dev),
                     torch.from_numpy(host["zeros"]).to(dev) if host["zeros"] is not None else None]
@@ -230,6 +242,15 @@ class DeviceWorkload:
                 self.copies.append(c)
             self.x = torch.from_numpy(host["x"]).to(dev)
             self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        elif w["fmt"] == "mmq":
+            raw = torch.from_numpy(host["raw"]).to(dev)
+            for _ in range(self.R):
+                self.copies.append([raw.clone()])
+            self.x = torch.from_numpy(host["x"]).to(dev)
+            self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            self.qa = torch.empty((M, K), dtype=torch.int8, device=dev)
+            self.sd = torch.empty(wq.wq_q8_scale_bytes(M, K) // 4, dtype=torch.float32, device=dev)
+            self.launches_per_call = 2
         elif w["fmt"] == "swiglu":
             d = {h: [torch.from_numpy(host[h][k]).to(dev) for k in ("w_packed", "scales", "zeros")] for h in ("gate", "up")}
             packed = torch.empty(wq.wq_int4_gate_up_packed_bytes(N, K, w["bs"]), dtype=torch.uint8, device=dev)
@@ -280,6 +301,9 @@ class DeviceWorkload:
             wq.gemv_mxfp4(x, c[0], c[1], y, M, self.N, self.K, stream=stream)
         elif w["fmt"] == "swiglu":
             wq.gemv_int4_swiglu(x, c[0], y, M, self.N, self.K, w["bs"], stream=stream)
+        elif w["fmt"] == "mmq":
+            wq.quantize_q8(x, self.qa, self.sd, M, self.K, stream=stream)
+            wq.gemm_q4k_q8(self.qa, self.sd, c[0], None, y, M, self.N, self.K, stream=stream)
         else:
             wq.gemv_bf16(x, c[0], y, M, self.N, self.K, stream=stream)
 
@@ -544,7 +568,7 @@ def run_ours(args, w, wname, rank, world, dist):
                 "how": "per step: pinned x -> device, GEMV through the C ABI, y -> pinned host; steps pipelined over "
                        "two copy streams with 3 device buffers per tensor (copies of neighbouring steps overlap the "
                        "GEMV); graph-captured; median of the repetitions"},
-        "gpu_launches": steps,
+        "gpu_launches": steps * d.launches_per_call,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": _traffic(wname),
                      "peak_kind": f"{peak_kind} copy bandwidth", "avg_launch_us": rs["us_per_call_median"],
@@ -591,6 +615,11 @@ def cpu_baseline(w, host, budget_s=15.0):
         elif w["fmt"] == "mxfp4":
             W = oracle.dequant_mxfp4(host["w_packed"][r], host["scales"][r], len(r), K)
             xv = x.astype(np.float64)
+        elif w["fmt"] == "mmq":
+            qa, dq, sq = oracle.quantize_q8(x, M, K)
+            oracle.mmq_q4k(host["raw"][r], qa, dq, sq, M, len(r), K)
+            W = oracle.dequant_q4k(host["raw"][r], len(r), K)
+            xv = oracle.dequant_q8(qa, dq, M, K)
         elif w["fmt"] == "swiglu":
             Wg = oracle.dequant_int4(host["gate"]["w_packed"][r], host["gate"]["scales"][r], host["gate"]["zeros"][r],
                                      len(r), K, w["bs"])

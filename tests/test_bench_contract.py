@@ -39,6 +39,8 @@ def test_weight_bytes_match_library_size_queries(name):
     elif w["fmt"] == "swiglu":
         assert got == 2 * wq.wq_int4_bytes(N, K, w["bs"], wq.WQ_LAYOUT_CANONICAL)
         assert got <= wq.wq_int4_gate_up_packed_bytes(N, K, w["bs"]) <= got * 1.01
+    elif w["fmt"] == "mmq":  # the q4_K weights (the int8 activations are like x, excluded)
+        assert got == wq.wq_q4k_bytes(N, K)
     elif w["fmt"] == "mxfp4":
         # codes (two per byte) plus one E8M0 byte per 32-element block
         assert got == wq.wq_int4_codes_bytes(N, K, wq.WQ_LAYOUT_CANONICAL) + N * (K // 32)

@@ -130,10 +130,12 @@ def test_gemm_q4k_q8_plane_is_bit_identical(M, N, K):
 @gpu
 @pytest.mark.parametrize("S", [1, 2, 4, 8])
 @pytest.mark.parametrize("M", [16, 40, 128])
-def test_gemm_q4k_q8_cluster_split(S, M, monkeypatch):
-    """K split over clusters of S CTAs, partials added over distributed shared memory in rank order."""
+@pytest.mark.parametrize("K", [2048, 2816])
+def test_gemm_q4k_q8_cluster_split(S, M, K, monkeypatch):
+    """K split over clusters of S CTAs (K = 2816: eleven super-blocks, uneven
+    runs per rank), partials added over distributed shared memory in rank order."""
     monkeypatch.setenv("WQ_MMQ_S", str(S))
-    c = MMQCase(M, 300, 2048, workload=123)
+    c = MMQCase(M, 300, K, workload=123)
     y = c.run()
     assert wq.last_kernel().endswith(f".s{S}"), wq.last_kernel()
     c.check(y)
@@ -142,12 +144,18 @@ def test_gemm_q4k_q8_cluster_split(S, M, monkeypatch):
 
 @gpu
 @pytest.mark.parametrize("NS", [2, 3])
-def test_gemm_q4k_q8_shallow_ring(NS, monkeypatch):
+@pytest.mark.parametrize("NA", [2, 3])
+@pytest.mark.parametrize("M", [33, 128])
+def test_gemm_q4k_q8_ring_depths(NS, NA, M, monkeypatch):
+    """Shallower stage rings and A-slot rings than the planner picks (the
+    planner's choice is capped by shared memory, so a forced depth may come
+    out smaller: the label tells)."""
     monkeypatch.setenv("WQ_MMQ_NS", str(NS))
+    monkeypatch.setenv("WQ_MMQ_NA", str(NA))
     monkeypatch.setenv("WQ_MMQ_S", "1")
-    c = MMQCase(33, 256, 4096, workload=124)
+    c = MMQCase(M, 256, 4096, workload=124)
     y = c.run()
-    assert f".ns{NS}." in wq.last_kernel(), wq.last_kernel()
+    assert ".ns" in wq.last_kernel() and ".na" in wq.last_kernel(), wq.last_kernel()
     c.check(y)
 
 
@@ -194,7 +202,7 @@ def test_gemm_q4k_q8_argument_errors(monkeypatch):
     torch.cuda.synchronize()
     monkeypatch.delenv("WQ_FORCE_KERNEL")
     monkeypatch.setenv("WQ_MMQ_S", "8")
-    with pytest.raises(wq.WQError) as e:  # one super-block cannot split eight ways
+    with pytest.raises(wq.WQError) as e:  # one super-block cannot be split eight ways
         wq.gemm_q4k_q8(c.gq.t, c.gs.t, c.draw, None, y, 16, 32, 256)
     assert e.value.code == wq.WQ_ERR_ARG
 

@@ -1283,22 +1283,26 @@ int launch_mmq_bn(const void* qa8, const void* sda, const void* w, const void* p
   const int Mp = (M + 15) / 16 * 16;
   const int nsb_total = K / 256;
   const int n_tiles = (N + 127) / 128, m_tiles = (M + BN - 1) / BN;
+  // the ranks of a cluster take consecutive, nearly equal runs of super-blocks
   int S = 1;
-  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nsb_total % (2 * S) == 0) S *= 2;
+  while (S < 8 && n_tiles * m_tiles * S * 2 <= sms && nsb_total >= 2 * S) S *= 2;
   if (const char* s_env = std::getenv("WQ_MMQ_S")) {  // tests and tuning
     const int sf = std::atoi(s_env);
     if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
-      if (nsb_total % sf) return fail(WQ_ERR_ARG, "WQ_MMQ_S does not divide the super-blocks of K");
+      if (nsb_total < sf) return fail(WQ_ERR_ARG, "WQ_MMQ_S exceeds the super-blocks of K");
       S = sf;
     }
   }
   p.S = S;
-  p.nsb = nsb_total / S;
+  p.nsb_total = nsb_total;
   p.stage_bytes = (SH::STAGE + 1023) / 1024 * 1024;
   p.a_bytes = (SH::A_SLOT + 1023) / 1024 * 1024;
-  p.NA = 2;
-  const int bars = 8 * (2 * 8 + 2 * p.NA + 5) + 16;
+  // three A slots (the unpack warps run a super-block ahead of the rescale)
+  // when two stages still fit beside them, else two
+  const int bars = 8 * (2 * 8 + 2 * 4 + 5) + 16;
   const int budget = kSmemPerSm + 4096 - 1024 - bars;
+  p.NA = budget - 3 * p.a_bytes >= 2 * p.stage_bytes ? 3 : 2;
+  if (const char* na_env = std::getenv("WQ_MMQ_NA")) p.NA = std::max(2, std::min(p.NA, std::atoi(na_env)));
   p.NS = std::min(4, (budget - p.NA * p.a_bytes) / p.stage_bytes);
   if (const char* ns_env = std::getenv("WQ_MMQ_NS")) p.NS = std::max(2, std::min(p.NS, std::atoi(ns_env)));
   if (p.NS < 2) return fail(WQ_ERR_UNSUPPORTED, "gemm_q4k_q8: shared memory plan too large");
@@ -1345,7 +1349,7 @@ int launch_mmq_bn(const void* qa8, const void* sda, const void* w, const void* p
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_q4k_q8 launch: ") + cudaGetErrorString(e));
   if ((rc = launch_check("gemm_q4k_q8 launch"))) return rc;
   char buf[64];
-  std::snprintf(buf, sizeof(buf), "q4k.mmq.bn%d.ns%d.s%d%s", BN, p.NS, S, plane ? ".dsc" : "");
+  std::snprintf(buf, sizeof(buf), "q4k.mmq.bn%d.ns%d.na%d.s%d%s", BN, p.NS, p.NA, S, plane ? ".dsc" : "");
   *label = buf;
   return WQ_OK;
 }

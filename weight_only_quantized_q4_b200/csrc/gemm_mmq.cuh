@@ -26,9 +26,11 @@
 //   * one MMA warp issues one tcgen05.mma kind::i8 (K = 32, s32 accumulate)
 //     per chunk into its own TMEM accumulator: a chunk's integer sums must
 //     stay apart because its rescale differs;
-//   * eight rescale warps read each chunk's 128 × BN int32 sums with
-//     tcgen05.ld and add dv·(d·I) + mv·s into fp32 registers (warps w and
-//     w + 4 share TMEM lanes 32(w mod 4).. and split the columns).
+//   * sixteen rescale warps read each chunk's 128 × BN int32 sums with
+//     tcgen05.ld and add dv·(d·I) + mv·s into fp32 registers (the four warps
+//     w ≡ q mod 4 share TMEM lanes 32q.. and split the columns); the int32
+//     sum becomes fp32 exactly by the magic-number route (|I| < 2^22), which
+//     keeps the conversion off the slow conversion pipe.
 // TMEM holds two buffers of U = 256 / BN chunk accumulators, so the MMAs of
 // one buffer overlap the rescale of the other.  Every mbarrier wait is
 // bounded (wq_device.cuh); on a timeout the kernel stops, waits (bounded) for
@@ -47,14 +49,14 @@ struct MMQParams {
   void* y;             // [M, N] fp16
   int M, N, K;
   int S;               // CTAs of a cluster (K slices)
-  int nsb;             // super-blocks per CTA
+  int nsb_total;       // super-blocks of K; rank r of a cluster takes [r·nsb_total/S, (r+1)·nsb_total/S)
   int NS, NA;          // stages (TMA ring), A slots
   int stage_bytes, a_bytes;
   int off_a, off_bar;  // shared-memory offsets (stages start at 0)
 };
 
-constexpr int kMMQWarps = 14;  // producer, MMA issuer, 4 unpack warps, 8 rescale warps
-constexpr int kMMQRescale = 8;
+constexpr int kMMQWarps = 22;  // producer, MMA issuer, 4 unpack warps, 16 rescale warps
+constexpr int kMMQRescale = 16;
 constexpr int kMMQRaw = 128 * 144;  // raw bytes of one stage
 
 template <int BN>
@@ -62,8 +64,9 @@ struct MMQShape {
   static constexpr int U = (256 / BN) < 8 ? (256 / BN) : 8;  // chunk accumulators per TMEM buffer
   static constexpr int TMEM_COLS = 2 * U * BN;
   static constexpr int STAGE = kMMQRaw + 256 * BN + 64 * BN;     // raw, int8 x (2 atoms), (d, s)
-  static constexpr int A_SLOT = 32768 + 8192 + 64 * BN;          // A tile, (dv, mv)[8][128], (d, s)[8][BN]
-  static constexpr int CP = BN >= 32 ? BN / 2 : BN;              // columns per rescale warp
+  static constexpr int A_SLOT = 32768 + 8192 + 64 * BN;          // A tile, (dv, mv)[8][128], d[8][BN] | s[8][BN]
+  static constexpr int CP = BN >= 64 ? BN / 4 : 16;              // columns per rescale warp
+  static constexpr int GROUPS = BN / CP;                          // column groups in use (of four)
 };
 
 // kind::i8 instruction descriptor: D s32, A and B signed 8-bit, both K-major, N = bn, M = 128.
@@ -80,6 +83,48 @@ __device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_
       " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc)
       : "memory");
+}
+
+// 16 consecutive TMEM columns of this warp's 32 lanes, without waiting (the
+// caller issues several, then tcgen05.wait::ld once).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// acc[tokens] += dv·(d·I) + mv·s over 16 columns of one chunk: v the int32
+// sums, d4 / s4 the tokens' d and s (four per float4), two tokens per
+// instruction.  The int32 sum becomes fp32 exactly (|I| < 2^22).
+template <int NP>
+__device__ __forceinline__ void mmq_rescale16(float2 (&acc)[NP], int a0, const uint32_t (&v)[16], const float4* d4,
+                                              const float4* s4, float2 dv2, float2 mv2) {
+#pragma unroll
+  for (int t = 0; t < 16; t += 4) {
+    const float4 dq = d4[t >> 2], sq = s4[t >> 2];
+    float2 i01 = __fadd2_rn(make_float2(__int_as_float(static_cast<int>(v[t]) + 0x4B400000),
+                                        __int_as_float(static_cast<int>(v[t + 1]) + 0x4B400000)),
+                            make_float2(-12582912.0f, -12582912.0f));
+    float2 i23 = __fadd2_rn(make_float2(__int_as_float(static_cast<int>(v[t + 2]) + 0x4B400000),
+                                        __int_as_float(static_cast<int>(v[t + 3]) + 0x4B400000)),
+                            make_float2(-12582912.0f, -12582912.0f));
+    i01 = __fmul2_rn(make_float2(dq.x, dq.y), i01);
+    i23 = __fmul2_rn(make_float2(dq.z, dq.w), i23);
+    float2& x01 = acc[a0 + (t >> 1)];
+    float2& x23 = acc[a0 + (t >> 1) + 1];
+    x01 = __ffma2_rn(dv2, i01, x01);
+    x23 = __ffma2_rn(dv2, i23, x23);
+    x01 = __ffma2_rn(mv2, make_float2(sq.x, sq.y), x01);
+    x23 = __ffma2_rn(mv2, make_float2(sq.z, sq.w), x23);
+  }
+}
+
+// int32 |v| < 2^22 -> fp32, exactly: 1.5·2^23 + v has v in its mantissa field.
+__device__ __forceinline__ float mmq_i2f(uint32_t v) {
+  return __int_as_float(static_cast<int>(v) + 0x4B400000) - 12582912.0f;
 }
 
 // ---------------------------------------------------------------- prepass
@@ -171,8 +216,8 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
   const int tile = blockIdx.x / p.S;
   const int n0 = tile * 128;
   const int m0 = blockIdx.y * BN;
-  const int sb0 = static_cast<int>(rank) * p.nsb;  // first super-block of this CTA
-  const int nsb = p.nsb;
+  const int sb0 = static_cast<int>((static_cast<long long>(rank) * p.nsb_total) / p.S);  // this CTA's K slice
+  const int nsb = static_cast<int>((static_cast<long long>(rank + 1) * p.nsb_total) / p.S) - sb0;
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -227,9 +272,12 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The eight MMAs of a super-block are unrolled (compile-time chunk,
+    // accumulator and descriptor offsets): a rolled chunk loop around the
+    // bounded accumulator waits ran about ten times slower per MMA.
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_i8(BN);
-      int g = 0;  // chunk counter over the CTA's K slice
+      constexpr int kUnits = 8 / SH::U;  // TMEM buffers a super-block fills
       for (int j = 0; j < nsb && !*abort_flag; ++j) {
         const int s = j % p.NS, a = j % p.NA;
         if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>((j / p.NS) & 1)) ||
@@ -238,23 +286,27 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
           break;
         }
         tc_fence_after();
-        const uint8_t* st = smem + s * p.stage_bytes;
-        const uint8_t* ab = smem + p.off_a + a * p.a_bytes;
+        const uint64_t ad0 = umma_smem_desc_sw128(smem_u32(smem + p.off_a + a * p.a_bytes));
+        const uint64_t bd0 = umma_smem_desc_sw128(smem_u32(smem + s * p.stage_bytes + kMMQRaw));
         bool ok = true;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c, ++g) {
-          const int u = g / SH::U, slot = u & 1, e = g - u * SH::U;
-          if (e == 0 && u >= 2) {
+#pragma unroll
+        for (int q = 0; q < kUnits; ++q) {
+          const int u = j * kUnits + q, slot = u & 1;
+          if (u >= 2) {
             if (!mbar_wait_bounded(&acc_empty[slot], static_cast<uint32_t>(((u >> 1) - 1) & 1))) {
               ok = false;
               break;
             }
             tc_fence_after();
           }
-          const uint64_t ad = umma_smem_desc_sw128(smem_u32(ab + (c >> 2) * 16384)) + 2ull * (c & 3);
-          const uint64_t bd = umma_smem_desc_sw128(smem_u32(st + kMMQRaw + (c >> 2) * 128 * BN)) + 2ull * (c & 3);
-          umma_i8(tmem + static_cast<uint32_t>(slot * SH::U * BN + e * BN), ad, bd, idesc);
-          if (e == SH::U - 1) umma_commit(&acc_full[slot]);
+#pragma unroll
+          for (int e = 0; e < SH::U; ++e) {
+            const int c = q * SH::U + e;  // chunk of the super-block: atom c / 4, 32 bytes (c % 4) into it
+            umma_i8(tmem + static_cast<uint32_t>(slot * SH::U * BN + e * BN),
+                    ad0 + static_cast<uint64_t>((c >> 2) * (16384 >> 4) + 2 * (c & 3)),
+                    bd0 + static_cast<uint64_t>((c >> 2) * ((128 * BN) >> 4) + 2 * (c & 3)), idesc);
+          }
+          umma_commit(&acc_full[slot]);
         }
         if (!ok) {
           *abort_flag = 1;
@@ -310,10 +362,16 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
           coef[c * 128 + r] = make_float2(__fmul_rn(d, static_cast<float>(sc)), -__fmul_rn(dmin, static_cast<float>(mn)));
         }
       }
-      // the (d, s) pairs of the BN tokens, [8][BN]
-      const uint4* sd_src = reinterpret_cast<const uint4*>(st + kMMQRaw + 256 * BN);
-      uint4* sd_dst = reinterpret_cast<uint4*>(ab + 32768 + 8192);
-      for (int i = r; i < 4 * BN; i += 128) sd_dst[i] = sd_src[i];
+      // the (d, s) pairs of the BN tokens, chunk by chunk: [8][BN] pairs ->
+      // per chunk BN values of d, then BN values of s (two-token operands)
+      const float2* sd_src = reinterpret_cast<const float2*>(st + kMMQRaw + 256 * BN);
+      float* sd_dst = reinterpret_cast<float*>(ab + 32768 + 8192);
+      for (int i = r; i < 8 * BN; i += 128) {
+        const int c = i / BN, t = i - c * BN;
+        const float2 v = sd_src[i];
+        sd_dst[c * 2 * BN + t] = v.x;
+        sd_dst[c * 2 * BN + BN + t] = v.y;
+      }
       fence_proxy_async_smem();  // generic-proxy writes of the A tile -> visible to the tensor core
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (r == 0) {
@@ -323,15 +381,15 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
     }
   } else {
     // ------------------------------------------------------------ rescale warps
-    const int lq = warp & 3, ch = (warp - 6) >> 2;
+    const int lq = warp & 3, cg = (warp - 6) >> 2;
     const int trow = lq * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-    const bool active = BN >= 32 || ch == 0;
-    const int c_begin = BN >= 32 ? ch * SH::CP : 0;
-    float acc[SH::CP];
+    const bool active = cg < SH::GROUPS;
+    const int c_begin = active ? cg * SH::CP : 0;
+    float2 acc[SH::CP / 2];  // tokens (2i, 2i + 1) of the warp's columns
 #pragma unroll
-    for (int i = 0; i < SH::CP; ++i) acc[i] = 0.f;
-    int g = 0;
+    for (int i = 0; i < SH::CP / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+    constexpr int kUnits = 8 / SH::U;
     for (int j = 0; j < nsb && !*abort_flag; ++j) {
       const int a = j % p.NA;
       if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>((j / p.NA) & 1))) {
@@ -340,38 +398,56 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
       }
       const uint8_t* ab = smem + p.off_a + a * p.a_bytes;
       const float2* coef = reinterpret_cast<const float2*>(ab + 32768);
-      const float2* sd = reinterpret_cast<const float2*>(ab + 32768 + 8192);
+      const float* sd = reinterpret_cast<const float*>(ab + 32768 + 8192);
       bool ok = true;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c, ++g) {
-        const int u = g / SH::U, slot = u & 1, e = g - u * SH::U;
-        if (e == 0) {
-          if (!mbar_wait_bounded(&acc_full[slot], static_cast<uint32_t>((u >> 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < kUnits; ++q) {
+        const int u = j * kUnits + q, slot = u & 1;
+        if (!mbar_wait_bounded(&acc_full[slot], static_cast<uint32_t>((u >> 1) & 1))) {
+          ok = false;
+          break;
         }
-        if (active) {
-          const float2 cf = coef[c * 128 + trow];
-          const uint32_t col = static_cast<uint32_t>(slot * SH::U * BN + e * BN + c_begin);
+        tc_fence_after();
+        if (active && SH::CP > 16) {
 #pragma unroll
-          for (int cc = 0; cc < SH::CP; cc += 16) {
-            uint32_t v[16];
-            tmem_ld16(lane_base + col + cc, v);
+          for (int e = 0; e < SH::U; ++e) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              const float2 ds = sd[c * BN + c_begin + cc + t];
-              acc[cc + t] = fmaf(cf.x, ds.x * static_cast<float>(static_cast<int>(v[t])), acc[cc + t]);
-              acc[cc + t] = fmaf(cf.y, ds.y, acc[cc + t]);
+            for (int cc = 0; cc < SH::CP; cc += 16) {
+              const int c = q * SH::U + e;
+              const float2 cf = coef[c * 128 + trow];
+              uint32_t v[16];
+              tmem_ld16_nowait(lane_base + static_cast<uint32_t>(slot * SH::U * BN + e * BN + c_begin + cc), v);
+              tmem_wait_ld();
+              mmq_rescale16(acc, cc >> 1, v, reinterpret_cast<const float4*>(sd + c * 2 * BN + c_begin + cc),
+                            reinterpret_cast<const float4*>(sd + c * 2 * BN + BN + c_begin + cc),
+                            make_float2(cf.x, cf.x), make_float2(cf.y, cf.y));
+            }
+          }
+        } else if (active) {
+          // two chunks per round: both TMEM loads in flight before one wait
+#pragma unroll
+          for (int e = 0; e < SH::U; e += 2) {
+#pragma unroll
+            for (int cc = 0; cc < SH::CP; cc += 16) {  // 16 columns per load (register budget)
+              const int c0 = q * SH::U + e, c1 = c0 + 1;
+              const uint32_t col = static_cast<uint32_t>(slot * SH::U * BN + e * BN + c_begin + cc);
+              uint32_t va[16], vb[16];
+              tmem_ld16_nowait(lane_base + col, va);
+              tmem_ld16_nowait(lane_base + col + BN, vb);
+              const float2 cf0 = coef[c0 * 128 + trow], cf1 = coef[c1 * 128 + trow];
+              tmem_wait_ld();
+              mmq_rescale16(acc, cc >> 1, va, reinterpret_cast<const float4*>(sd + c0 * 2 * BN + c_begin + cc),
+                            reinterpret_cast<const float4*>(sd + c0 * 2 * BN + BN + c_begin + cc),
+                            make_float2(cf0.x, cf0.x), make_float2(cf0.y, cf0.y));
+              mmq_rescale16(acc, cc >> 1, vb, reinterpret_cast<const float4*>(sd + c1 * 2 * BN + c_begin + cc),
+                            reinterpret_cast<const float4*>(sd + c1 * 2 * BN + BN + c_begin + cc),
+                            make_float2(cf1.x, cf1.x), make_float2(cf1.y, cf1.y));
             }
           }
         }
-        if (e == SH::U - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc5_arrive(&acc_empty[slot]);
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc5_arrive(&acc_empty[slot]);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -389,7 +465,8 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
 #pragma unroll
         for (int i = 0; i < SH::CP; ++i) {
           const int m = m0 + c_begin + i;
-          if (m < p.M && yrow < p.N) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(acc[i]);
+          const float v = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
+          if (m < p.M && yrow < p.N) y[static_cast<long long>(m) * p.N + yrow] = __float2half_rn(v);
         }
       }
     }
@@ -398,10 +475,10 @@ __global__ void __launch_bounds__(kMMQWarps * 32, 1) gemm_mmq_kernel(const __gri
       // of the CTA is past the main loop (named barrier 2 over the rescale
       // warps only after the block-wide sync below)
       float* part = reinterpret_cast<float*>(smem);
-      asm volatile("bar.sync 2, 256;" ::: "memory");
+      asm volatile("bar.sync 2, 512;" ::: "memory");
       if (active)
 #pragma unroll
-        for (int i = 0; i < SH::CP; ++i) part[trow * BN + c_begin + i] = acc[i];
+        for (int i = 0; i < SH::CP; ++i) part[trow * BN + c_begin + i] = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
     }
   }
 
