@@ -235,6 +235,44 @@ int dequant_q4k(const void* w_q4k, const void* w_dsc, float* w_out, int N, int K
 int dequant_mxfp4(const void* w_packed, const void* scales_e8m0, float* w_out, int N, int K, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Row-split (tensor-parallel) layers: each GPU holds a run of W's rows and
+ * computes those outputs; the all-gather of y is done by the GEMV's own
+ * stores.  No counterpart on the pages (they run one GPU): this is the
+ * N-split the hot-path scope table names for more than one GPU.
+ * ------------------------------------------------------------------------- */
+
+/* Rows [*n0, *n1) of rank `rank` of `world` for an N-row weight split in
+ * units of `align` rows (16: whole B200_V1 bands), as evenly as possible
+ * (the first N/align mod world ranks take one unit more; a rank may get
+ * none, n0 == n1).  Host only.  Errors: WQ_ERR_ARG. */
+int wq_tp_rows(int N, int world, int rank, int align, int* n0, int* n1);
+
+/* y rows n_offset .. n_offset + N_shard - 1 of an int4 layer whose B200_V1
+ * shard (rows n_offset.. of the full weight, repacked alone by
+ * wq_repack_int4) is w_shard, stored into every one of the n_dsts (1..8)
+ * buffers y_dsts[d] (a host array of device pointers), each a full [M][N_total]
+ * fp16 output: this GPU's own y and, mapped into this process with
+ * wq_ipc_open, the other GPUs' copies, so that when every rank's call has
+ * finished each GPU holds all of y (the caller orders that with its own
+ * barrier, e.g. stream synchronize + a host or NCCL barrier).  Runs the B200_V1
+ * band kernel (blocks >= 128, K % 128 == 0); other columns are not touched.
+ * x 16-byte aligned, destinations 2-byte aligned.  Errors: WQ_ERR_ARG,
+ * WQ_ERR_ALIGN, WQ_ERR_UNSUPPORTED, WQ_ERR_DEVICE, WQ_ERR_CUDA. */
+int gemv_int4_tp(const void* x_f16, const void* w_shard, void* const* y_dsts, int n_dsts, int M, int N_shard, int K,
+                 int block_size, int N_total, int n_offset, void* stream);
+
+/* CUDA IPC for the destinations of gemv_int4_tp.  wq_ipc_handle: the 64-byte
+ * handle of the allocation that holds dev_ptr (a pointer may sit inside a
+ * larger allocation, e.g. one made by a caching allocator) and the byte
+ * offset of dev_ptr in it.  wq_ipc_open: another process's (handle, offset)
+ * mapped into this one (peer access enabled lazily), the pointer to the same
+ * bytes.  wq_ipc_close: releases that mapping (same pointer and offset).
+ * Errors: WQ_ERR_ARG, WQ_ERR_CUDA. */
+int wq_ipc_handle(const void* dev_ptr, void* handle_out, unsigned long long* offset_out);
+int wq_ipc_open(const void* handle, unsigned long long offset, void** dev_ptr_out);
+int wq_ipc_close(void* dev_ptr, unsigned long long offset);
+
+/* ---------------------------------------------------------------------------
  * int8-activation batched q4_K (minfer doc 62 "r59 — q4_K W_dsc plane", §3.2:
  * the MMQ dispatch arm quantizes the activations to int8 in a prepass and
  * runs an integer GEMM whose (chunk, row) pairs are rescaled by the §2.1

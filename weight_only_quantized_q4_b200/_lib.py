@@ -42,6 +42,11 @@ SIGNATURES = {
     "dequant_q4k": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "dequant_mxfp4": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
     "quantize_q8": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
+    "wq_tp_rows": (_i, [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "gemv_int4_tp": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_void_p), _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "wq_ipc_handle": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_ulonglong)]),
+    "wq_ipc_open": (_i, [_vp, ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_void_p)]),
+    "wq_ipc_close": (_i, [_vp, ctypes.c_ulonglong]),
     "gemm_q4k_q8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "wq_q8_bytes": (_sz, [_i, _i]),
     "wq_q8_scale_bytes": (_sz, [_i, _i]),

@@ -171,3 +171,34 @@ def wq_device_status() -> None:
 
 def wq_test_expire_wait(limit_ns: int, stream=None) -> None:
     _check(lib().wq_test_expire_wait(int(limit_ns), _stream(stream)), "wq_test_expire_wait")
+
+
+def wq_tp_rows(N, world, rank, align=16):
+    """Rows (n0, n1) of rank `rank` in a row split of N rows over `world` GPUs."""
+    n0, n1 = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().wq_tp_rows(N, world, rank, align, ctypes.byref(n0), ctypes.byref(n1)), "wq_tp_rows")
+    return n0.value, n1.value
+
+
+def gemv_int4_tp(x, w_shard, y_dsts, M, N_shard, K, block_size, N_total, n_offset, stream=None):
+    ptrs = (ctypes.c_void_p * len(y_dsts))(*[_ptr(t) for t in y_dsts])
+    _check(lib().gemv_int4_tp(_ptr(x), _ptr(w_shard), ptrs, len(y_dsts), M, N_shard, K, block_size, N_total, n_offset,
+                              _stream(stream)), "gemv_int4_tp")
+
+
+def wq_ipc_handle(t):
+    """(64-byte handle, byte offset) of the device allocation holding t."""
+    buf = ctypes.create_string_buffer(64)
+    off = ctypes.c_ulonglong(0)
+    _check(lib().wq_ipc_handle(_ptr(t), buf, ctypes.byref(off)), "wq_ipc_handle")
+    return buf.raw, off.value
+
+
+def wq_ipc_open(handle: bytes, offset: int) -> int:
+    p = ctypes.c_void_p(0)
+    _check(lib().wq_ipc_open(ctypes.create_string_buffer(handle, 64), offset, ctypes.byref(p)), "wq_ipc_open")
+    return int(p.value)
+
+
+def wq_ipc_close(ptr: int, offset: int) -> None:
+    _check(lib().wq_ipc_close(ptr, offset), "wq_ipc_close")

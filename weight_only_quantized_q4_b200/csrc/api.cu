@@ -560,6 +560,9 @@ bool plan_v1_geom(int M, int N, int K, int block_size, int C, int W, int n_clust
   p.M = M;
   p.N = N;
   p.K = K;
+  p.n_dst = 0;  // y only, unless the caller names destinations (row-split layers)
+  p.y_ld = 0;
+  p.y_off = 0;
   p.n_bands = (N + 15) / 16;
   p.tpb = tpb;
   p.tpc = tpb / C;
@@ -752,9 +755,16 @@ int launch_v1r(const V1RPlan& plan, cudaStream_t st) {
 }
 
 
-int launch_v1(const V1Plan& plan, cudaStream_t st) {
+int launch_v1(const V1Plan& plan_in, cudaStream_t st) {
   int rc = v1_configure();
   if (rc) return rc;
+  V1Plan plan = plan_in;
+  if (plan.p.n_dst == 0) {  // a plain call: y is the only destination
+    plan.p.ydst[0] = plan.p.y;
+    plan.p.n_dst = 1;
+    plan.p.y_ld = plan.p.N;
+    plan.p.y_off = 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.grid, 1, 1);
   cfg.blockDim = dim3(plan.threads, 1, 1);
@@ -1692,6 +1702,110 @@ int gemv_mxfp4(const void* x_f16, const void* w_packed, const void* scales_e8m0,
   char buf[64];
   std::snprintf(buf, sizeof(buf), "mxfp4.gemv.mx.m%d%s", std::min(8, M), M > 8 ? ".chunked" : "");
   set_last_kernel(buf);
+  return WQ_OK;
+}
+
+int wq_tp_rows(int N, int world, int rank, int align, int* n0, int* n1) {
+  if (N <= 0 || world <= 0 || rank < 0 || rank >= world || align <= 0 || !n0 || !n1)
+    return fail(WQ_ERR_ARG, "wq_tp_rows: need N, world, align > 0, 0 <= rank < world and output pointers");
+  const long long units = (static_cast<long long>(N) + align - 1) / align;
+  const long long base = units / world, extra = units % world;
+  const long long u0 = rank * base + std::min<long long>(rank, extra);
+  const long long cnt = base + (rank < extra ? 1 : 0);
+  *n0 = static_cast<int>(std::min<long long>(N, u0 * align));
+  *n1 = static_cast<int>(std::min<long long>(N, (u0 + cnt) * align));
+  return WQ_OK;
+}
+
+int gemv_int4_tp(const void* x_f16, const void* w_shard, void* const* y_dsts, int n_dsts, int M, int N_shard, int K,
+                 int block_size, int N_total, int n_offset, void* stream) {
+  int rc = check_dims(M, N_shard, K);
+  if (rc) return rc;
+  if ((rc = check_int4(K, block_size, WQ_LAYOUT_B200_V1))) return rc;
+  if (!x_f16 || !w_shard || !y_dsts) return fail(WQ_ERR_ARG, "gemv_int4_tp: null pointer");
+  if (n_dsts < 1 || n_dsts > kV1MaxDst) return fail(WQ_ERR_ARG, "gemv_int4_tp: 1 to 8 destinations");
+  if (n_offset < 0 || N_total < N_shard || n_offset > N_total - N_shard)
+    return fail(WQ_ERR_ARG, "gemv_int4_tp: the shard's rows must lie inside the full output");
+  for (int d = 0; d < n_dsts; ++d)
+    if (!y_dsts[d] || !aligned2(y_dsts[d])) return fail(WQ_ERR_ALIGN, "gemv_int4_tp: destinations must be 2-byte aligned device pointers");
+  if (!aligned16(x_f16) || !aligned16(w_shard)) return fail(WQ_ERR_ALIGN, "gemv_int4_tp: x and w_shard must be 16-byte aligned");
+  if (const char* force = forced_variant())
+    if (std::strcmp(force, "v1s") != 0)
+      return fail(WQ_ERR_UNSUPPORTED, std::string("WQ_FORCE_KERNEL=") + force + ": the row-split GEMV runs the v1s kernel only");
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int mc_first = 0;
+  for (int m0 = 0; m0 < M; m0 += 8) {  // batches past 8 rows in chunks of 8 (the shard is read once per chunk)
+    const int mc = std::min(8, M - m0);
+    if (m0 == 0) mc_first = mc;
+    V1Plan vplan;
+    if (!plan_v1(mc, N_shard, K, block_size, di.sms, &vplan))
+      return fail(WQ_ERR_UNSUPPORTED, "gemv_int4_tp: needs blocks >= 128 and K % 128 == 0 (B200_V1 band kernel)");
+    vplan.p.x = static_cast<const uint8_t*>(x_f16) + 2ll * m0 * K;
+    vplan.p.w = static_cast<const uint8_t*>(w_shard);
+    vplan.p.y = static_cast<uint8_t*>(y_dsts[0]) + 2ll * m0 * N_total;
+    for (int d = 0; d < n_dsts; ++d) vplan.p.ydst[d] = static_cast<uint8_t*>(y_dsts[d]) + 2ll * m0 * N_total;
+    vplan.p.n_dst = n_dsts;
+    vplan.p.y_ld = N_total;
+    vplan.p.y_off = n_offset;
+    if ((rc = launch_v1(vplan, st))) return rc;
+  }
+  char buf[64];
+  std::snprintf(buf, sizeof(buf), "int4.gemv.v1s.tp.m%d.d%d%s", mc_first, n_dsts, M > 8 ? ".chunked" : "");
+  set_last_kernel(buf);
+  return WQ_OK;
+}
+
+// cuMemGetAddressRange from the driver, looked up once (no link-time
+// dependency on libcuda): the allocation an IPC handle stands for.
+using MemRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+MemRangeFn mem_range_fn() {
+  static MemRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<MemRangeFn>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+int wq_ipc_handle(const void* dev_ptr, void* handle_out, unsigned long long* offset_out) {
+  if (!dev_ptr || !handle_out || !offset_out) return fail(WQ_ERR_ARG, "wq_ipc_handle: null pointer");
+  MemRangeFn range = mem_range_fn();
+  if (!range) return fail(WQ_ERR_CUDA, "cuMemGetAddressRange is not available from the driver");
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return fail(WQ_ERR_ARG, "wq_ipc_handle: not a device allocation");
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaIpcGetMemHandle: ") + cudaGetErrorString(e));
+  std::memcpy(handle_out, &h, sizeof(h));
+  *offset_out = static_cast<unsigned long long>(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return WQ_OK;
+}
+
+int wq_ipc_open(const void* handle, unsigned long long offset, void** dev_ptr_out) {
+  if (!handle || !dev_ptr_out) return fail(WQ_ERR_ARG, "wq_ipc_open: null pointer");
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  void* base = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaIpcOpenMemHandle: ") + cudaGetErrorString(e));
+  *dev_ptr_out = static_cast<uint8_t*>(base) + offset;
+  return WQ_OK;
+}
+
+int wq_ipc_close(void* dev_ptr, unsigned long long offset) {
+  if (!dev_ptr) return fail(WQ_ERR_ARG, "wq_ipc_close: null pointer");
+  cudaError_t e = cudaIpcCloseMemHandle(static_cast<uint8_t*>(dev_ptr) - offset);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaIpcCloseMemHandle: ") + cudaGetErrorString(e));
   return WQ_OK;
 }
 

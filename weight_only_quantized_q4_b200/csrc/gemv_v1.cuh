@@ -34,10 +34,18 @@
 
 namespace wq {
 
+constexpr int kV1MaxDst = 8;
+
 struct V1Params {
   const void* x;     // [M][K] fp16
   const uint8_t* w;  // B200_V1 stream
   void* y;           // [M][N] fp16
+  // Where y goes: n_dst buffers of [M][y_ld] fp16 (this GPU's output and, for
+  // a row-split layer, the other GPUs' copies mapped into this process), the
+  // N rows of this call landing at columns y_off .. y_off + N - 1 of each.
+  // A plain call has one destination, y itself (y_ld = N, y_off = 0).
+  void* ydst[kV1MaxDst];
+  int n_dst, y_ld, y_off;
   int M, N, K;
   int n_bands;       // ceil(N / 16)
   int tpb;           // tiles per band (K / 128)
@@ -64,6 +72,13 @@ struct V1Params {
 };
 
 namespace v1d {
+
+// y[n][r] (fp16, RN) into every destination of the call
+__device__ __forceinline__ void store_y(const V1Params& p, int n, int r, float v) {
+  const __half h = __float2half_rn(v);
+  for (int d = 0; d < p.n_dst; ++d)
+    reinterpret_cast<__half*>(p.ydst[d])[static_cast<long long>(n) * p.y_ld + p.y_off + r] = h;
+}
 
 constexpr int kBarFull0 = 1;  // named barriers 1, 2: partial slot s is full
 constexpr int kBarFree0 = 3;  // named barriers 3, 4: partial slot s is free again
@@ -324,7 +339,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
         if (p.C > 1) {
           part[(bl * 16 + row) * p.M + n] = sum;
         } else if (r0 + row < p.N && !*abort_flag) {
-          reinterpret_cast<__half*>(p.y)[static_cast<long long>(n) * p.N + r0 + row] = __float2half_rn(sum * kYScale);
+          v1d::store_y(p, n, r0 + row, sum * kYScale);
         }
       }
       if (bl + 2 < n_bl) v1d::bar_arrive(v1d::kBarFree0 + s, nthr_all);
@@ -453,7 +468,7 @@ __global__ void __launch_bounds__(kV1MaxWarps * 32, 1) gemv_v1_kernel(const V1Pa
       float sum = 0.f;
       for (int c = 0; c < p.C; ++c) sum += v1d::dsmem_ld(part + i, static_cast<uint32_t>(c));
       if (r < p.N && !*abort_flag)
-        reinterpret_cast<__half*>(p.y)[static_cast<long long>(n) * p.N + r] = __float2half_rn(sum * kYScale);
+        v1d::store_y(p, n, r, sum * kYScale);
     }
     v1d::cluster_sync();
   }
