@@ -626,11 +626,13 @@ def test_full_batched_sampled(fmt, N, K):
 @gpu
 @pytest.mark.parametrize("M", [9, 16, 33, 64, 128, 200])
 @pytest.mark.parametrize("N,K,bs", [(300, 1024, 128), (37, 4096, 256), (1000, 384, 128), (16, 128, 128)])
-def test_gemm_v1tc_batched(M, N, K, bs):
-    """Batches of 9 and more over B200_V1 int4 weights run the tcgen05 kernel
-    that reads the band stream: ragged row tiles (N = 300, 37, 1000), an odd
-    number of 128-k steps (K = 384), a single step (K = 128), two batch tiles
-    (M = 200).  Guard bands around every output; two calls agree bit for bit."""
+def test_gemm_v1tc_batched(M, N, K, bs, monkeypatch):
+    """The tcgen05 kernel that reads the B200_V1 band stream (forced: below 17
+    rows the default is the chunked warp-MMA GEMV): ragged row tiles (N = 300,
+    37, 1000), an odd number of 128-k steps (K = 384), a single step (K = 128),
+    two batch tiles (M = 200).  Guard bands around every output; two calls
+    agree bit for bit."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
     c = Int4Case(M, N, K, bs, True, workload=40, layout=wq.WQ_LAYOUT_B200_V1)
     y = c.run()
     assert ".gemm.v1tc." in wq.last_kernel(), wq.last_kernel()
@@ -645,6 +647,7 @@ def test_gemm_v1tc_cluster_split_k(S, M, monkeypatch):
     """K split over a cluster of S CTAs whose fp32 accumulators are added
     through distributed shared memory in rank order."""
     monkeypatch.setenv("WQ_V1TC_S", str(S))
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
     c = Int4Case(M, 300, 4096, 128, True, workload=41, layout=wq.WQ_LAYOUT_B200_V1)
     y = c.run()
     label = wq.last_kernel()
@@ -657,6 +660,7 @@ def test_gemm_v1tc_cluster_split_k(S, M, monkeypatch):
 def test_gemm_v1tc_forced_split_follows_the_rule(monkeypatch):
     """A forced split must leave every CTA an even number of 128-k steps."""
     monkeypatch.setenv("WQ_V1TC_S", "4")
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
     c = Int4Case(16, 300, 768, 128, True, workload=41, layout=wq.WQ_LAYOUT_B200_V1)
     with pytest.raises(wq.WQError) as e:
         c.run()
@@ -669,6 +673,7 @@ def test_gemm_v1tc_weights_beyond_fp16_range(S, monkeypatch):
     """Half the rows with scales up to 9000 (|w| up to 135000): formed as
     w·2^-e and rescaled in fp32, every output finite and within tolerance."""
     monkeypatch.setenv("WQ_V1TC_S", str(S))
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
     M, N, K = 16, 300, 2048
     rng = np.random.default_rng(42)
     big = rng.random(N) < 0.5
@@ -707,7 +712,8 @@ def test_full_batched_v1tc_sampled(N, K):
         wq.gemv_int4_blockwise(dev(x), g.t, None, None, gy.t, M, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1)
         torch.cuda.synchronize()
         label = wq.last_kernel()
-        assert ".gemm.v1tc." in label, label
+        # up to 16 rows the chunked warp-MMA GEMV is the default, from 17 the tcgen05 kernel
+        assert (".gemv." in label and label.endswith(".chunked")) if M <= 16 else (".gemm.v1tc." in label), label
         gy.check(f"v1tc full {N}x{K} M={M}")
         y = gy.t.cpu().numpy().astype(np.float64)
         check(y[:, rows], Wr, x, f"v1tc full {N}x{K} M={M} [{label}]")

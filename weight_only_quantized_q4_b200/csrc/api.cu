@@ -1384,7 +1384,11 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     if constexpr (F == Fmt::Int4) {
       // B200_V1 int4 with blocks of at least 128: the tcgen05 kernel reads the band stream itself
       const bool v1tc_ok = layout == WQ_LAYOUT_B200_V1 && K % 128 == 0 && block_size >= 128 && aligned16(x);
-      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : M >= 9;
+      // up to 16 rows of x the warp-MMA GEMV in two chunks of 8 is faster (B200,
+      // 14336x4096 M=16: 31.4 against 39.0 us; 4096x14336: 27.1 against 39.0;
+      // 4096x4096: 11.6 against 16.7); from 32 rows the tcgen05 kernel is
+      // (M=32 14336x4096: 39.0 against 62.2)
+      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : M > 16;
       if (v1tc_ok && want_v1tc) {
         rc = launch_v1tc(x, w, y, M, N, K, block_size, di.sms, st, &label);
         if (rc) return rc;
@@ -1458,7 +1462,12 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
         continue;
       }
       V1Plan vplan;
-      const bool want_v1 = force ? std::strcmp(force, "v1s") == 0 : true;
+      // the band-stream kernel for up to 3 rows of x per chunk; from 4 rows the
+      // warp-MMA GEMV over the same stream is faster (B200, M=4 / 6 / 8:
+      // 4096x4096 5.7 / 5.8 / 5.9 against 6.6 / 7.4 / 8.2 us; 11008x4096 12.0 /
+      // 12.1 / 12.2 against 12.2 / 14.2 / 15.5; 4096x14336 M=4 13.2 against
+      // 13.6; 14336x4096 M=4 15.8 against 15.3, M=6 15.9 against 18.2)
+      const bool want_v1 = force ? std::strcmp(force, "v1s") == 0 : mc <= 3;
       if (want_v1 && layout == WQ_LAYOUT_B200_V1 && aligned16(xc) &&
           plan_v1(mc, N, K, block_size, di.sms, &vplan)) {
         vplan.p.x = xc;
