@@ -41,7 +41,7 @@
  *  - The first call on a device configures kernel attributes and looks up the
  *    driver's tensor-map encoder; make it before capturing a CUDA graph.
  *  - Environment variables read at each call, for tests and tuning only:
- *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc | mx | mmq) pins a kernel
+ *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc | v1w | mx | mmq) pins a kernel
  *    family (a call that family cannot run returns WQ_ERR_UNSUPPORTED; there
  *    is no silent substitute), WQ_PDL=0 disables programmatic dependent
  *    launch, and WQ_V1_*, WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch

@@ -178,7 +178,7 @@ class BF16Case:
         return oracle.dequant_bf16(self.xb, self.M, self.K)
 
 
-VARIANTS = ("tc", "cc", "simple", "tc5", "v1s", "v1r", "v1k", "v1tc", None)
+VARIANTS = ("tc", "cc", "simple", "tc5", "v1s", "v1r", "v1k", "v1tc", "v1w", None)
 
 
 def each_variant(run, W, x, what):

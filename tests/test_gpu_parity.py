@@ -712,8 +712,76 @@ def test_full_batched_v1tc_sampled(N, K):
         wq.gemv_int4_blockwise(dev(x), g.t, None, None, gy.t, M, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1)
         torch.cuda.synchronize()
         label = wq.last_kernel()
-        # up to 16 rows the chunked warp-MMA GEMV is the default, from 17 the tcgen05 kernel
-        assert (".gemv." in label and label.endswith(".chunked")) if M <= 16 else (".gemm.v1tc." in label), label
+        # up to 24 rows the warp-MMA GEMM over the stream is the default, from 25 the tcgen05 kernel
+        assert (".gemm.v1w." in label) if M <= 24 else (".gemm.v1tc." in label), label
         gy.check(f"v1tc full {N}x{K} M={M}")
         y = gy.t.cpu().numpy().astype(np.float64)
         check(y[:, rows], Wr, x, f"v1tc full {N}x{K} M={M} [{label}]")
+
+
+# ----------------------------------------------------- warp-MMA GEMM over the B200_V1 stream
+
+@gpu
+@pytest.mark.parametrize("M", [9, 16, 17, 24, 25, 33, 40, 57, 64])
+@pytest.mark.parametrize("N,K,bs", [(300, 1024, 128), (37, 4096, 256), (1000, 384, 128), (16, 128, 128), (129, 896, 256)])
+def test_gemm_v1w_batched(M, N, K, bs, monkeypatch):
+    """The warp-MMA GEMM over the B200_V1 stream (M = 9..64, every column-group
+    count 2..8 and both warp arrangements): ragged row tiles, an odd number of
+    128-k steps, a single step, a ragged last block (896 = 3·256 + 128).  Guard
+    bands around every output; two calls agree bit for bit."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1w")
+    c = Int4Case(M, N, K, bs, True, workload=44, layout=wq.WQ_LAYOUT_B200_V1)
+    y = c.run()
+    assert ".gemm.v1w." in wq.last_kernel(), wq.last_kernel()
+    check(y, c.W(), c.x, f"v1w M={M} N={N} K={K} bs={bs}")
+    assert np.array_equal(y, c.run())
+
+
+@gpu
+@pytest.mark.parametrize("S", [1, 2, 4, 8])
+@pytest.mark.parametrize("M", [16, 48])
+@pytest.mark.parametrize("K", [4096, 1408])
+def test_gemm_v1w_cluster_split_k(S, M, K, monkeypatch):
+    """K split over a cluster of S CTAs (K = 1408: eleven steps, uneven runs
+    per rank), partials added through distributed shared memory in rank order."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1w")
+    monkeypatch.setenv("WQ_V1W_S", str(S))
+    c = Int4Case(M, 300, K, 128, True, workload=45, layout=wq.WQ_LAYOUT_B200_V1)
+    y = c.run()
+    label = wq.last_kernel()
+    assert ".gemm.v1w." in label and label.endswith(f".s{S}"), label
+    check(y, c.W(), c.x, f"v1w M={M} K={K} S={S}")
+    assert np.array_equal(y, c.run())
+
+
+@gpu
+@pytest.mark.parametrize("T", [1, 2, 5])
+def test_gemm_v1w_raw_slot_sizes(T, monkeypatch):
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1w")
+    monkeypatch.setenv("WQ_V1W_T", str(T))
+    monkeypatch.setenv("WQ_V1W_S", "1")  # all 16 steps in one CTA, so T is not capped by the slice
+    c = Int4Case(33, 200, 2048, 128, True, workload=46, layout=wq.WQ_LAYOUT_B200_V1)
+    y = c.run()
+    assert f".t{T}." in wq.last_kernel(), wq.last_kernel()
+    check(y, c.W(), c.x, f"v1w T={T}")
+
+
+@gpu
+@pytest.mark.parametrize("N,K", FULL_BATCHED)
+def test_full_batched_v1w_sampled(N, K, monkeypatch):
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1w")
+    t = synth.int4_weights(N, K, 128, scale_lo=0.002, scale_hi=0.01, with_zeros=True, workload=5)
+    g = Guarded((wq.wq_int4_packed_bytes(N, K, 128),), torch.uint8)
+    wq.wq_repack_int4(dev(t["w_packed"]), dev(t["scales"]), dev(t["zeros"]), g.t, N, K, 128)
+    torch.cuda.synchronize()
+    rows = sample_rows(N)
+    Wr = oracle.dequant_int4(t["w_packed"][rows], t["scales"][rows], t["zeros"][rows], len(rows), K, 128)
+    for M in (16, 32, 64):
+        x = synth.activations_f16(M, K, workload=5)
+        gy = Guarded((M, N), torch.float16)
+        wq.gemv_int4_blockwise(dev(x), g.t, None, None, gy.t, M, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1)
+        torch.cuda.synchronize()
+        assert ".gemm.v1w." in wq.last_kernel(), wq.last_kernel()
+        gy.check(f"v1w full {N}x{K} M={M}")
+        y = gy.t.cpu().numpy().astype(np.float64)
+        check(y[:, rows], Wr, x, f"v1w full {N}x{K} M={M}")

@@ -28,6 +28,7 @@
 #include "gemm_v1tc.cuh"
 #include "gemv_mxfp4.cuh"
 #include "gemm_mmq.cuh"
+#include "gemm_v1w.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -1364,6 +1365,99 @@ int launch_mmq_bn(const void* qa8, const void* sda, const void* w, const void* p
   return WQ_OK;
 }
 
+// Warp-MMA GEMM over the int4 B200_V1 stream (M = 9..64): MG = ceil(M / 8)
+// column groups of 8 batch rows, one CTA per 8 bands and K slice, clusters of
+// S CTAs splitting K while the CTAs still fit one wave.
+template <int MG>
+int launch_v1w_mg(const void* x, const uint8_t* w, void* y, int M, int N, int K, int block_size, int sms,
+                  cudaStream_t st, std::string* label) {
+  V1WParams p{};
+  p.w = w;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_bands = (N + 15) / 16;
+  p.tpb = K / 128;
+  p.tb = int4_v1_tile_bytes(block_size);
+  const int n_tiles = (p.n_bands + kV1WBands - 1) / kV1WBands;
+  int S = 1;
+  while (S < 8 && n_tiles * S * 2 <= sms && p.tpb >= 4 * S) S *= 2;  // every rank keeps at least two steps
+  if (const char* s_env = std::getenv("WQ_V1W_S")) {  // tests and tuning
+    const int sf = std::atoi(s_env);
+    if (sf == 1 || sf == 2 || sf == 4 || sf == 8) {
+      if (p.tpb < sf) return fail(WQ_ERR_ARG, "WQ_V1W_S exceeds the 128-k steps of K");
+      S = sf;
+    }
+  }
+  p.S = S;
+  const int xslot = 8 * MG * 256;
+  p.NX = 4;
+  p.NR = 3;
+  const int bars = 8 * (2 * p.NR + 2 * p.NX) + 16;
+  const int budget = kSmemPerSm + 4096 - 1024 - bars;
+  const int min_steps = p.tpb / S;
+  p.T = std::min(16, (budget - p.NX * xslot - 1024) / (p.NR * kV1WBands * p.tb));
+  if (const char* t_env = std::getenv("WQ_V1W_T")) p.T = std::max(1, std::min(p.T, std::atoi(t_env)));
+  p.T = std::max(1, std::min(p.T, std::max(1, min_steps)));
+  p.off_x = (p.NR * kV1WBands * p.T * p.tb + 1023) / 1024 * 1024;
+  p.off_bar = p.off_x + p.NX * xslot;
+  const int smem = 1024 + p.off_bar + bars;
+  if (smem > kSmemPerSm + 4096 || p.T < 1) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1w: shared memory plan too large");
+  if (v1w_par(MG) * 16 * kV1WBands * 8 * MG * 4 > p.off_bar) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1w: partials do not fit");
+  int rc = encode_2d(&p.tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, 2ull * K, 64, 8 * MG,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  {
+    static std::mutex mu;
+    static bool configured[64] = {};
+    std::lock_guard<std::mutex> lk(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemm_v1w_kernel<MG>),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+      if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      configured[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles * S, 1, 1);
+  cfg.blockDim = dim3(v1w_warps(MG) * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemm_v1w_kernel<MG>, p);
+  if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_v1w launch: ") + cudaGetErrorString(e));
+  if ((rc = launch_check("gemm_v1w launch"))) return rc;
+  char buf[64];
+  std::snprintf(buf, sizeof(buf), "int4.gemm.v1w.g%d.t%d.s%d", MG, p.T, S);
+  *label = buf;
+  return WQ_OK;
+}
+
+int launch_v1w(const void* x, const uint8_t* w, void* y, int M, int N, int K, int block_size, int sms,
+               cudaStream_t st, std::string* label) {
+  if (K % 128 || block_size < 128 || M < 1 || M > 64)
+    return fail(WQ_ERR_UNSUPPORTED, "gemm_v1w: needs K % 128 == 0, blocks >= 128 and M <= 64");
+  switch ((M + 7) / 8) {
+    case 1: return launch_v1w_mg<1>(x, w, y, M, N, K, block_size, sms, st, label);
+    case 2: return launch_v1w_mg<2>(x, w, y, M, N, K, block_size, sms, st, label);
+    case 3: return launch_v1w_mg<3>(x, w, y, M, N, K, block_size, sms, st, label);
+    case 4: return launch_v1w_mg<4>(x, w, y, M, N, K, block_size, sms, st, label);
+    case 5: return launch_v1w_mg<5>(x, w, y, M, N, K, block_size, sms, st, label);
+    case 6: return launch_v1w_mg<6>(x, w, y, M, N, K, block_size, sms, st, label);
+    case 7: return launch_v1w_mg<7>(x, w, y, M, N, K, block_size, sms, st, label);
+    default: return launch_v1w_mg<8>(x, w, y, M, N, K, block_size, sms, st, label);
+  }
+}
+
 // Run one format over all M in chunks of at most 8 rows of x.
 template <Fmt F>
 int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_t* scales, const uint8_t* zeros,
@@ -1384,11 +1478,19 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     if constexpr (F == Fmt::Int4) {
       // B200_V1 int4 with blocks of at least 128: the tcgen05 kernel reads the band stream itself
       const bool v1tc_ok = layout == WQ_LAYOUT_B200_V1 && K % 128 == 0 && block_size >= 128 && aligned16(x);
-      // up to 16 rows of x the warp-MMA GEMV in two chunks of 8 is faster (B200,
-      // 14336x4096 M=16: 31.4 against 39.0 us; 4096x14336: 27.1 against 39.0;
-      // 4096x4096: 11.6 against 16.7); from 32 rows the tcgen05 kernel is
-      // (M=32 14336x4096: 39.0 against 62.2)
-      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : M > 16;
+      // 9..24 rows: the warp-MMA GEMM over the stream (B200, M=16 14336x4096
+      // 26.6 us, 4096x14336 24.8, 4096x4096 11.5, against 31.4 / 27.2 / 11.6 for
+      // two GEMV chunks and 39.3 / 39.3 / 17.0 for the tcgen05 kernel); from 25
+      // rows the tcgen05 kernel (M=32 14336x4096: 39.4 against 41.2; M=64: 39.6
+      // against 64.5)
+      const bool want_v1w = force ? std::strcmp(force, "v1w") == 0 : (M >= 9 && M <= 24);
+      if (v1tc_ok && want_v1w) {
+        rc = launch_v1w(x, w, y, M, N, K, block_size, di.sms, st, &label);
+        if (rc) return rc;
+        set_last_kernel(label);
+        return WQ_OK;
+      }
+      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : M > 24;
       if (v1tc_ok && want_v1tc) {
         rc = launch_v1tc(x, w, y, M, N, K, block_size, di.sms, st, &label);
         if (rc) return rc;
