@@ -275,7 +275,7 @@ __device__ __forceinline__ float tc5_dsmem_ld(const float* local, uint32_t rank)
 
 constexpr int kTc5SzAhead = 8;  // int4 scale / zero-point words fetched ahead in registers
 constexpr int kTc5NA = 4;       // A slots (16 KB each)
-constexpr int kTc5Warps = 10;   // 8 dequant / epilogue warps, producer, MMA issuer
+constexpr int kTc5Warps = 11;   // 8 dequant / epilogue warps, producer, two MMA issuers (even / odd stages)
 
 __device__ __forceinline__ void tc5_arrive(uint64_t* bar) {
   asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(smem_u32(bar)) : "memory");
@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
       mbar_init(&a_full[i], F == Fmt::BF16 ? 1 : 8);  // bf16: the producer's TMA fills A directly
       mbar_init(&a_empty[i], 1);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 2);  // one commit per MMA warp
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -383,13 +383,15 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
         }
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 9) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 9 the even stages, warp 10 the odd ones (a second issuing thread
+    // nearly doubles the rate tcgen05.mma instructions reach the tensor core)
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(p.BN, F == Fmt::BF16);
-      int xs = 0, xu = 0;
-      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+      for (int ls = warp - 9; ls < nks && !*abort_flag; ls += 2) {
         const int a = ls & (kTc5NA - 1), au = ls / kTc5NA;
+        const int xs = ls % p.NX, xu = ls / p.NX;
         if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>(au & 1)) ||
             !mbar_wait_bounded(&x_full[xs], static_cast<uint32_t>(xu & 1))) {
           *abort_flag = 1;
@@ -406,12 +408,8 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
           umma_f16(dacc, ad + 2ull * j, bd + 2ull * j, idesc, (ls > 1 || j > 0) ? 1u : 0u);
         umma_commit(&a_empty[a]);
         umma_commit(&x_empty[xs]);
-        if (++xs == p.NX) {
-          xs = 0;
-          ++xu;
-        }
       }
-      umma_commit(done);  // arrives when every MMA issued above has completed
+      umma_commit(done);  // arrives when every MMA this thread issued has completed
     }
   } else {
     // ------------------------------------------------------------ dequant warps

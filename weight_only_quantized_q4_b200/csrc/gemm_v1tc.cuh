@@ -52,7 +52,7 @@ struct V1TCParams {
   int off_x, off_raw, off_rowe, off_bar;  // shared-memory offsets (A slots start at 0)
 };
 
-constexpr int kV1TCWarps = 18;  // 16 dequant / epilogue warps, producer, MMA issuer
+constexpr int kV1TCWarps = 19;  // 16 dequant / epilogue warps, producer, two MMA issuers (even / odd steps)
 constexpr int kV1TCA = 32768;   // bytes of one A slot: 128 rows × 128 k fp16 (two 64-k atoms)
 
 // One int4 B200_V1 tile (16 rows × 128 k) at tp into rows 16·band.. of the A
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
       mbar_init(&a_full[i], 8);
       mbar_init(&a_empty[i], 1);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 2);  // one commit per MMA warp
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -198,11 +198,16 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
         }
       }
     }
-  } else if (warp == 17) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 17) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 17 takes the even steps (accumulator 0), warp 18 the odd ones
+    // (accumulator 1): one thread issuing tcgen05.mma waits about 100 cycles
+    // per instruction on B200, and a second issuing thread nearly doubles the
+    // rate the tensor core receives them (B200: 107 -> 55-66 cycles per MMA).
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(p.BN);
-      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+      const int par = warp - 17;
+      for (int ls = par; ls < nks && !*abort_flag; ls += 2) {
         const int a = ls % p.NA, au = ls / p.NA, xs = ls % p.NX, xu = ls / p.NX;
         if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>(au & 1)) ||
             !mbar_wait_bounded(&x_full[xs], static_cast<uint32_t>(xu & 1))) {
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
         umma_commit(&a_empty[a]);
         umma_commit(&x_empty[xs]);
       }
-      umma_commit(done);  // arrives when every MMA issued above has completed
+      umma_commit(done);  // arrives when every MMA this thread issued has completed
     }
   } else {
     // ------------------------------------------------------------ dequant warps
