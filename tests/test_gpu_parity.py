@@ -623,29 +623,38 @@ def test_full_batched_sampled(fmt, N, K):
 
 # ----------------------------------------------------- tcgen05 over the B200_V1 stream
 
+V1TC_A = [pytest.param("1", id="A_tmem"), pytest.param("0", id="A_smem")]
+
+
 @gpu
+@pytest.mark.parametrize("ta", V1TC_A)
 @pytest.mark.parametrize("M", [9, 16, 33, 64, 128, 200])
 @pytest.mark.parametrize("N,K,bs", [(300, 1024, 128), (37, 4096, 256), (1000, 384, 128), (16, 128, 128)])
-def test_gemm_v1tc_batched(M, N, K, bs, monkeypatch):
-    """The tcgen05 kernel that reads the B200_V1 band stream (forced: below 17
-    rows the default is the chunked warp-MMA GEMV): ragged row tiles (N = 300,
-    37, 1000), an odd number of 128-k steps (K = 384), a single step (K = 128),
+def test_gemm_v1tc_batched(M, N, K, bs, ta, monkeypatch):
+    """The tcgen05 kernel that reads the B200_V1 band stream (forced: below 25
+    rows the default is the warp-MMA GEMM), with the fp16 A rows in tensor
+    memory (default) or in shared memory: ragged row tiles (N = 300, 37,
+    1000), an odd number of 128-k steps (K = 384), a single step (K = 128),
     two batch tiles (M = 200).  Guard bands around every output; two calls
     agree bit for bit."""
     monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
+    monkeypatch.setenv("WQ_V1TC_TA", ta)
     c = Int4Case(M, N, K, bs, True, workload=40, layout=wq.WQ_LAYOUT_B200_V1)
     y = c.run()
     assert ".gemm.v1tc." in wq.last_kernel(), wq.last_kernel()
+    assert (".v1tc.ta." in wq.last_kernel()) == (ta == "1"), wq.last_kernel()
     check(y, c.W(), c.x, f"v1tc M={M} N={N} K={K} bs={bs}")
     assert np.array_equal(y, c.run())
 
 
 @gpu
+@pytest.mark.parametrize("ta", V1TC_A)
 @pytest.mark.parametrize("S", [1, 2, 4, 8])
 @pytest.mark.parametrize("M", [16, 48, 128])
-def test_gemm_v1tc_cluster_split_k(S, M, monkeypatch):
+def test_gemm_v1tc_cluster_split_k(S, M, ta, monkeypatch):
     """K split over a cluster of S CTAs whose fp32 accumulators are added
     through distributed shared memory in rank order."""
+    monkeypatch.setenv("WQ_V1TC_TA", ta)
     monkeypatch.setenv("WQ_V1TC_S", str(S))
     monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
     c = Int4Case(M, 300, 4096, 128, True, workload=41, layout=wq.WQ_LAYOUT_B200_V1)
@@ -654,6 +663,24 @@ def test_gemm_v1tc_cluster_split_k(S, M, monkeypatch):
     assert ".gemm.v1tc." in label and label.endswith(f".s{S}"), label
     check(y, c.W(), c.x, f"v1tc M={M} S={S}")
     assert np.array_equal(y, c.run())
+
+
+@gpu
+@pytest.mark.parametrize("T,ta", [(T, ta) for T in (1, 2, 3, 4) for ta in ("1", "0")] + [(5, "1"), (6, "1")])
+def test_gemm_v1tc_raw_slot_sizes(T, ta, monkeypatch):
+    """Raw slots of T steps per band: odd and even T (the band stride inside a
+    slot is padded to an odd number of 16-byte units when T·1072 is not).
+    With A in shared memory at most 4 steps per raw slot fit at this M."""
+    monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
+    monkeypatch.setenv("WQ_V1TC_TA", ta)
+    monkeypatch.setenv("WQ_V1TC_T", str(T))
+    monkeypatch.setenv("WQ_V1TC_S", "1")  # all 16 steps in one CTA, so T is not cut by the split
+    monkeypatch.setenv("WQ_V1TC_NX", "2")  # a short activation ring leaves room for six steps per raw slot
+    c = Int4Case(40, 260, 2048, 128, True, workload=43, layout=wq.WQ_LAYOUT_B200_V1)
+    y = c.run()
+    label = wq.last_kernel()
+    assert f".t{T}." in label, label
+    check(y, c.W(), c.x, f"v1tc T={T} ta={ta}")
 
 
 @gpu
@@ -668,10 +695,12 @@ def test_gemm_v1tc_forced_split_follows_the_rule(monkeypatch):
 
 
 @gpu
+@pytest.mark.parametrize("ta", V1TC_A)
 @pytest.mark.parametrize("S", [1, 4])
-def test_gemm_v1tc_weights_beyond_fp16_range(S, monkeypatch):
+def test_gemm_v1tc_weights_beyond_fp16_range(S, ta, monkeypatch):
     """Half the rows with scales up to 9000 (|w| up to 135000): formed as
     w·2^-e and rescaled in fp32, every output finite and within tolerance."""
+    monkeypatch.setenv("WQ_V1TC_TA", ta)
     monkeypatch.setenv("WQ_V1TC_S", str(S))
     monkeypatch.setenv("WQ_FORCE_KERNEL", "v1tc")
     M, N, K = 16, 300, 2048

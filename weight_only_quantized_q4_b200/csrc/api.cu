@@ -1200,9 +1200,18 @@ int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, i
   p.tpb = K / 128;
   p.tb = int4_v1_tile_bytes(block_size);
   p.BN = std::min(128, (M + 15) / 16 * 16);
+  // A operand in tensor memory (default) or in shared memory (WQ_V1TC_TA=0)
+  const char* ta_env = std::getenv("WQ_V1TC_TA");
+  const bool ta = !(ta_env && std::atoi(ta_env) == 0);
+  // accumulators: even / odd steps, and NACC = 2 per parity (the MMAs of a
+  // step alternate between them) where the columns allow; WQ_V1TC_NACC=1
+  // keeps one per parity (tuning)
+  const char* nacc_env = std::getenv("WQ_V1TC_NACC");
+  p.NACC = (ta ? 4 * p.BN <= kV1TAColA : 4 * p.BN <= 512) ? 2 : 1;
+  if (nacc_env && std::atoi(nacc_env) == 1) p.NACC = 1;
   int cols = 32;
-  while (cols < 2 * p.BN) cols *= 2;  // two accumulator tiles (even / odd steps)
-  p.tmem_cols = cols;
+  while (cols < 2 * p.NACC * p.BN) cols *= 2;
+  p.tmem_cols = ta ? 512 : cols;      // A slots after the accumulators: 256 + 4 × 64 columns
   const int n_tiles = (p.n_bands + 7) / 8, m_tiles = (M + p.BN - 1) / p.BN;
   // Split K over a cluster of S CTAs (one CTA per SM) while the CTAs still fit
   // one wave; every CTA keeps an even number of 128-k steps.
@@ -1221,46 +1230,59 @@ int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, i
   // steps (one bulk copy of T tiles per band: few, large copies keep the
   // copy engine streaming), row exponents, barriers
   const int x_slot = p.BN * 256;
-  p.NA = 2;
-  p.NX = p.BN <= 32 ? 4 : p.BN <= 64 ? 3 : 2;
+  p.NA = ta ? kV1TANA : 2;
+  // activation slots: with A in TMEM the shared memory has room for a deeper
+  // ring (WQ_V1TC_NX overrides, tuning)
+  p.NX = ta ? (p.BN <= 32 ? 8 : p.BN <= 64 ? 6 : 3) : (p.BN <= 32 ? 4 : p.BN <= 64 ? 3 : 2);
+  if (const char* nx_env = std::getenv("WQ_V1TC_NX")) p.NX = std::max(2, std::min(8, std::atoi(nx_env)));
+  const char* rot_env = std::getenv("WQ_V1TC_ROT");  // 0: every row tile starts at step 0 (A/B runs)
+  p.rotate = !(rot_env && std::atoi(rot_env) == 0);
   const int budget = kSmemPerSm + 4096 - 1024;
-  p.off_x = p.NA * 32768;
+  p.off_a = 0;
+  p.off_x = ta ? 0 : p.NA * 32768;
   p.off_raw = p.off_x + p.NX * x_slot;
   const int fixed = 512 + 16 + 8 * (2 * 4 + 2 * p.NX + 2 * p.NA + 1) + 16;
   const char* t_env = std::getenv("WQ_V1TC_T");  // steps per raw slot (tuning)
   p.NR = 3;
-  p.T = std::min(16, (budget - p.off_raw - fixed) / (p.NR * 8 * p.tb));
+  // (+16: room for the band-stride pad below)
+  p.T = std::min(16, (budget - p.off_raw - fixed) / (p.NR * 8 * p.tb + p.NR * 8 * 16));
   if (p.T < 2) {
     p.NR = 2;
-    p.T = std::min(16, (budget - p.off_raw - fixed) / (p.NR * 8 * p.tb));
+    p.T = std::min(16, (budget - p.off_raw - fixed) / (p.NR * 8 * p.tb + p.NR * 8 * 16));
   }
   if (t_env) p.T = std::max(1, std::min(p.T, std::atoi(t_env)));
   p.T = std::max(1, std::min(p.T, p.nks));
   if (p.T < 1 || p.NR < 2) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: shared memory plan too large");
-  p.off_rowe = static_cast<int>(round16(static_cast<long long>(p.off_raw) + static_cast<long long>(p.NR) * 8 * p.T * p.tb));
+  // bands of a raw slot an odd number of 16-byte units apart (the TMEM-A
+  // dequant reads chunks of four bands at once: eight bank groups)
+  p.band_stride = p.T * p.tb + ((p.T * p.tb / 16) % 2 == 0 ? 16 : 0);
+  p.off_rowe = static_cast<int>(round16(static_cast<long long>(p.off_raw) + static_cast<long long>(p.NR) * 8 * p.band_stride));
   p.off_bar = p.off_rowe + 512;
   const int smem = 1024 + p.off_bar + 8 * (2 * p.NR + 2 * p.NX + 2 * p.NA + 1) + 16;
   if (smem > kSmemPerSm + 4096) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: shared memory plan too large");
-  if (S > 1 && 512 * p.BN > p.off_raw) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: cluster partials do not fit");
+  if (S > 1 && 512 * p.BN > p.off_rowe) return fail(WQ_ERR_UNSUPPORTED, "gemm_v1tc: cluster partials do not fit");
   int rc = encode_2d(&p.tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, 2ull * K, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   {
     static std::mutex mu;
-    static bool configured[64] = {};
+    static bool configured[2][64] = {};
     std::lock_guard<std::mutex> lk(mu);
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemm_v1tc_kernel),
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+    if (dev >= 0 && dev < 64 && !configured[ta][dev]) {
+      cudaError_t e = cudaFuncSetAttribute(
+          ta ? reinterpret_cast<const void*>(&gemm_v1tc_kernel<true>) : reinterpret_cast<const void*>(&gemm_v1tc_kernel<false>),
+          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
       if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-      configured[dev] = true;
+      configured[ta][dev] = true;
     }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles * S, m_tiles, 1);
   cfg.blockDim = dim3(kV1TCWarps * 32, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  // one CTA per SM: a second CTA would wait in tcgen05.alloc for the first
+  // one's 512 columns, and with clusters two such waits could close a cycle
+  cfg.dynamicSmemBytes = ta ? std::max(smem, kSmemPerSm / 2 + 8192) : smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1269,12 +1291,13 @@ int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, i
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = S > 1 ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemm_v1tc_kernel, p);
+  cudaError_t e = ta ? cudaLaunchKernelEx(&cfg, &gemm_v1tc_kernel<true>, p)
+                     : cudaLaunchKernelEx(&cfg, &gemm_v1tc_kernel<false>, p);
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_v1tc launch: ") + cudaGetErrorString(e));
   rc = launch_check("gemm_v1tc launch");
   if (rc) return rc;
   char buf[64];
-  std::snprintf(buf, sizeof(buf), "int4.gemm.v1tc.bn%d.t%d.s%d", p.BN, p.T, S);
+  std::snprintf(buf, sizeof(buf), "int4.gemm.v1tc.%sbn%d.x%d.a%d.t%d.s%d", ta ? "ta." : "", p.BN, p.NX, p.NACC, p.T, S);
   *label = buf;
   return WQ_OK;
 }

@@ -275,7 +275,7 @@ __device__ __forceinline__ float tc5_dsmem_ld(const float* local, uint32_t rank)
 
 constexpr int kTc5SzAhead = 8;  // int4 scale / zero-point words fetched ahead in registers
 constexpr int kTc5NA = 4;       // A slots (16 KB each)
-constexpr int kTc5Warps = 11;   // 8 dequant / epilogue warps, producer, two MMA issuers (even / odd stages)
+constexpr int kTc5Warps = 12;   // 8 dequant / epilogue warps, weight producer, activation producer, two MMA issuers
 
 __device__ __forceinline__ void tc5_arrive(uint64_t* bar) {
   asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(smem_u32(bar)) : "memory");
@@ -344,9 +344,11 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
   const float row_up = __int_as_float((127 + row_e) << 23);  // 2^e
 
   if (warp == 8) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ weight producer
+    // (the activation copies have a warp of their own: a weight copy waits for
+    // its ring slot, which the activation stream should not wait behind)
     if (lane == 0) {
-      int rs = 0, ru = 0, xs = 0, xu = 0;  // slot index and use count of each ring
+      int rs = 0, ru = 0;  // slot index and use count of the raw ring
       for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
         const int gs = s_begin + ls;
         if constexpr (F == Fmt::BF16) {
@@ -371,6 +373,14 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
             ++ru;
           }
         }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      int xs = 0, xu = 0;  // slot index and use count of the activation ring
+      for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
+        const int gs = s_begin + ls;
         if (xu > 0 && !mbar_wait_bounded(&x_empty[xs], static_cast<uint32_t>((xu - 1) & 1))) {
           *abort_flag = 1;
           break;
@@ -383,13 +393,13 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
         }
       }
     }
-  } else if (warp >= 9) {
+  } else if (warp >= 10) {
     // ------------------------------------------------------------ MMA issuers
-    // warp 9 the even stages, warp 10 the odd ones (a second issuing thread
+    // warp 10 the even stages, warp 11 the odd ones (a second issuing thread
     // nearly doubles the rate tcgen05.mma instructions reach the tensor core)
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(p.BN, F == Fmt::BF16);
-      for (int ls = warp - 9; ls < nks && !*abort_flag; ls += 2) {
+      for (int ls = warp - 10; ls < nks && !*abort_flag; ls += 2) {
         const int a = ls & (kTc5NA - 1), au = ls / kTc5NA;
         const int xs = ls % p.NX, xu = ls / p.NX;
         if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>(au & 1)) ||

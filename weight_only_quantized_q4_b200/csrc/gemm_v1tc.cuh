@@ -29,6 +29,18 @@
 // Rows whose weights could pass the fp16 range (15·max|s| > 65504 over the
 // row's blocks) are formed as w·2^-e and their result multiplied by 2^e, as
 // in the 64-k kernel.  Every mbarrier wait is bounded (wq_device.cuh).
+//
+// A in tensor memory (TA).  The fp16 A rows can also skip shared memory: the
+// dequant warps store them into TMEM (tcgen05.st, one row per TMEM lane) and
+// the MMAs read A from there, so shared memory carries only the raw tiles and
+// the activations (in the shared-memory form each weight is written there as
+// fp16 and read back by the tensor core: about 89 KB of shared-memory traffic
+// per 8.6 KB of weights per step).  A warp may only reach its own quarter of
+// the TMEM lanes, so a lane holds one row: TMEM lane L carries tile row
+// v1ta_row(L), chosen so that the 32 rows of a quarter come from four bands
+// and four row indices g, and the 16-byte code chunks a warp reads at once fall
+// into eight different bank groups (band stride in the raw slot an odd number
+// of 16-byte units).  The epilogue maps the accumulator rows back.
 #pragma once
 
 #include "gemm_tc5.cuh"
@@ -48,12 +60,73 @@ struct V1TCParams {
   int S;               // CTAs of a cluster (K slices)
   int nks;             // steps per CTA (tpb / S, even)
   int NA, NR, NX;      // A slots (32 KB), raw slots (8 bands × T tiles), activation slots (BN × 256 B)
+  int NACC;            // accumulators per step parity (1 or 2: the MMAs of a step alternate between them)
+  int rotate;          // 1: each row tile starts its K loop at its own step (spreads the activation reads)
   int T;               // 128-k steps per raw slot: one copy of T consecutive tiles per band
-  int off_x, off_raw, off_rowe, off_bar;  // shared-memory offsets (A slots start at 0)
+  int band_stride;     // bytes between the bands of a raw slot (T·tb, + 16 when that is an even number of 16 B units)
+  int off_a;           // shared-memory A slots (shared-memory A form)
+  int off_x, off_raw, off_rowe, off_bar;  // shared-memory offsets
 };
 
-constexpr int kV1TCWarps = 19;  // 16 dequant / epilogue warps, producer, two MMA issuers (even / odd steps)
+constexpr int kV1TCWarps = 20;  // 16 dequant / epilogue warps, weight producer, activation producer, two MMA issuers
 constexpr int kV1TCA = 32768;   // bytes of one A slot: 128 rows × 128 k fp16 (two 64-k atoms)
+constexpr int kV1TANA = 4;      // TMEM A slots (A in tensor memory): 64 columns each, after 256 accumulator columns
+constexpr int kV1TAColA = 256;  // first TMEM column of the A slots
+
+// Tile row (16·band + 8·half + g) held in TMEM lane L when A lives in tensor
+// memory: quarter Q = L / 32 takes bands 4·(Q / 2) .. + 3 and row indices
+// g = 4·(Q mod 2) .. + 3 of both halves.
+__host__ __device__ __forceinline__ int v1ta_row(int L) {
+  const int Q = L >> 5, i = L & 31;
+  const int band = 4 * (Q >> 1) + (i >> 3), g = 4 * (Q & 1) + ((i >> 1) & 3), half = i & 1;
+  return 16 * band + 8 * half + g;
+}
+
+// tcgen05.mma kind::f16 with A read from tensor memory (a_tmem) and B from a
+// shared-memory descriptor
+__device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane from registers
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// One row's half of a B200_V1 tile (k = 64·gp .. + 63) as 32 fp16 pairs in k
+// order, RN16((q − z)·s): the row's code words sit in the 16-byte chunks of
+// lanes 4g + t (t = 0..3) of the fragment order, word 2·gl + half of chunk t
+// holding k = 64·gp + 32·gl + 8·t .. + 7.
+__device__ __forceinline__ void v1ta_row_half(const uint8_t* tp, int gp, int g, int half, uint32_t zl, uint32_t zh,
+                                              uint32_t s2, uint32_t (&o)[32]) {
+  const uint8_t* cp = tp + gp * 512 + g * 64;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint4 c = *reinterpret_cast<const uint4*>(cp + 16 * t);
+#pragma unroll
+    for (int gl = 0; gl < 2; ++gl) {
+      const uint32_t a = gl == 0 ? (half ? c.y : c.x) : (half ? c.w : c.z), a8 = a >> 8;
+      uint32_t* q = o + 16 * gl + 4 * t;
+      q[0] = hmul2_f(hsub2_f(lop3_or(a, 0x000F000Fu, 0x64006400u), zl), s2);
+      q[1] = hmul2_f(hsub2_f(lop3_or(a, 0x00F000F0u, 0x54005400u), zh), s2);
+      q[2] = hmul2_f(hsub2_f(lop3_or(a8, 0x000F000Fu, 0x64006400u), zl), s2);
+      q[3] = hmul2_f(hsub2_f(lop3_or(a8, 0x00F000F0u, 0x54005400u), zh), s2);
+    }
+  }
+}
 
 // One int4 B200_V1 tile (16 rows × 128 k) at tp into rows 16·band.. of the A
 // slot at ab (two 128-byte-swizzled 64-k atoms).  s2: the two rows' scales as
@@ -107,6 +180,7 @@ __device__ __forceinline__ int v1tc_row_exponent(uint32_t smax) {
   return e;
 }
 
+template <bool TA>
 __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __grid_constant__ V1TCParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,6 +203,12 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
   const int m0 = blockIdx.y * p.BN;
   const int s_begin = static_cast<int>(rank) * p.nks;  // first 128-k step of this CTA
   const int nks = p.nks;
+  // Local step ls covers global step s_begin + (ls + rot) mod nks.  Every CTA
+  // reads the whole activation matrix; started in step, all row tiles would
+  // ask for the same activation slice at once, and those reads queue at the
+  // few L2 slices that hold it (B200: about 3 µs from request to arrival).
+  // Rotating the start by row tile spreads them over all of K.
+  const int rot = p.rotate ? static_cast<int>(static_cast<long long>(tile) * nks / (gridDim.x / p.S)) % nks : 0;
   const int x_slot = p.BN * 256;                        // two 64-k atoms of BN rows
 
   if (warp == 0) {
@@ -160,27 +240,40 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 16) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ weight producer
+    // raw slot r (steps [r·T, r·T + T)): one bulk copy per band of its tiles,
+    // which are contiguous in the band's stream.  A bulk copy can hold its
+    // issuing thread for a while when many bytes are in flight, so the
+    // activation copies have a warp of their own.
     if (lane == 0) {
       const long long band_bytes = static_cast<long long>(p.tpb) * p.tb;
       const int nslots = (nks + p.T - 1) / p.T;
-      int issued = 0;  // raw slots issued so far
-      // raw slot r (steps [r·T, r·T + T)): one copy per band of its tiles, which
-      // are contiguous in the band's stream; issued NR - 1 slots ahead of the
-      // step whose activations are being copied
-      auto issue_raw = [&](int r) {
+      for (int r = 0; r < nslots && !*abort_flag; ++r) {
         const int rs = r % p.NR, ru = r / p.NR;
-        if (ru > 0 && !mbar_wait_bounded(&raw_empty[rs], static_cast<uint32_t>((ru - 1) & 1))) return false;
+        if (ru > 0 && !mbar_wait_bounded(&raw_empty[rs], static_cast<uint32_t>((ru - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
         const int nt = min(p.T, nks - r * p.T);
+        // the slot's steps in local order: global steps g0 .. g0 + n1 - 1, then
+        // (past the end of the CTA's range) steps 0 .. nt - n1 - 1
+        const int g0 = (r * p.T + rot) % nks, n1 = min(nt, nks - g0);
         mbar_arrive_expect_tx(&raw_full[rs], static_cast<uint32_t>(nbt * nt * p.tb));
-        uint8_t* dst = smem + p.off_raw + rs * 8 * p.T * p.tb;
-        for (int i = 0; i < nbt; ++i)
-          bulk_g2s(dst + i * p.T * p.tb, p.w + (b0 + i) * band_bytes + static_cast<long long>(s_begin + r * p.T) * p.tb,
-                   static_cast<uint32_t>(nt * p.tb), &raw_full[rs]);
-        return true;
-      };
+        uint8_t* dst = smem + p.off_raw + rs * 8 * p.band_stride;
+        for (int i = 0; i < nbt; ++i) {
+          const uint8_t* band = p.w + (b0 + i) * band_bytes + static_cast<long long>(s_begin) * p.tb;
+          bulk_g2s(dst + i * p.band_stride, band + static_cast<long long>(g0) * p.tb, static_cast<uint32_t>(n1 * p.tb),
+                   &raw_full[rs]);
+          if (nt > n1)
+            bulk_g2s(dst + i * p.band_stride + n1 * p.tb, band, static_cast<uint32_t>((nt - n1) * p.tb), &raw_full[rs]);
+        }
+      }
+    }
+  } else if (warp == 17) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
       for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
-        const int gs = s_begin + ls;
+        const int gs = s_begin + (ls + rot) % nks;
         const int xs = ls % p.NX, xu = ls / p.NX;
         if (xu > 0 && !mbar_wait_bounded(&x_empty[xs], static_cast<uint32_t>((xu - 1) & 1))) {
           *abort_flag = 1;
@@ -190,23 +283,19 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
         uint8_t* xd = smem + p.off_x + xs * x_slot;
         tma_load_2d(xd, &p.tmap_x, gs * 128, m0, &x_full[xs]);
         tma_load_2d(xd + x_slot / 2, &p.tmap_x, gs * 128 + 64, m0, &x_full[xs]);
-        bool okr = true;
-        while (okr && issued < nslots && issued <= ls / p.T + p.NR - 1) okr = issue_raw(issued++);
-        if (!okr) {
-          *abort_flag = 1;
-          break;
-        }
       }
     }
-  } else if (warp >= 17) {
+  } else if (warp >= 18) {
     // ------------------------------------------------------------ MMA issuers
-    // Warp 17 takes the even steps (accumulator 0), warp 18 the odd ones
-    // (accumulator 1): one thread issuing tcgen05.mma waits about 100 cycles
-    // per instruction on B200, and a second issuing thread nearly doubles the
-    // rate the tensor core receives them (B200: 107 -> 55-66 cycles per MMA).
+    // Warp 18 takes the even steps, warp 19 the odd ones, each into its own
+    // accumulators: one thread issuing tcgen05.mma waits about 100 cycles per
+    // instruction on B200 when each MMA adds into the previous one's result,
+    // and a second issuing thread nearly doubles the rate the tensor core
+    // receives them (B200: 107 -> 55-66 cycles per MMA).  With NACC = 2 the
+    // MMAs of a step also alternate between two accumulators.
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(p.BN);
-      const int par = warp - 17;
+      const int par = warp - 18;
       for (int ls = par; ls < nks && !*abort_flag; ls += 2) {
         const int a = ls % p.NA, au = ls / p.NA, xs = ls % p.NX, xu = ls / p.NX;
         if (!mbar_wait_bounded(&a_full[a], static_cast<uint32_t>(au & 1)) ||
@@ -215,14 +304,26 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
           break;
         }
         tc_fence_after();
-        const uint32_t dacc = tmem + static_cast<uint32_t>((ls & 1) * p.BN);
+        const uint32_t dacc = tmem + static_cast<uint32_t>((ls & 1) * p.NACC * p.BN);
+        const uint32_t dsub = p.NACC > 1 ? static_cast<uint32_t>(p.BN) : 0u;  // second accumulator of the parity
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // the two 64-k atoms of the step
-          const uint64_t ad = umma_smem_desc_sw128(smem_u32(smem + a * kV1TCA + h * 16384));
           const uint64_t bd = umma_smem_desc_sw128(smem_u32(smem + p.off_x + xs * x_slot + h * (x_slot / 2)));
 #pragma unroll
-          for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
-            umma_f16(dacc, ad + 2ull * j, bd + 2ull * j, idesc, (ls > 1 || h > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < 4; ++j) {  // K = 16 per MMA
+            const int q = 4 * h + j;
+            const uint32_t d = dacc + ((q & 1) ? dsub : 0u);
+            // the first MMA into each accumulator (steps 0 and 1) overwrites it
+            const uint32_t accum = (ls > 1 || q >= p.NACC) ? 1u : 0u;
+            if constexpr (TA) {
+              // A slot a: 64 TMEM columns, 16 k (8 columns) per MMA
+              umma_f16_ta(d, tmem + static_cast<uint32_t>(kV1TAColA + 64 * a + 8 * q), bd + 2ull * j, idesc, accum);
+            } else {
+              // advance 32 bytes inside the swizzle atom per MMA
+              const uint64_t ad = umma_smem_desc_sw128(smem_u32(smem + p.off_a + a * kV1TCA + h * 16384));
+              umma_f16(d, ad + 2ull * j, bd + 2ull * j, idesc, accum);
+            }
+          }
         }
         umma_commit(&a_empty[a]);
         umma_commit(&x_empty[xs]);
@@ -289,6 +390,15 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
     asm volatile("bar.sync 1, 512;" ::: "memory");  // the row exponents are in place
     const int e0 = rowe[16 * band + g], e1 = rowe[16 * band + g + 8];
     const float dn0 = __int_as_float((127 - e0) << 23), dn1 = __int_as_float((127 - e1) << 23);
+    // A in tensor memory: this thread's row (TMEM lane 32·(warp mod 4) + lane)
+    // and 64-k half gp of every step of parity par
+    const int ta_q = warp & 3, ta_gp = (warp >> 2) & 1;
+    const int ta_r = v1ta_row(32 * ta_q + lane);
+    const int ta_band = ta_r >> 4, ta_g = ta_r & 7, ta_half = (ta_r >> 3) & 1;
+    const bool ta_have = ta_band < nbt;
+    const int ta_e = rowe[ta_r];
+    const float ta_dn = __int_as_float((127 - ta_e) << 23);
+    const uint32_t ta_col = tmem + (static_cast<uint32_t>(32 * ta_q) << 16) + static_cast<uint32_t>(kV1TAColA + 32 * ta_gp);
     // every dequant warp visits every raw slot (count 16 on its empty barrier)
     // and converts the slot's steps of its parity
     for (int r = 0; r * p.T < nks && !*abort_flag; ++r) {
@@ -304,13 +414,31 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
           *abort_flag = 1;
           break;
         }
-        if (have) {
-          const uint8_t* tp = smem + p.off_raw + (rs * 8 + band) * p.T * p.tb + (ls - r * p.T) * p.tb;
+        if constexpr (TA) {
+          if (au > 0) tc_fence_after();  // the MMAs that read this slot have completed
+          uint32_t o[32];
+          if (ta_have) {
+            const uint8_t* tp = smem + p.off_raw + (rs * 8 + ta_band) * p.band_stride + (ls - r * p.T) * p.tb;
+            uint32_t sv = *reinterpret_cast<const unsigned short*>(tp + 1024 + 2 * (8 * ta_half + ta_g));
+            if (ta_e) sv = __half_as_ushort(__float2half_rn(h16_to_f32(sv) * ta_dn));
+            const uint32_t zw = *reinterpret_cast<const uint32_t*>(tp + 1056 + 4 * ta_half);
+            const uint32_t z = (zw >> (4 * ta_g)) & 15u;
+            v1ta_row_half(tp, ta_gp, ta_g, ta_half, (0x6400u | z) * 0x00010001u, (0x5400u | (z << 4)) * 0x00010001u,
+                          sv * 0x00010001u, o);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+          tmem_st32(ta_col + static_cast<uint32_t>(64 * a), o);
+          tmem_wait_st();
+          tc_fence_before();
+        } else if (have) {
+          const uint8_t* tp = smem + p.off_raw + (rs * 8 + band) * p.band_stride + (ls - r * p.T) * p.tb;
           uint32_t sg = *reinterpret_cast<const unsigned short*>(tp + 1024 + 2 * g);
           uint32_t sg8 = *reinterpret_cast<const unsigned short*>(tp + 1024 + 2 * (g + 8));
           if (e0) sg = __half_as_ushort(__float2half_rn(h16_to_f32(sg) * dn0));
           if (e1) sg8 = __half_as_ushort(__float2half_rn(h16_to_f32(sg8) * dn1));
-          v1tc_tile_to_a(tp, smem + a * kV1TCA, band, lane, sg * 0x00010001u, sg8 * 0x00010001u);
+          v1tc_tile_to_a(tp, smem + p.off_a + a * kV1TCA, band, lane, sg * 0x00010001u, sg8 * 0x00010001u);
           fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         }
         __syncwarp();
@@ -327,23 +455,27 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
   tc_fence_after();
   const int lq = warp & 3, ch = (warp >> 2) & 1;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-  const int trow = lq * 32 + lane;  // tile row this thread reads back
+  const int tlane = lq * 32 + lane;                  // TMEM lane this thread reads back
+  const int trow = TA ? v1ta_row(tlane) : tlane;     // its tile row
   const bool split_cols = p.BN % 32 == 0;
   const int cols_per = split_cols ? p.BN / 2 : p.BN;
   const int c_begin = split_cols ? ch * cols_per : 0;
   const bool reads = warp < 8 && (split_cols || ch == 0);
   const float row_up = __int_as_float((127 + rowe[trow & 127]) << 23);  // 2^e
+  // the accumulators in a fixed order: even steps (NACC of them), then odd steps
+  const int n_acc = (nks > 1 ? 2 : 1) * p.NACC;
   auto acc16 = [&](int c0, float (&v)[16]) {
-    uint32_t r0[16], r1[16];
+    uint32_t r0[16];
     tmem_ld16(lane_base + c0, r0);
-    if (nks > 1) {
-      tmem_ld16(lane_base + p.BN + c0, r1);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = (__uint_as_float(r0[j]) + __uint_as_float(r1[j])) * row_up;
-    } else {
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]);
+    for (int c = 1; c < n_acc; ++c) {
+      tmem_ld16(lane_base + c * p.BN + c0, r0);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]) * row_up;
+      for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r0[j]);
     }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] *= row_up;
   };
   __half* y = reinterpret_cast<__half*>(p.y);
   if (p.S == 1) {
