@@ -1235,8 +1235,6 @@ int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, i
   // ring (WQ_V1TC_NX overrides, tuning)
   p.NX = ta ? (p.BN <= 32 ? 8 : p.BN <= 64 ? 6 : 3) : (p.BN <= 32 ? 4 : p.BN <= 64 ? 3 : 2);
   if (const char* nx_env = std::getenv("WQ_V1TC_NX")) p.NX = std::max(2, std::min(8, std::atoi(nx_env)));
-  const char* rot_env = std::getenv("WQ_V1TC_ROT");  // 0: every row tile starts at step 0 (A/B runs)
-  p.rotate = !(rot_env && std::atoi(rot_env) == 0);
   const int budget = kSmemPerSm + 4096 - 1024;
   p.off_a = 0;
   p.off_x = ta ? 0 : p.NA * 32768;

@@ -61,7 +61,6 @@ struct V1TCParams {
   int nks;             // steps per CTA (tpb / S, even)
   int NA, NR, NX;      // A slots (32 KB), raw slots (8 bands × T tiles), activation slots (BN × 256 B)
   int NACC;            // accumulators per step parity (1 or 2: the MMAs of a step alternate between them)
-  int rotate;          // 1: each row tile starts its K loop at its own step (spreads the activation reads)
   int T;               // 128-k steps per raw slot: one copy of T consecutive tiles per band
   int band_stride;     // bytes between the bands of a raw slot (T·tb, + 16 when that is an even number of 16 B units)
   int off_a;           // shared-memory A slots (shared-memory A form)
@@ -203,12 +202,6 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
   const int m0 = blockIdx.y * p.BN;
   const int s_begin = static_cast<int>(rank) * p.nks;  // first 128-k step of this CTA
   const int nks = p.nks;
-  // Local step ls covers global step s_begin + (ls + rot) mod nks.  Every CTA
-  // reads the whole activation matrix; started in step, all row tiles would
-  // ask for the same activation slice at once, and those reads queue at the
-  // few L2 slices that hold it (B200: about 3 µs from request to arrival).
-  // Rotating the start by row tile spreads them over all of K.
-  const int rot = p.rotate ? static_cast<int>(static_cast<long long>(tile) * nks / (gridDim.x / p.S)) % nks : 0;
   const int x_slot = p.BN * 256;                        // two 64-k atoms of BN rows
 
   if (warp == 0) {
@@ -255,25 +248,18 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
           break;
         }
         const int nt = min(p.T, nks - r * p.T);
-        // the slot's steps in local order: global steps g0 .. g0 + n1 - 1, then
-        // (past the end of the CTA's range) steps 0 .. nt - n1 - 1
-        const int g0 = (r * p.T + rot) % nks, n1 = min(nt, nks - g0);
         mbar_arrive_expect_tx(&raw_full[rs], static_cast<uint32_t>(nbt * nt * p.tb));
         uint8_t* dst = smem + p.off_raw + rs * 8 * p.band_stride;
-        for (int i = 0; i < nbt; ++i) {
-          const uint8_t* band = p.w + (b0 + i) * band_bytes + static_cast<long long>(s_begin) * p.tb;
-          bulk_g2s(dst + i * p.band_stride, band + static_cast<long long>(g0) * p.tb, static_cast<uint32_t>(n1 * p.tb),
-                   &raw_full[rs]);
-          if (nt > n1)
-            bulk_g2s(dst + i * p.band_stride + n1 * p.tb, band, static_cast<uint32_t>((nt - n1) * p.tb), &raw_full[rs]);
-        }
+        for (int i = 0; i < nbt; ++i)
+          bulk_g2s(dst + i * p.band_stride, p.w + (b0 + i) * band_bytes + static_cast<long long>(s_begin + r * p.T) * p.tb,
+                   static_cast<uint32_t>(nt * p.tb), &raw_full[rs]);
       }
     }
   } else if (warp == 17) {
     // ------------------------------------------------------------ activation producer
     if (lane == 0) {
       for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
-        const int gs = s_begin + (ls + rot) % nks;
+        const int gs = s_begin + ls;
         const int xs = ls % p.NX, xu = ls / p.NX;
         if (xu > 0 && !mbar_wait_bounded(&x_empty[xs], static_cast<uint32_t>((xu - 1) & 1))) {
           *abort_flag = 1;
