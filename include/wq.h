@@ -4,8 +4,11 @@
  *
  * Shapes: x is [M, K] row-major, W is logically [N, K], y is [M, N] row-major.
  * M is the decode batch (the GEMV family serves M = 1..8; M >= 9 runs the
- * tensor-core dequant-then-MMA family), N the output features, K the input
- * features.  Every floating-point result is accumulated in fp32.
+ * batched family: for B200_V1 int4 a warp-MMA GEMM over the band stream up to
+ * M = 24 and the tcgen05 dequant-then-MMA kernel beyond, for the canonical
+ * formats the tcgen05 kernel where it applies, else the GEMV in chunks of 8
+ * rows of x), N the output features, K the input features.  Every
+ * floating-point result is accumulated in fp32.
  *
  * Conventions for every entry point below:
  *  - Pointers named *_host are host pointers; every other pointer is a CUDA
@@ -44,8 +47,10 @@
  *    WQ_FORCE_KERNEL (tc | cc | simple | tc5 | v1s | v1r | v1k | v1tc | v1w | mx | mmq) pins a kernel
  *    family (a call that family cannot run returns WQ_ERR_UNSUPPORTED; there
  *    is no silent substitute), WQ_PDL=0 disables programmatic dependent
- *    launch, and WQ_V1_*, WQ_V1R_*, WQ_TC_*, WQ_TC5_S override launch
- *    geometry.
+ *    launch, and WQ_V1_*, WQ_V1R_*, WQ_V1K_*, WQ_V1W_*, WQ_V1TC_*, WQ_TC_*,
+ *    WQ_TC5_S and WQ_MMQ_* override launch geometry (WQ_V1TC_TA=0 keeps the
+ *    batched B200_V1 kernel's fp16 A rows in shared memory instead of tensor
+ *    memory; same results within the tolerance, slower).
  *
  * Weight formats (canonical byte layouts, layout version WQ_LAYOUT_CANONICAL):
  *  - int4 MatMulNBits-style blocks (onnx-genai PR #1000, "What it does": int4
