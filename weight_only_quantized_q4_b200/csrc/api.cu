@@ -1231,10 +1231,13 @@ int launch_v1tc(const void* x, const uint8_t* w, void* y, int M, int N, int K, i
   // copy engine streaming), row exponents, barriers
   const int x_slot = p.BN * 256;
   p.NA = ta ? kV1TANA : 2;
-  // activation slots: with A in TMEM the shared memory has room for a deeper
-  // ring (WQ_V1TC_NX overrides, tuning)
-  p.NX = ta ? (p.BN <= 32 ? 8 : p.BN <= 64 ? 6 : 3) : (p.BN <= 32 ? 4 : p.BN <= 64 ? 3 : 2);
-  if (const char* nx_env = std::getenv("WQ_V1TC_NX")) p.NX = std::max(2, std::min(8, std::atoi(nx_env)));
+  // activation slots: with A in TMEM as many as A slots (an activation slot is
+  // freed by the same commit as its step's A slot: one commit per step, B200
+  // M=32/64/128 14336x4096 25.2/25.9/27.9 us against 25.7/26.4/28.2 with six
+  // activation slots and a commit each); with A in shared memory a ring of
+  // its own (WQ_V1TC_NX overrides, tuning)
+  p.NX = ta ? p.NA : (p.BN <= 32 ? 4 : p.BN <= 64 ? 3 : 2);
+  if (const char* nx_env = std::getenv("WQ_V1TC_NX"); nx_env && !ta) p.NX = std::max(2, std::min(8, std::atoi(nx_env)));
   const int budget = kSmemPerSm + 4096 - 1024;
   p.off_a = 0;
   p.off_x = ta ? 0 : p.NA * 32768;

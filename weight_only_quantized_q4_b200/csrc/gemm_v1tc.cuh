@@ -261,7 +261,11 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
       for (int ls = 0; ls < nks && !*abort_flag; ++ls) {
         const int gs = s_begin + ls;
         const int xs = ls % p.NX, xu = ls / p.NX;
-        if (xu > 0 && !mbar_wait_bounded(&x_empty[xs], static_cast<uint32_t>((xu - 1) & 1))) {
+        // A in TMEM: the activation ring is as deep as the A ring (NX == NA), and
+        // slot xs is free once the MMAs of step ls - NA have completed, which the
+        // A slot's barrier already tracks (one commit per step instead of two)
+        uint64_t* xfree = TA ? a_empty : x_empty;
+        if (xu > 0 && !mbar_wait_bounded(&xfree[xs], static_cast<uint32_t>((xu - 1) & 1))) {
           *abort_flag = 1;
           break;
         }
@@ -312,7 +316,7 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
           }
         }
         umma_commit(&a_empty[a]);
-        umma_commit(&x_empty[xs]);
+        if constexpr (!TA) umma_commit(&x_empty[xs]);
       }
       umma_commit(done);  // arrives when every MMA this thread issued has completed
     }
