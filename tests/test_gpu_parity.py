@@ -365,12 +365,24 @@ def test_gemv_larger_batches(M):
     each_variant(b.run, b.W(), b.X(), f"bf16 M={M}")
 
 
+TC5_A = [pytest.param("1", id="A_tmem"), pytest.param("0", id="A_smem")]
+
+
+def _tc5_a_placement(label, ta, M):
+    """TMEM-A runs for batch tiles of at most 128 columns unless turned off."""
+    assert (".tc5.ta." in label) == (ta == "1" and M <= 128), label
+
+
 @gpu
+@pytest.mark.parametrize("ta", TC5_A)
 @pytest.mark.parametrize("M", [9, 16, 32, 64, 128, 200, 300])
 @pytest.mark.parametrize("fmt", ["int4", "q4k"])
-def test_gemm_tcgen05_batched(M, fmt):
+def test_gemm_tcgen05_batched(M, fmt, ta, monkeypatch):
     """The tcgen05 dequant-then-MMA path (default for M >= 9) on ragged row
-    tiles (N = 300) and batches that span one or two N tiles of the MMA."""
+    tiles (N = 300) and batches that span one or two N tiles of the MMA, with
+    the fp16 A rows in tensor memory (batch tiles up to 128) or in shared
+    memory."""
+    monkeypatch.setenv("WQ_TC5_TA", ta)
     if fmt == "int4":
         c = Int4Case(M, 300, 1024, 128, True, workload=29)
         y = c.run()
@@ -380,6 +392,7 @@ def test_gemm_tcgen05_batched(M, fmt):
         y = c.run(False)
         W, x = c.W(), c.x
     assert ".gemm.tc5." in wq.last_kernel(), wq.last_kernel()
+    _tc5_a_placement(wq.last_kernel(), ta, M)
     check(y, W, x, f"tcgen05 {fmt} M={M}")
 
 
@@ -398,13 +411,15 @@ def test_gemm_tcgen05_bf16(M, N, K):
 
 
 @gpu
+@pytest.mark.parametrize("ta", TC5_A)
 @pytest.mark.parametrize("S", [1, 2, 4, 8])
 @pytest.mark.parametrize("M", [16, 33, 128])
 @pytest.mark.parametrize("fmt", ["int4", "q4k"])
-def test_gemm_tcgen05_cluster_split_k(S, M, fmt, monkeypatch):
+def test_gemm_tcgen05_cluster_split_k(S, M, fmt, ta, monkeypatch):
     """The tcgen05 batched path with K split over a cluster of S CTAs whose fp32
     accumulators are added through distributed shared memory (ragged N tiles,
     batch tiles of 16..128 columns).  Two calls in a row agree bit for bit."""
+    monkeypatch.setenv("WQ_TC5_TA", ta)
     monkeypatch.setenv("WQ_TC5_S", str(S))
     if fmt == "int4":
         c = Int4Case(M, 300, 4096, 128, True, workload=31)
@@ -420,14 +435,16 @@ def test_gemm_tcgen05_cluster_split_k(S, M, fmt, monkeypatch):
 
 
 @gpu
+@pytest.mark.parametrize("ta", TC5_A)
 @pytest.mark.parametrize("S", [1, 4])
 @pytest.mark.parametrize("fmt", ["int4", "q4k"])
-def test_gemm_tcgen05_weights_beyond_fp16_range(fmt, S, monkeypatch):
+def test_gemm_tcgen05_weights_beyond_fp16_range(fmt, S, ta, monkeypatch):
     """Half the rows dequantize beyond the fp16 range (int4 scales up to 9000,
     |w| up to 135000; q4_K d up to 100, |w| up to about 95000) beside ordinary
     rows.  The tcgen05 path forms such rows as w·2^-e and rescales their fp32
     result, so every output stays finite and within the tolerance (small
     activations keep y itself inside fp16)."""
+    monkeypatch.setenv("WQ_TC5_TA", ta)
     monkeypatch.setenv("WQ_TC5_S", str(S))
     M, N, K = 16, 300, 2048
     rng = np.random.default_rng(32)

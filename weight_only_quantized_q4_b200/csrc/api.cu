@@ -1100,10 +1100,14 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   p.zb = zb;
   p.block_shift = block_size > 0 ? ilog2_int(block_size) : 0;
   p.BN = std::min(256, (M + 15) / 16 * 16);
+  // int4 and q4_K with BN <= 128: fp16 A rows in tensor memory (columns 256 ..
+  // 383, after the two accumulator tiles); WQ_TC5_TA=0 keeps them in shared memory
+  const char* ta_env = std::getenv("WQ_TC5_TA");
+  const bool ta = F != Fmt::BF16 && p.BN <= 128 && !(ta_env && std::atoi(ta_env) == 0);
   int cols = 32;
   while (cols < 2 * p.BN) cols *= 2;  // two accumulator tiles (even / odd stages)
-  p.tmem_cols = cols;
-  // shared memory: 4 A slots (16 KB), NX activation slots, NR raw slots, barriers
+  p.tmem_cols = ta ? 512 : cols;
+  // shared memory: 4 A slots (16 KB; none with A in TMEM), NX activation slots, NR raw slots, barriers
   const int x_slot = (p.BN * 128 + 1023) / 1024 * 1024;
   // raw slots of 256 k: int4 128 B per row, q4_K one 144-byte super-block per row
   // (256-byte int4 rows measured no faster on B200)
@@ -1112,8 +1116,9 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   p.raw_bytes = F == Fmt::BF16 ? 0 : 128 * p.raw_pitch;  // bf16 weights go straight into the A slots
   p.NR = F == Fmt::BF16 ? 0 : 3;
   const int budget = kSmemPerSm - 1024 - 1024;
-  p.NX = std::max(2, std::min(8, (budget - kTc5NA * 16384 - p.NR * p.raw_bytes) / x_slot));
-  p.off_x = kTc5NA * 16384;
+  const int a_bytes = ta ? 0 : kTc5NA * 16384;
+  p.NX = std::max(2, std::min(8, (budget - a_bytes - p.NR * p.raw_bytes) / x_slot));
+  p.off_x = a_bytes;
   p.off_raw = p.off_x + p.NX * x_slot;
   p.off_bar = (p.off_raw + p.NR * p.raw_bytes + 127) / 128 * 128;
   const int smem = 1024 + p.off_bar + (2 * p.NR + 2 * p.NX + 2 * kTc5NA + 1) * 8 + 16;
@@ -1150,23 +1155,27 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
                  M, 2ull * K, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   static std::mutex mu;
-  static bool configured[3][64] = {};
+  static bool configured[3][2][64] = {};
   const int fi = F == Fmt::Int4 ? 0 : F == Fmt::Q4K ? 1 : 2;
+  constexpr bool kTA = F != Fmt::BF16;  // (bf16 weights are the A operand as stored: never TA)
+  const void* fn = ta ? reinterpret_cast<const void*>(&gemm_tc5_kernel<F, kTA>)
+                      : reinterpret_cast<const void*>(&gemm_tc5_kernel<F, false>);
   {
     std::lock_guard<std::mutex> lk(mu);
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !configured[fi][dev]) {
-      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&gemm_tc5_kernel<F>),
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
+    if (dev >= 0 && dev < 64 && !configured[fi][ta][dev]) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm + 4096);
       if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-      configured[fi][dev] = true;
+      configured[fi][ta][dev] = true;
     }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles * S, m_tiles, 1);
   cfg.blockDim = dim3(kTc5Warps * 32, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  // with A in TMEM a CTA holds all 512 TMEM columns: one CTA per SM (a second
+  // one would wait in tcgen05.alloc, and with clusters two waits could cycle)
+  cfg.dynamicSmemBytes = ta ? std::max(smem, kSmemPerSm / 2 + 8192) : smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1175,13 +1184,14 @@ int launch_tc5(const void* x, const uint8_t* w, const uint8_t* scales, const uin
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = S > 1 ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, &gemm_tc5_kernel<F>, p);
+  cudaError_t e = ta ? cudaLaunchKernelEx(&cfg, &gemm_tc5_kernel<F, kTA>, p)
+                     : cudaLaunchKernelEx(&cfg, &gemm_tc5_kernel<F, false>, p);
   if (e != cudaSuccess) return fail(WQ_ERR_CUDA, std::string("gemm_tc5 launch: ") + cudaGetErrorString(e));
   rc = launch_check("gemm_tc5 launch");
   if (rc) return rc;
   char buf[64];
-  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.bn%d.s%d", F == Fmt::Int4 ? "int4" : F == Fmt::Q4K ? "q4k" : "bf16",
-                p.BN, S);
+  std::snprintf(buf, sizeof(buf), "%s.gemm.tc5.%sbn%d.s%d", F == Fmt::Int4 ? "int4" : F == Fmt::Q4K ? "q4k" : "bf16",
+                ta ? "ta." : "", p.BN, S);
   *label = buf;
   return WQ_OK;
 }

@@ -93,6 +93,39 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.mma kind::f16 with A read from tensor memory (a_tmem) and B from a
+// shared-memory descriptor
+__device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane from registers
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// 16 consecutive TMEM columns of this thread's lane from registers
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lop3_or(uint32_t v, uint32_t mask, uint32_t magic) {
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(magic));  // (v & mask) | magic
@@ -289,7 +322,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-template <Fmt F>
+// TA (int4, q4_K with BN <= 128): the dequant threads store their fp16 A rows
+// into tensor memory (tcgen05.st; a thread's weight row is its TMEM lane) and
+// the MMAs read A from there, instead of a 128-byte-swizzled shared-memory
+// tile that the tensor core reads back.
+constexpr int kTc5TAColA = 256;  // first TMEM column of the A slots (4 × 32 columns)
+
+template <Fmt F, bool TA = false>
 __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __grid_constant__ TC5Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
@@ -408,14 +447,22 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
           break;
         }
         tc_fence_after();
-        const uint64_t ad = umma_smem_desc_sw128(smem_u32(smem + a * 16384));
         const uint64_t bd = umma_smem_desc_sw128(smem_u32(smem + p.off_x + xs * ((x_bytes + 1023) & ~1023)));
         // even and odd stages accumulate into two TMEM tiles (columns [0, BN) and
         // [BN, 2BN)), so consecutive stages' MMAs do not wait for each other
         const uint32_t dacc = tmem + static_cast<uint32_t>((ls & 1) * p.BN);
+        if constexpr (TA) {
+          // A slot a: 32 TMEM columns (64 k), 8 columns per MMA
+          const uint32_t at = tmem + static_cast<uint32_t>(kTc5TAColA + 32 * a);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
-          umma_f16(dacc, ad + 2ull * j, bd + 2ull * j, idesc, (ls > 1 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < 4; ++j)
+            umma_f16_ta(dacc, at + 8u * j, bd + 2ull * j, idesc, (ls > 1 || j > 0) ? 1u : 0u);
+        } else {
+          const uint64_t ad = umma_smem_desc_sw128(smem_u32(smem + a * 16384));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
+            umma_f16(dacc, ad + 2ull * j, bd + 2ull * j, idesc, (ls > 1 || j > 0) ? 1u : 0u);
+        }
         umma_commit(&a_empty[a]);
         umma_commit(&x_empty[xs]);
       }
@@ -465,11 +512,22 @@ __global__ void __launch_bounds__(kTc5Warps * 32, 1) gemm_tc5_kernel(const __gri
                                               : rrow + 16 + 32 * (ls & 3);
         uint32_t o[16];
         if constexpr (F != Fmt::BF16) dequant_stage<F>(s_begin + ls, h, codes, rrow, sz, down, o);
-        uint8_t* at = smem + a * 16384;
+        if constexpr (TA) {
+          // row rl is TMEM lane rl (warp w reaches lanes 32·(w mod 4) ..); k = 32·h .. + 31 of the stage
+          if (au > 0) tc_fence_after();  // the MMAs that read this slot have completed
+          tmem_st16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                        static_cast<uint32_t>(kTc5TAColA + 32 * a + 16 * h),
+                    o);
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+          uint8_t* at = smem + a * 16384;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(at + sw128(rl, 4 * h + c)) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(at + sw128(rl, 4 * h + c)) =
+                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        }
         __syncwarp();
         if (lane == 0) tc5_arrive(&a_full[a]);
         if ((ls & (p.spr - 1)) == p.spr - 1) {  // every stage of the raw slot is dequantized
