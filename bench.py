@@ -318,11 +318,18 @@ def _peaks():
 
 
 def _kernel_src_hash() -> str:
+    """Hash of the kernel sources the committed DRAM counters must match: every
+    file under csrc/ with its // comments and trailing blanks removed (a
+    comment edit does not change the code the counters were taken on)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_quantized_q4_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        path = os.path.join(csrc, name)
+        if not os.path.isfile(path):
+            continue
+        with open(path, encoding="utf-8") as f:
+            lines = [ln.split("//", 1)[0].rstrip() for ln in f]
+        h.update(name.encode() + "\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,17 +7,21 @@
 // their fp32 accumulators through distributed shared memory (fixed rank
 // order).  Warp-specialized pipeline over 64-k stages, with full / empty
 // mbarrier rings and no block-wide synchronisation in the main loop:
-//   * producer warp: 2-D TMA copies (tensor maps, no multicast) of the raw
-//     weight bytes, 128 rows × 256 k per copy (int4: 128 B per row; q4_K: one
-//     144-byte super-block per row), and of the BN × 64 activation slice,
+//   * weight producer warp: 2-D TMA copies (tensor maps, no multicast) of the
+//     raw weight bytes, 128 rows × 256 k per copy (int4: 128 B per row; q4_K:
+//     one 144-byte super-block per row);
+//   * activation producer warp: the BN × 64 activation slice per stage,
 //     128-byte swizzled so it lands in the UMMA K-major layout;
 //   * eight dequant warps (two threads per weight row, 32 k each) turn the raw
-//     bytes into a 128-byte-swizzled fp16 A tile in natural k order: int4 as
-//     RN16((q - z)·s) (q - z exact via magic-number codes, one rounding of the
-//     exact product), q4_K as RN16(d·sc·q - dmin·m) from the exact fp32 value;
-//   * one MMA warp issues four tcgen05.mma (K = 16 each) into an fp32 TMEM
-//     accumulator of 128 lanes × BN columns and commits them to the mbarriers
-//     that free the A and activation slots.
+//     bytes into fp16 A rows in natural k order: int4 as RN16((q - z)·s)
+//     (q - z exact via magic-number codes, one rounding of the exact product),
+//     q4_K as RN16(d·sc·q - dmin·m) from the exact fp32 value.  With batch
+//     tiles of at most 128 columns a thread stores its row's 32 k into tensor
+//     memory (its row is its TMEM lane) and the MMAs read A from there;
+//     otherwise the rows go to a 128-byte-swizzled shared-memory tile;
+//   * two MMA warps (even / odd stages) issue four tcgen05.mma (K = 16 each)
+//     per stage into fp32 TMEM accumulators of 128 lanes × BN columns and
+//     commit them to the mbarriers that free the A and activation slots.
 // The epilogue reads the accumulator with tcgen05.ld (warps w and w + 4 share
 // TMEM lanes 32(w mod 4).. and split the columns) and stores fp16 y.  Weights
 // are rounded to fp16 once before the MMA (error <= 2^-11 relative per weight,

@@ -11,36 +11,45 @@
 // K; the S CTAs of a cluster share the rows, split K and add their fp32
 // accumulators through distributed shared memory in rank order.  The CTA's
 // stream is consumed one 128-k step at a time (eight tiles, one per band):
-//   * producer warp: one bulk copy per band and step (the tiles of a band are
-//     contiguous in the stream, so no tensor map is needed for the weights),
-//     and two TMA copies of the BN × 128 activation slice, 128-byte swizzled
-//     into the UMMA K-major layout (no multicast);
-//   * sixteen dequant warps: warp w turns the tile of band w mod 8 of every
-//     step of parity w / 8 into fp16 A rows: (q - z) exactly through
-//     magic-number codes, times s in one fp16 rounding (as the 64-k kernel
-//     does).  The tile's codes are in warp-MMA fragment order, so a lane holds
-//     8 consecutive k of two rows per 32-bit word and writes them as one
-//     16-byte chunk of the swizzled A tile; lanes with odd row index take the
-//     two words of a pair in the opposite order, so the eight lanes of a
-//     quarter-warp always write eight different bank groups;
-//   * MMA warp: eight tcgen05.mma (K = 16) per step into one of two fp32 TMEM
-//     accumulators (even / odd steps), each commit freeing the step's A and
-//     activation slots.
+//   * weight producer warp: one bulk copy per band and raw slot of T steps
+//     (the tiles of a band are contiguous in the stream, so no tensor map is
+//     needed for the weights);
+//   * activation producer warp: two TMA copies of the BN × 128 activation
+//     slice per step, 128-byte swizzled into the UMMA K-major layout (no
+//     multicast).  A bulk copy can hold its issuing thread for about a
+//     microsecond when many bytes are in flight, so the two streams do not
+//     share a thread;
+//   * sixteen dequant warps turn the tiles into fp16 A rows: (q - z) exactly
+//     through magic-number codes, times s in one fp16 rounding (as the 64-k
+//     kernel does);
+//   * two MMA warps (even / odd steps): eight tcgen05.mma (K = 16) per step,
+//     each warp into its own fp32 TMEM accumulators, alternating between two
+//     per step where the columns allow.
 // Rows whose weights could pass the fp16 range (15·max|s| > 65504 over the
 // row's blocks) are formed as w·2^-e and their result multiplied by 2^e, as
 // in the 64-k kernel.  Every mbarrier wait is bounded (wq_device.cuh).
 //
-// A in tensor memory (TA).  The fp16 A rows can also skip shared memory: the
-// dequant warps store them into TMEM (tcgen05.st, one row per TMEM lane) and
-// the MMAs read A from there, so shared memory carries only the raw tiles and
-// the activations (in the shared-memory form each weight is written there as
-// fp16 and read back by the tensor core: about 89 KB of shared-memory traffic
-// per 8.6 KB of weights per step).  A warp may only reach its own quarter of
-// the TMEM lanes, so a lane holds one row: TMEM lane L carries tile row
-// v1ta_row(L), chosen so that the 32 rows of a quarter come from four bands
-// and four row indices g, and the 16-byte code chunks a warp reads at once fall
-// into eight different bank groups (band stride in the raw slot an odd number
-// of 16-byte units).  The epilogue maps the accumulator rows back.
+// A in tensor memory (TA, the default).  The dequant warps store the fp16 A
+// rows into TMEM (tcgen05.st, one row per TMEM lane) and the MMAs read A from
+// there, so shared memory carries only the raw tiles and the activations.  A
+// warp may only reach its own quarter of the TMEM lanes, so a thread holds one
+// row and one 64-k half of a step: TMEM lane L carries tile row v1ta_row(L),
+// chosen so that the 32 rows of a quarter come from four bands and four row
+// indices g, and the 16-byte code chunks a warp reads at once fall into eight
+// different bank groups (band stride in the raw slot an odd number of 16-byte
+// units).  The epilogue maps the accumulator rows back.  One commit per step
+// frees both the step's A slot and its activation slot (the activation ring is
+// as deep as the A ring).
+//
+// A in shared memory (WQ_V1TC_TA=0).  Warp w turns the tile of band w mod 8 of
+// every step of parity w / 8 into a 128-byte-swizzled fp16 A tile.  The
+// tile's codes are in warp-MMA fragment order, so a lane holds 8 consecutive k
+// of two rows per 32-bit word and writes them as one 16-byte chunk; lanes with
+// odd row index take the two words of a pair in the opposite order, so the
+// eight lanes of a quarter-warp always write eight different bank groups.
+// Each weight then crosses shared memory twice as fp16 (about 89 KB of
+// shared-memory traffic per 8.6 KB of weights per step), and the activation
+// ring has a commit of its own.
 #pragma once
 
 #include "gemm_tc5.cuh"
