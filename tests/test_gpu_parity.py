@@ -758,8 +758,10 @@ def test_full_batched_v1tc_sampled(N, K):
         wq.gemv_int4_blockwise(dev(x), g.t, None, None, gy.t, M, N, K, 128, layout=wq.WQ_LAYOUT_B200_V1)
         torch.cuda.synchronize()
         label = wq.last_kernel()
-        # up to 24 rows the warp-MMA GEMM over the stream is the default, from 25 the tcgen05 kernel
-        assert (".gemm.v1w." in label) if M <= 24 else (".gemm.v1tc." in label), label
+        # the tcgen05 kernel from 25 rows, and from 9 when its 128-row tiles fill
+        # the GPU without a K split (2·ceil(N/128) > SMs); else the warp-MMA GEMM
+        fills = 2 * -(-N // 128) > torch.cuda.get_device_properties(0).multi_processor_count
+        assert (".gemm.v1tc." in label) if (M > 24 or fills) else (".gemm.v1w." in label), label
         gy.check(f"v1tc full {N}x{K} M={M}")
         y = gy.t.cpu().numpy().astype(np.float64)
         check(y[:, rows], Wr, x, f"v1tc full {N}x{K} M={M} [{label}]")

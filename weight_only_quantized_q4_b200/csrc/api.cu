@@ -1512,19 +1512,21 @@ int run_gemv(const char* fmt_name, const void* x, const uint8_t* w, const uint8_
     if constexpr (F == Fmt::Int4) {
       // B200_V1 int4 with blocks of at least 128: the tcgen05 kernel reads the band stream itself
       const bool v1tc_ok = layout == WQ_LAYOUT_B200_V1 && K % 128 == 0 && block_size >= 128 && aligned16(x);
-      // 9..24 rows: the warp-MMA GEMM over the stream (B200, M=16 14336x4096
-      // 26.6 us, 4096x14336 24.8, 4096x4096 11.5, against 31.4 / 27.2 / 11.6 for
-      // two GEMV chunks and 39.3 / 39.3 / 17.0 for the tcgen05 kernel); from 25
-      // rows the tcgen05 kernel (M=32 14336x4096: 39.4 against 41.2; M=64: 39.6
-      // against 64.5)
-      const bool want_v1w = force ? std::strcmp(force, "v1w") == 0 : (M >= 9 && M <= 24);
+      // The tcgen05 kernel from 25 rows, and from 9 rows when its 128-row tiles
+      // alone fill the GPU (no K split); otherwise the warp-MMA GEMM over the
+      // stream up to 24 rows.  B200, M=16 / 24: 14336x4096 v1tc 25.7 / 25.6 us
+      // against v1w 26.6 / 32.4, 32000x4096 50.4 / 50.3 against 53.1 / 64.5;
+      // 4096x14336 (K split) v1w 25.1 / 27.5 against 26.9 / 29.4, 4096x4096
+      // 11.6 / 13.1 against 13.9 / 16.4.  M=64 14336x4096: v1tc 25.9, v1w 64.5.
+      const bool v1tc_fills = ((N + 127) / 128) * ((M + 127) / 128) * 2 > di.sms;
+      const bool want_v1w = force ? std::strcmp(force, "v1w") == 0 : (M >= 9 && M <= 24 && !v1tc_fills);
       if (v1tc_ok && want_v1w) {
         rc = launch_v1w(x, w, y, M, N, K, block_size, di.sms, st, &label);
         if (rc) return rc;
         set_last_kernel(label);
         return WQ_OK;
       }
-      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : M > 24;
+      const bool want_v1tc = force ? std::strcmp(force, "v1tc") == 0 : (M > 24 || (M >= 9 && v1tc_fills));
       if (v1tc_ok && want_v1tc) {
         rc = launch_v1tc(x, w, y, M, N, K, block_size, di.sms, st, &label);
         if (rc) return rc;
