@@ -4,10 +4,11 @@
  *
  * Shapes: x is [M, K] row-major, W is logically [N, K], y is [M, N] row-major.
  * M is the decode batch (the GEMV family serves M = 1..8; M >= 9 runs the
- * batched family: for B200_V1 int4 a warp-MMA GEMM over the band stream up to
- * M = 24 and the tcgen05 dequant-then-MMA kernel beyond, for the canonical
- * formats the tcgen05 kernel where it applies, else the GEMV in chunks of 8
- * rows of x), N the output features, K the input features.  Every
+ * batched family: for B200_V1 int4 the tcgen05 dequant-then-MMA kernel from
+ * M = 25, and from M = 9 when its 128-row tiles alone fill the GPU, else a
+ * warp-MMA GEMM over the band stream; for the canonical formats the tcgen05
+ * kernel where it applies, else the GEMV in chunks of 8 rows of x), N the
+ * output features, K the input features.  Every
  * floating-point result is accumulated in fp32.
  *
  * Conventions for every entry point below:
