@@ -263,11 +263,11 @@ __global__ void __launch_bounds__(kV1TCWarps * 32, 1) gemm_v1tc_kernel(const __g
   } else if (warp >= 18) {
     // ------------------------------------------------------------ MMA issuers
     // Warp 18 takes the even steps, warp 19 the odd ones, each into its own
-    // accumulators: one thread issuing tcgen05.mma waits about 100 cycles per
-    // instruction on B200 when each MMA adds into the previous one's result,
-    // and a second issuing thread nearly doubles the rate the tensor core
-    // receives them (B200: 107 -> 55-66 cycles per MMA).  With NACC = 2 the
-    // MMAs of a step also alternate between two accumulators.
+    // accumulators: on B200 one issuing thread is held about 100 cycles per
+    // tcgen05.mma at these N (16 to 128), and a second issuing thread nearly
+    // doubles the rate the tensor core receives them (107 -> 55-66 cycles per
+    // MMA in a microbenchmark).  With NACC = 2 the MMAs of a step also
+    // alternate between two accumulators (no measurable effect on B200).
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(p.BN);
       const int par = warp - 18;
