@@ -49,9 +49,9 @@
  *    family (a call that family cannot run returns WQ_ERR_UNSUPPORTED; there
  *    is no silent substitute), WQ_PDL=0 disables programmatic dependent
  *    launch, and WQ_V1_*, WQ_V1R_*, WQ_V1K_*, WQ_V1W_*, WQ_V1TC_*, WQ_TC_*,
- *    WQ_TC5_S and WQ_MMQ_* override launch geometry (WQ_V1TC_TA=0 keeps the
- *    batched B200_V1 kernel's fp16 A rows in shared memory instead of tensor
- *    memory; same results within the tolerance, slower).
+ *    WQ_TC5_S, WQ_TC5_TA and WQ_MMQ_* override launch geometry (WQ_V1TC_TA=0 and
+ *    WQ_TC5_TA=0 keep the tcgen05 kernels' fp16 A rows in shared memory
+ *    instead of tensor memory; same results within the tolerance, slower).
  *
  * Weight formats (canonical byte layouts, layout version WQ_LAYOUT_CANONICAL):
  *  - int4 MatMulNBits-style blocks (onnx-genai PR #1000, "What it does": int4
